@@ -1,0 +1,203 @@
+/*
+ * aqua.h -- C ABI of the B200 (sm_100a) library for AQUA's online attention step.
+ *
+ * AQUA (Attention via QUery mAgnitudes, arXiv 2509.11155): an orthogonal d x d
+ * projection P is computed once offline from an SVD of calibration queries and
+ * keys; online, every query and key is projected (q~ = qP, k~ = kP), each query
+ * head keeps the k dimensions where |q~| is largest (ties to the lower index),
+ * scores are computed on those dimensions only (scaled by 1/sqrt(d)), followed
+ * by softmax and the weighted sum of the unprojected values.  Sources: the
+ * paper's abstract; edgentiq blog "How AQUA Works: A Two-Phase Approach" and
+ * "AQUA-Memory: Dual Savings" (statically truncated cache); H2O eviction is
+ * named in the abstract ("synergistically accelerate existing token eviction
+ * methods like H2O").
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise, owned by
+ *     the caller, 16-byte aligned, dense row-major in the layout given.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; 0 = legacy
+ *     default stream).  No entry point allocates or frees device memory and no
+ *     entry point synchronises the stream.  Scratch space is caller-provided
+ *     (`workspace`, size from the matching *_workspace_size call).
+ *   - Return value: AQUA_OK or a negative status.  On a negative status nothing
+ *     was enqueued (argument errors are detected on the host before any launch),
+ *     except AQUA_ERR_CUDA, which reports a failed launch.  aqua_last_error()
+ *     returns a thread-local message describing the last failure.
+ *   - Device-side waits are bounded (about 2 s); a wait that runs out records
+ *     AQUA_ERR_TIMEOUT in the cache's status word (read by aqua_status) and the
+ *     kernel returns early instead of hanging.
+ *   - head_dim d must be 128.
+ */
+#ifndef AQUA_H_
+#define AQUA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AQUA_API __attribute__((visibility("default")))
+#else
+#define AQUA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* aqua_stream_t; /* identical to cudaStream_t */
+
+enum aqua_status_code {
+  AQUA_OK = 0,
+  AQUA_ERR_ARG = -1,         /* bad argument (null pointer, size out of range, misalignment) */
+  AQUA_ERR_UNSUPPORTED = -2, /* shape or dtype this build does not implement */
+  AQUA_ERR_WORKSPACE = -3,   /* workspace smaller than the *_workspace_size result */
+  AQUA_ERR_CUDA = -4,        /* a CUDA call or launch failed */
+  AQUA_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out (reported by aqua_status) */
+};
+
+enum aqua_dtype { AQUA_F32 = 0, AQUA_BF16 = 1 };
+
+/* Number of int32 control words the cache's `ctrl` buffer must hold. */
+#define AQUA_CTRL_WORDS 16
+
+/*
+ * The KV cache descriptor.  The struct itself is host memory owned by the
+ * caller; the buffers it points to are device memory owned by the caller.
+ *
+ *   k_proj  [B][Hkv][d_store][Tcap]  dtype  projected keys k~ = kP, DIMENSION-MAJOR:
+ *                                           row j of (b, g) holds dimension j of
+ *                                           every cached token, contiguous over
+ *                                           tokens.  d_store = m < d keeps only the
+ *                                           first m projected dimensions
+ *                                           (AQUA-Memory static truncation).
+ *   v       [B][Hkv][Tcap][d]        dtype  unprojected values, token-major.
+ *   len     [B]                      int32  tokens (slots) in use per sequence.
+ *   n_abs   [B]                      int32  tokens ever appended per sequence (the
+ *                                           absolute position of the next token);
+ *                                           nullable unless pos != NULL.
+ *   pos     [B][Hkv][Tcap]           int32  nullable; absolute position held by each
+ *                                           slot (required for H2O eviction).
+ *   score   [B][Hkv][Tcap]           f32    nullable; H2O cumulative attention score
+ *                                           of each slot.
+ *   ctrl    [AQUA_CTRL_WORDS]        int32  control words; must be zero when the
+ *                                           cache is created; the library leaves
+ *                                           them zero except the sticky status
+ *                                           word read by aqua_status.
+ *   max_len  host int: an upper bound of every len[b]; aqua_project_keys adds L,
+ *            aqua_h2o_update lowers it to the budget.
+ *   Tcap must be a multiple of 16; dtype is AQUA_BF16 or AQUA_F32 for both k_proj and v.
+ */
+typedef struct aqua_cache {
+  void* k_proj;
+  void* v;
+  int32_t* len;
+  int32_t* n_abs;
+  int32_t* pos;
+  float* score;
+  int32_t* ctrl;
+  int B, Hkv, d, d_store, Tcap;
+  int max_len;
+  int dtype;
+} aqua_cache;
+
+/* Thread-local text of the last failure on this host thread ("" if none). */
+AQUA_API const char* aqua_last_error(void);
+
+/* Library ABI version (increments when a signature changes). */
+AQUA_API int aqua_version(void);
+
+/*
+ * Reads and clears the sticky device status word of `cache` (synchronises
+ * `stream`).  *status_out receives AQUA_OK or the first device-side error
+ * (AQUA_ERR_TIMEOUT).  Returns AQUA_OK unless the copy itself failed.
+ */
+AQUA_API int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream);
+
+/*
+ * Offline calibration (abstract: "a universal, language agnostic projection
+ * matrix via SVD on a calibration dataset"; edgentiq, "Offline Projection
+ * Computation").  X [n][d] f32 stacks calibration queries and keys (not
+ * centred).  Writes P [d][d] f32 whose COLUMNS are the right singular vectors
+ * of X ordered by descending singular value, and sigma [d] f32.  Each column's
+ * largest-magnitude entry is made positive.  Computed on the GPU: the Gram
+ * matrix X^T X in f64, then cyclic Jacobi eigen-decomposition in f64.
+ * Requires 1 <= n, d == 128.
+ */
+AQUA_API size_t aqua_calibrate_workspace_size(int n, int d);
+AQUA_API int aqua_calibrate(const float* X, int n, int d, float* P_out, float* sigma_out,
+                   void* workspace, size_t workspace_bytes, aqua_stream_t stream);
+
+/*
+ * Key projection and append (abstract: "project query and key vectors";
+ * edgentiq, "Online Inference").  For every sequence b and new token l < L:
+ * k~ = k_new[b][l][g] . P[g] is computed in f32, its first d_store dimensions
+ * are rounded to the cache dtype (bf16: round-to-nearest-even) and written into
+ * slot len[b] + l of k_proj (dimension-major); v_new is copied into the same
+ * slot of v.  If pos/score are present the slot's position is n_abs[b] + l and
+ * its score 0.  Afterwards len[b] += L and n_abs[b] += L on the device, and
+ * cache->max_len += L on the host.
+ *   k_new, v_new  [B][L][Hkv][d]  cache dtype
+ *   P             [Hkv][d][d]     f32, q~ = q P (row vector times P)
+ * Errors: AQUA_ERR_ARG if cache->max_len + L > Tcap or L < 1.
+ */
+AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void* v_new, const float* P,
+                      int L, aqua_stream_t stream);
+
+/*
+ * One decode step of AQUA attention for every sequence and query head, over
+ * the len[b] cached tokens (the step's own key must already be appended).
+ *   q          [B][Hq][d]  cache dtype; query head h uses KV head h / (Hq/Hkv)
+ *   P          [Hkv][d][d] f32
+ *   k          dimensions kept per query head, 1 <= k <= d_store
+ *   scale      score scale; <= 0 selects 1/sqrt(d) (d = full head dim)
+ *   out        [B][Hq][d]  out_dtype (AQUA_F32 or AQUA_BF16, RNE)
+ *   sel_out    nullable [B][Hq][k] int32: selected dimensions, ascending
+ *   qproj_out  nullable [B][Hq][d] f32: the projected query q~ the selection used
+ *   scores_out nullable [B][Hq][Tcap] f32: score of every cached slot (scaled)
+ *   lse_out    nullable [B][Hq] f32: log-sum-exp of the scores
+ * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4}.  A sequence with
+ * len[b] = 0 gets a zero output and lse = -inf.
+ */
+AQUA_API size_t aqua_decode_workspace_size(const aqua_cache* cache, int Hq);
+AQUA_API int aqua_decode_attn(const aqua_cache* cache, const void* q, const float* P, int Hq, int k,
+                     float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out,
+                     float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
+                     aqua_stream_t stream);
+
+/*
+ * Causal AQUA attention for a chunk of L prompt tokens at absolute positions
+ * pos0 .. pos0+L-1 of every sequence (their keys must already be appended, so
+ * len[b] >= pos0 + L).  Row i of sequence b attends to slots 0 .. pos0+i; each
+ * (row, head) selects its own k dimensions; the dimension-masked Q K~^T and
+ * P V run on the tensor cores.
+ *   q    [B][L][Hq][d] cache dtype (bf16 only)
+ *   out  [B][L][Hq][d] out_dtype
+ *   sel_out nullable [B][L][Hq][k] int32
+ */
+AQUA_API size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L);
+AQUA_API int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, const float* P,
+                      int Hq, int k, float scale, void* out, int out_dtype, int32_t* sel_out,
+                      void* workspace, size_t workspace_bytes, aqua_stream_t stream);
+
+/*
+ * H2O heavy-hitter update after a decode step (abstract: AQUA accelerates
+ * token eviction methods like H2O).  Reading of the rule: for every (b, KV
+ * head g) and slot t < len[b], score[t] += sum over the group's query heads h
+ * of exp(scores[b][h][t] - lse[b][h]) (the AQUA softmax probabilities from
+ * aqua_decode_attn).  Then, if len[b] > budget, exactly one slot is evicted
+ * per (b, g): the lowest score among slots whose position is at most
+ * newest - recent (newest = n_abs[b] - 1), ties to the smaller position; the
+ * last slot is moved into its place and len[b] becomes len[b] - 1.
+ *   scores [B][Hq][Tcap], lse [B][Hq]  from aqua_decode_attn
+ *   evicted_out nullable [B][Hkv] int32: evicted absolute position, or -1
+ * Requires pos, score and n_abs in the cache.  cache->max_len is lowered to
+ * min(max_len, budget) on the host.
+ */
+AQUA_API int aqua_h2o_update(aqua_cache* cache, const float* scores, const float* lse, int Hq, int budget,
+                    int recent, int32_t* evicted_out, aqua_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQUA_H_ */

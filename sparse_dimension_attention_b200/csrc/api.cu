@@ -1,0 +1,235 @@
+// extern "C" entry points: argument checks on the host (nothing is launched on
+// a failed check), workspace sizing, and dispatch to the kernel launchers.
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "aqua_internal.cuh"
+
+namespace aqua {
+
+static thread_local char g_err[512] = "";
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return AQUA_OK;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+// launchers (defined next to their kernels)
+int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
+                        cudaStream_t st);
+size_t decode_workspace_bytes(int n_units, int G);
+int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale,
+                  void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
+                  float* lse_out, void* ws, cudaStream_t st);
+size_t prefill_workspace_bytes(const aqua_cache* c, int Hq, int L);
+int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const float* P, int Hq, int k,
+                   float scale, void* out, int out_dtype, int32_t* sel_out, void* ws, cudaStream_t st);
+int launch_h2o_update(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
+                      int32_t* evicted_out, cudaStream_t st);
+size_t calibrate_workspace_bytes(int n, int d);
+int launch_calibrate(const float* X, int n, float* P_out, float* sigma_out, void* ws, cudaStream_t st);
+
+}  // namespace aqua
+
+using aqua::set_error;
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int validate_cache(const aqua_cache* c) {
+  if (c == nullptr) return set_error(AQUA_ERR_ARG, "cache descriptor is NULL");
+  if (c->k_proj == nullptr || c->v == nullptr || c->len == nullptr || c->ctrl == nullptr)
+    return set_error(AQUA_ERR_ARG, "cache: k_proj, v, len and ctrl must be non-NULL");
+  if (c->d != aqua::kHeadDim) return set_error(AQUA_ERR_UNSUPPORTED, "cache: head dim %d (only 128)", c->d);
+  if (c->d_store < 1 || c->d_store > c->d)
+    return set_error(AQUA_ERR_ARG, "cache: d_store %d outside [1, d]", c->d_store);
+  if (c->B < 1 || c->Hkv < 1) return set_error(AQUA_ERR_ARG, "cache: B=%d Hkv=%d", c->B, c->Hkv);
+  if (c->Tcap < 16 || c->Tcap % 16 != 0)
+    return set_error(AQUA_ERR_ARG, "cache: Tcap %d must be a positive multiple of 16", c->Tcap);
+  if (c->dtype != AQUA_F32 && c->dtype != AQUA_BF16)
+    return set_error(AQUA_ERR_UNSUPPORTED, "cache: dtype %d", c->dtype);
+  if (c->max_len < 0 || c->max_len > c->Tcap)
+    return set_error(AQUA_ERR_ARG, "cache: max_len %d outside [0, Tcap=%d]", c->max_len, c->Tcap);
+  if (!aligned(c->k_proj, 16) || !aligned(c->v, 16))
+    return set_error(AQUA_ERR_ARG, "cache: k_proj and v must be 16-byte aligned");
+  if (c->pos != nullptr && (c->score == nullptr || c->n_abs == nullptr))
+    return set_error(AQUA_ERR_ARG, "cache: pos requires score and n_abs");
+  if ((long long)c->B * c->Hkv > (1LL << 24))
+    return set_error(AQUA_ERR_UNSUPPORTED, "cache: B*Hkv too large");
+  return AQUA_OK;
+}
+
+int check_out_dtype(int out_dtype) {
+  if (out_dtype != AQUA_F32 && out_dtype != AQUA_BF16)
+    return set_error(AQUA_ERR_UNSUPPORTED, "out_dtype %d", out_dtype);
+  return AQUA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* aqua_last_error(void) { return aqua::g_err; }
+
+int aqua_version(void) { return 1; }
+
+int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream) {
+  if (cache == nullptr || cache->ctrl == nullptr || status_out == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_status: NULL argument");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, cache->ctrl + aqua::kCtrlStatus, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return aqua::check_launch("aqua_status copy");
+  if (v != 0) {
+    if (cudaMemsetAsync(cache->ctrl + aqua::kCtrlStatus, 0, sizeof(int32_t), st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return aqua::check_launch("aqua_status clear");
+  }
+  *status_out = v;
+  return AQUA_OK;
+}
+
+size_t aqua_calibrate_workspace_size(int n, int d) {
+  if (n < 1 || d != aqua::kHeadDim) return 0;
+  return aqua::calibrate_workspace_bytes(n, d);
+}
+
+int aqua_calibrate(const float* X, int n, int d, float* P_out, float* sigma_out, void* workspace,
+                   size_t workspace_bytes, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  if (X == nullptr || P_out == nullptr || sigma_out == nullptr || workspace == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_calibrate: NULL pointer");
+  if (d != aqua::kHeadDim) return set_error(AQUA_ERR_UNSUPPORTED, "aqua_calibrate: d=%d (only 128)", d);
+  if (n < 1) return set_error(AQUA_ERR_ARG, "aqua_calibrate: n=%d", n);
+  if (!aligned(X, 16) || !aligned(workspace, 256))
+    return set_error(AQUA_ERR_ARG, "aqua_calibrate: X 16-byte, workspace 256-byte alignment required");
+  if (workspace_bytes < aqua::calibrate_workspace_bytes(n, d))
+    return set_error(AQUA_ERR_WORKSPACE, "aqua_calibrate: workspace %zu < %zu bytes", workspace_bytes,
+                     aqua::calibrate_workspace_bytes(n, d));
+  return aqua::launch_calibrate(X, n, P_out, sigma_out, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int aqua_project_keys(aqua_cache* cache, const void* k_new, const void* v_new, const float* P, int L,
+                      aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  int rc = validate_cache(cache);
+  if (rc != AQUA_OK) return rc;
+  if (k_new == nullptr || v_new == nullptr || P == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_project_keys: NULL input");
+  if (L < 1) return set_error(AQUA_ERR_ARG, "aqua_project_keys: L=%d", L);
+  if ((long long)cache->max_len + L > cache->Tcap)
+    return set_error(AQUA_ERR_ARG, "aqua_project_keys: max_len %d + L %d exceeds Tcap %d", cache->max_len, L,
+                     cache->Tcap);
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(P, 16))
+    return set_error(AQUA_ERR_ARG, "aqua_project_keys: inputs must be 16-byte aligned");
+  rc = aqua::launch_project_keys(cache, k_new, v_new, P, L, reinterpret_cast<cudaStream_t>(stream));
+  if (rc == AQUA_OK) cache->max_len += L;
+  return rc;
+}
+
+size_t aqua_decode_workspace_size(const aqua_cache* cache, int Hq) {
+  if (validate_cache(cache) != AQUA_OK || Hq < 1 || Hq % cache->Hkv != 0) return 0;
+  return aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv);
+}
+
+int aqua_decode_attn(const aqua_cache* cache, const void* q, const float* P, int Hq, int k, float scale,
+                     void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
+                     float* lse_out, void* workspace, size_t workspace_bytes, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  int rc = validate_cache(cache);
+  if (rc != AQUA_OK) return rc;
+  if ((rc = check_out_dtype(out_dtype)) != AQUA_OK) return rc;
+  if (q == nullptr || P == nullptr || out == nullptr || workspace == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: NULL q, P, out or workspace");
+  if (Hq < 1 || Hq % cache->Hkv != 0)
+    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: Hq=%d not a multiple of Hkv=%d", Hq, cache->Hkv);
+  const int G = Hq / cache->Hkv;
+  if (G != 1 && G != 2 && G != 4)
+    return set_error(AQUA_ERR_UNSUPPORTED, "aqua_decode_attn: Hq/Hkv=%d not in {1,2,4}", G);
+  if (k < 1 || k > cache->d_store)
+    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k=%d outside [1, d_store=%d]", k, cache->d_store);
+  if (!aligned(q, 16) || !aligned(P, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: q, P, out 16-byte and workspace 256-byte alignment required");
+  const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, G);
+  if (workspace_bytes < need)
+    return set_error(AQUA_ERR_WORKSPACE, "aqua_decode_attn: workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)cache->d);
+  return aqua::launch_decode(cache, q, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, scores_out, lse_out,
+                             workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L) {
+  if (validate_cache(cache) != AQUA_OK || Hq < 1 || Hq % cache->Hkv != 0 || L < 1) return 0;
+  return aqua::prefill_workspace_bytes(cache, Hq, L);
+}
+
+int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, const float* P, int Hq, int k,
+                      float scale, void* out, int out_dtype, int32_t* sel_out, void* workspace,
+                      size_t workspace_bytes, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  int rc = validate_cache(cache);
+  if (rc != AQUA_OK) return rc;
+  if ((rc = check_out_dtype(out_dtype)) != AQUA_OK) return rc;
+  if (q == nullptr || P == nullptr || out == nullptr || workspace == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: NULL q, P, out or workspace");
+  if (cache->dtype != AQUA_BF16) return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: bf16 cache only");
+  if (Hq < 1 || Hq % cache->Hkv != 0)
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: Hq=%d not a multiple of Hkv=%d", Hq, cache->Hkv);
+  if (k < 1 || k > cache->d_store)
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: k=%d outside [1, d_store=%d]", k, cache->d_store);
+  if (L < 1 || pos0 < 0 || (long long)pos0 + L > cache->Tcap)
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: pos0=%d L=%d outside Tcap=%d", pos0, L, cache->Tcap);
+  if (!aligned(q, 16) || !aligned(P, 16) || !aligned(out, 16) || !aligned(workspace, 256))
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: alignment");
+  const size_t need = aqua::prefill_workspace_bytes(cache, Hq, L);
+  if (workspace_bytes < need)
+    return set_error(AQUA_ERR_WORKSPACE, "aqua_prefill_attn: workspace %zu < %zu bytes", workspace_bytes, need);
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)cache->d);
+  return aqua::launch_prefill(cache, q, pos0, L, P, Hq, k, scale, out, out_dtype, sel_out, workspace,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int aqua_h2o_update(aqua_cache* cache, const float* scores, const float* lse, int Hq, int budget, int recent,
+                    int32_t* evicted_out, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  int rc = validate_cache(cache);
+  if (rc != AQUA_OK) return rc;
+  if (cache->pos == nullptr || cache->score == nullptr || cache->n_abs == nullptr)
+    return set_error(AQUA_ERR_ARG, "aqua_h2o_update: cache needs pos, score and n_abs");
+  if (scores == nullptr || lse == nullptr) return set_error(AQUA_ERR_ARG, "aqua_h2o_update: NULL scores or lse");
+  if (Hq < 1 || Hq % cache->Hkv != 0)
+    return set_error(AQUA_ERR_ARG, "aqua_h2o_update: Hq=%d not a multiple of Hkv=%d", Hq, cache->Hkv);
+  if (budget < 1 || recent < 0 || recent > budget)
+    return set_error(AQUA_ERR_ARG, "aqua_h2o_update: need budget >= 1 and 0 <= recent <= budget (%d, %d)", budget,
+                     recent);
+  rc = aqua::launch_h2o_update(cache, scores, lse, Hq, budget, recent, evicted_out,
+                               reinterpret_cast<cudaStream_t>(stream));
+  if (rc == AQUA_OK && cache->max_len > budget) cache->max_len -= 1;
+  return rc;
+}
+
+}  // extern "C"

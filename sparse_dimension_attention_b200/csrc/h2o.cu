@@ -1,0 +1,137 @@
+// H2O heavy-hitter update on top of AQUA decode.
+//
+// The AQUA abstract names H2O ("synergistically accelerate existing token
+// eviction methods like H2O") without giving its rule; the reading taken:
+// every cached token of a (sequence, KV head) carries a cumulative score, the
+// sum over the group's query heads and over the decode steps it has seen of
+// its AQUA softmax probability; after a step that leaves more than `budget`
+// tokens, the lowest-scored token outside the `recent` newest positions is
+// evicted (ties to the older position) and its slot is reused.
+#include <math.h>
+
+#include "aqua_internal.cuh"
+
+namespace aqua {
+
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kThreads = 256;
+
+struct Cand {
+  float score;
+  int pos;
+  int slot;
+};
+
+__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
+  if (a.slot < 0) return false;
+  if (b.slot < 0) return true;
+  return a.score < b.score || (a.score == b.score && a.pos < b.pos);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kproj, T* __restrict__ vcache,
+                                                              int32_t* len, const int32_t* __restrict__ n_abs,
+                                                              int32_t* __restrict__ pos, float* __restrict__ score,
+                                                              int32_t* ctrl, const float* __restrict__ scores,
+                                                              const float* __restrict__ lse, int32_t* evicted_out,
+                                                              int B, int Hq, int Hkv, int d_store, int Tcap,
+                                                              int budget, int recent) {
+  __shared__ Cand wbest[kThreads / 32];
+  __shared__ int s_victim, s_vpos, is_last;
+  const int u = blockIdx.x;
+  const int b = u / Hkv, g = u % Hkv;
+  const int G = Hq / Hkv;
+  const int n = min(max(__ldcg(len + b), 0), Tcap);   // read before the ticket below
+  const int newest = __ldcg(n_abs + b) - 1;
+  const size_t ub = (size_t)u * Tcap;
+
+  Cand best{INFINITY, 0, -1};
+  for (int t = threadIdx.x; t < n; t += kThreads) {
+    float acc = 0.f;
+    for (int h = g * G; h < (g + 1) * G; ++h) {
+      const size_t bh = (size_t)b * Hq + h;
+      acc += expf(scores[bh * Tcap + t] - lse[bh]);
+    }
+    const float sc = score[ub + t] + acc;
+    score[ub + t] = sc;
+    const int ps = pos[ub + t];
+    if (ps <= newest - recent) {
+      const Cand cnd{sc, ps, t};
+      if (better(cnd, best)) best = cnd;
+    }
+  }
+  // block arg-min
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Cand other;
+    other.score = __shfl_xor_sync(0xffffffffu, best.score, o);
+    other.pos = __shfl_xor_sync(0xffffffffu, best.pos, o);
+    other.slot = __shfl_xor_sync(0xffffffffu, best.slot, o);
+    if (better(other, best)) best = other;
+  }
+  if ((threadIdx.x & 31) == 0) wbest[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Cand bb = wbest[0];
+    for (int w = 1; w < kThreads / 32; ++w)
+      if (better(wbest[w], bb)) bb = wbest[w];
+    const bool evict = n > budget && bb.slot >= 0;
+    s_victim = evict ? bb.slot : -1;
+    s_vpos = evict ? bb.pos : -1;
+    if (evicted_out) evicted_out[u] = s_vpos;
+  }
+  __syncthreads();
+  const int v = s_victim;
+  if (v >= 0 && v != n - 1) {
+    // move the last slot into the evicted one
+    const int last = n - 1;
+    T* kp = kproj + (size_t)u * d_store * Tcap;
+    for (int j = threadIdx.x; j < d_store; j += kThreads) kp[(size_t)j * Tcap + v] = kp[(size_t)j * Tcap + last];
+    T* vp = vcache + ub * D;
+    for (int j = threadIdx.x; j < D; j += kThreads) vp[(size_t)v * D + j] = vp[(size_t)last * D + j];
+    if (threadIdx.x == 0) {
+      pos[ub + v] = pos[ub + last];
+      score[ub + v] = score[ub + last];
+    }
+  }
+  // the last CTA shortens the sequences that evicted (all KV heads of a
+  // sequence evict together: they hold the same number of tokens and the same
+  // recent window)
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(ctrl + kCtrlH2OTicket, 1) == (int)gridDim.x - 1);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int bb = threadIdx.x; bb < B; bb += kThreads) {
+      const int nb = len[bb];
+      // eviction happened iff the sequence was over budget and some slot lay
+      // outside the recent window (the recent positions are always present)
+      if (nb > budget && nb - min(recent, n_abs[bb]) > 0) len[bb] = nb - 1;
+    }
+    if (threadIdx.x == 0) ctrl[kCtrlH2OTicket] = 0;
+  }
+}
+
+}  // namespace
+
+int launch_h2o_update(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
+                      int32_t* evicted_out, cudaStream_t st) {
+  const int n_units = c->B * c->Hkv;
+  if (c->dtype == AQUA_BF16) {
+    h2o_update_kernel<__nv_bfloat16><<<n_units, kThreads, 0, st>>>(
+        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos,
+        c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+  } else {
+    h2o_update_kernel<float><<<n_units, kThreads, 0, st>>>(
+        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl,
+        scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+  }
+  return check_launch("h2o_update_kernel");
+}
+
+}  // namespace aqua

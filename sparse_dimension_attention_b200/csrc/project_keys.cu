@@ -1,0 +1,125 @@
+// Key projection + append: k~ = k P, stored dimension-major (one contiguous row
+// per projected dimension over the tokens), values copied token-major.
+//
+// AQUA abstract / edgentiq "How AQUA Works", Online Inference: keys are
+// projected with the offline matrix before attention; AQUA-Memory
+// ("AQUA-Memory: Dual Savings") keeps only the leading d_store projected
+// dimensions in the cache.
+#include "aqua_internal.cuh"
+
+namespace aqua {
+
+namespace {
+
+constexpr int D = kHeadDim;
+constexpr int kTokPerCta = 8;  // one warp per token
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&f)[4]);
+template <>
+__device__ __forceinline__ void load4(const float* p, float (&f)[4]) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&f)[4]) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+}
+
+template <typename T>
+__device__ __forceinline__ void copy4(T* dst, const T* src);
+template <>
+__device__ __forceinline__ void copy4(float* dst, const float* src) {
+  *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
+}
+template <>
+__device__ __forceinline__ void copy4(__nv_bfloat16* dst, const __nv_bfloat16* src) {
+  *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+}
+
+// grid (ceil(L/8), Hkv, B), block 256: warp w projects token blockIdx.x*8+w of (b, g).
+template <typename T>
+__global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__ k_new,
+                                                           const T* __restrict__ v_new,
+                                                           const float* __restrict__ P,
+                                                           T* __restrict__ kproj, T* __restrict__ vcache,
+                                                           int32_t* len, int32_t* n_abs, int32_t* pos,
+                                                           float* score, int32_t* ctrl, int B, int L,
+                                                           int Hkv, int d_store, int Tcap) {
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int l = blockIdx.x * kTokPerCta + warp;
+  // Lengths are read before this CTA takes its ticket below; the last CTA
+  // advances them only after every CTA has taken one.
+  const int base = __ldcg(len + b);
+  const int abase = n_abs ? __ldcg(n_abs + b) : base;
+  if (l < L && (base < 0 || base + l >= Tcap)) {
+    if (lane == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
+  } else if (l < L) {
+    const size_t row = ((size_t)b * L + l) * Hkv + g;
+    float kv[4];
+    load4<T>(k_new + row * D + 4 * lane, kv);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* Pg = P + (size_t)g * D * D;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      const float ki = __shfl_sync(0xffffffffu, kv[i & 3], i >> 2);
+      const float4 pr = __ldg(reinterpret_cast<const float4*>(Pg + (size_t)i * D) + lane);
+      acc[0] = fmaf(ki, pr.x, acc[0]);
+      acc[1] = fmaf(ki, pr.y, acc[1]);
+      acc[2] = fmaf(ki, pr.z, acc[2]);
+      acc[3] = fmaf(ki, pr.w, acc[3]);
+    }
+    const int slot = base + l;
+    const size_t unit = (size_t)b * Hkv + g;
+    T* kp = kproj + unit * d_store * (size_t)Tcap + slot;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int j = 4 * lane + s;
+      if (j < d_store) kp[(size_t)j * Tcap] = Elem<T>::from_f32(acc[s]);
+    }
+    copy4<T>(vcache + (unit * Tcap + slot) * D + 4 * lane, v_new + row * D + 4 * lane);
+    if (pos != nullptr && lane == 0) {
+      pos[unit * Tcap + slot] = abase + l;
+      score[unit * Tcap + slot] = 0.f;
+    }
+  }
+  __shared__ int is_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int total = gridDim.x * gridDim.y * gridDim.z;
+    is_last = (atomicAdd(ctrl + kCtrlAppendTicket, 1) == total - 1);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int bb = threadIdx.x; bb < B; bb += blockDim.x) {
+      len[bb] += L;
+      if (n_abs) n_abs[bb] += L;
+    }
+    if (threadIdx.x == 0) ctrl[kCtrlAppendTicket] = 0;
+  }
+}
+
+}  // namespace
+
+int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
+                        cudaStream_t st) {
+  dim3 grid((L + kTokPerCta - 1) / kTokPerCta, c->Hkv, c->B);
+  if (c->dtype == AQUA_BF16) {
+    project_keys_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), P,
+        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs,
+        c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+  } else {
+    project_keys_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
+        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score,
+        c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+  }
+  return check_launch("project_keys_kernel");
+}
+
+}  // namespace aqua

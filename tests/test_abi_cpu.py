@@ -1,0 +1,151 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every symbol that
+include/aqua.h declares, the ctypes struct matches the C layout, and host-side
+argument checks reject bad calls without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_dimension_attention_b200 as aq
+from sparse_dimension_attention_b200 import abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "aqua.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"AQUA_API\s+[\w\s\*]+?\b(aqua_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_dimension_attention_b200 import build
+    build.build()
+    return aq.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(abi.EXPORTED)
+
+
+def test_exports_nothing_else(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True, text=True).stdout
+    syms = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert syms == set(_declared())
+
+
+def test_struct_layout():
+    # 7 pointers followed by 7 ints on LP64
+    assert ctypes.sizeof(abi.aqua_cache) == 7 * 8 + 7 * 4 + 4   # trailing padding to 8
+    assert abi.aqua_cache.B.offset == 56
+    assert abi.aqua_cache.dtype.offset == 56 + 6 * 4
+
+
+def test_version(lib):
+    assert aq.aqua_version() == 1
+
+
+def _desc(**kw):
+    base = dict(k_proj=0x1000, v=0x2000, len=0x3000, n_abs=0x3100, pos=None, score=None, ctrl=0x4000,
+                B=2, Hkv=2, d=128, d_store=128, Tcap=64, max_len=0, dtype=abi.AQUA_BF16)
+    base.update(kw)
+    return abi.aqua_cache(**base)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d", 64, abi.AQUA_ERR_UNSUPPORTED),
+    ("d_store", 0, abi.AQUA_ERR_ARG),
+    ("d_store", 129, abi.AQUA_ERR_ARG),
+    ("Tcap", 40, abi.AQUA_ERR_ARG),
+    ("dtype", 7, abi.AQUA_ERR_UNSUPPORTED),
+    ("k_proj", None, abi.AQUA_ERR_ARG),
+    ("k_proj", 0x1004, abi.AQUA_ERR_ARG),       # misaligned
+    ("max_len", 65, abi.AQUA_ERR_ARG),
+])
+def test_project_keys_rejects_bad_cache(lib, field, value, code):
+    c = _desc(**{field: value})
+    rc = lib.aqua_project_keys(ctypes.byref(c), 0x5000, 0x6000, 0x7000, 1, None)
+    assert rc == code
+    assert lib.aqua_last_error().decode() != ""
+
+
+def test_project_keys_rejects_overflow(lib):
+    c = _desc(max_len=60)
+    assert lib.aqua_project_keys(ctypes.byref(c), 0x5000, 0x6000, 0x7000, 5, None) == abi.AQUA_ERR_ARG
+    assert c.max_len == 60     # unchanged on failure
+    assert lib.aqua_project_keys(ctypes.byref(c), 0x5000, 0x6000, 0x7000, 0, None) == abi.AQUA_ERR_ARG
+
+
+def test_decode_argument_checks(lib):
+    c = _desc()
+    ws = lib.aqua_decode_workspace_size(ctypes.byref(c), 8)
+    assert ws > 0
+    call = lambda **kw: lib.aqua_decode_attn(
+        ctypes.byref(kw.get("c", c)), kw.get("q", 0x5000), 0x7000, kw.get("Hq", 8), kw.get("k", 96), 0.0,
+        0x8000, kw.get("od", abi.AQUA_BF16), None, None, None, None, kw.get("ws", 0x10000),
+        kw.get("wsb", ws), None)
+    assert call(Hq=7) == abi.AQUA_ERR_ARG                 # not a multiple of Hkv
+    assert call(Hq=16) == abi.AQUA_ERR_UNSUPPORTED        # group of 8
+    assert call(k=0) == abi.AQUA_ERR_ARG
+    assert call(k=129) == abi.AQUA_ERR_ARG
+    assert call(c=_desc(d_store=96), k=97) == abi.AQUA_ERR_ARG
+    assert call(q=None) == abi.AQUA_ERR_ARG
+    assert call(od=5) == abi.AQUA_ERR_UNSUPPORTED
+    assert call(wsb=ws - 1) == abi.AQUA_ERR_WORKSPACE
+    assert call(ws=0x10010) == abi.AQUA_ERR_ARG           # workspace alignment
+
+
+def test_decode_workspace_grows_with_units(lib):
+    a = lib.aqua_decode_workspace_size(ctypes.byref(_desc(B=1, Hkv=1)), 4)
+    b = lib.aqua_decode_workspace_size(ctypes.byref(_desc(B=8, Hkv=8)), 32)
+    assert 0 < a < b
+    assert lib.aqua_decode_workspace_size(ctypes.byref(_desc()), 3) == 0
+
+
+def test_h2o_argument_checks(lib):
+    c = _desc()
+    assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 8, 16, 4, None, None) == abi.AQUA_ERR_ARG  # no pos
+    c = _desc(pos=0x9000, score=0x9100)
+    assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 8, 16, 17, None, None) == abi.AQUA_ERR_ARG
+    assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 8, 0, 0, None, None) == abi.AQUA_ERR_ARG
+
+
+def test_prefill_argument_checks(lib):
+    c = _desc()
+    ws = lib.aqua_prefill_workspace_size(ctypes.byref(c), 8, 32)
+    assert lib.aqua_prefill_attn(ctypes.byref(c), 0x5000, 40, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
+                                 None, 0x10000, ws, None) == abi.AQUA_ERR_ARG   # pos0 + L > Tcap
+    c32 = _desc(dtype=abi.AQUA_F32)
+    assert lib.aqua_prefill_attn(ctypes.byref(c32), 0x5000, 0, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
+                                 None, 0x10000, ws, None) == abi.AQUA_ERR_UNSUPPORTED
+
+
+def test_calibrate_argument_checks(lib):
+    assert lib.aqua_calibrate_workspace_size(16384, 128) > 0
+    assert lib.aqua_calibrate_workspace_size(16384, 64) == 0
+    assert lib.aqua_calibrate(0x1000, 10, 64, 0x2000, 0x3000, 0x4000, 1 << 30, None) == abi.AQUA_ERR_UNSUPPORTED
+    need = lib.aqua_calibrate_workspace_size(100, 128)
+    assert lib.aqua_calibrate(0x1000, 100, 128, 0x2000, 0x3000, 0x4000, need - 8, None) == abi.AQUA_ERR_WORKSPACE
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "sparse_dimension_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "aqua_oracle" not in txt, f
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(abi, "_lib", None)
+    with pytest.raises(RuntimeError):
+        abi.load_library(str(tmp_path / "nope.so"))

@@ -1,0 +1,206 @@
+"""GPU parity of the decode path (key append, q projection + top-k, split-K
+sparse-dimension attention) against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import aqua_oracle as O
+import sparse_dimension_attention_b200 as aq
+from aqua_testlib import (calib_P, check_selection, fill_cache, oracle_cache, rel_err_rows, run_decode, tdev,
+                          torch_dtype)
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16_OUT = 2e-3   # bf16 output vs the oracle output rounded to bf16
+TOL_F32_OUT = 1e-5
+
+
+def _decode_case(B, Hq, Hkv, T, k, kv="bf16", out="bf16", lens=None, d_store=None, Tcap=None, chunk=None):
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, Hq, Hkv, T, bf16=(kv == "bf16"), steps=1)
+    k_all = np.concatenate([inp["k_hist"], inp["k_new"].transpose(1, 0, 2, 3)], axis=1)   # [B, T+1, Hkv, d]
+    v_all = np.concatenate([inp["v_hist"], inp["v_new"].transpose(1, 0, 2, 3)], axis=1)
+    cache = aq.AquaCache(B, Hkv, Tcap or (T + 1 + 15) // 16 * 16, d_store=d_store, dtype=torch_dtype(kv))
+    Pt = fill_cache(cache, k_all, v_all, P32, chunk=chunk)
+    Tn = T + 1
+    if lens is not None:
+        cache.len.copy_(torch.tensor(lens, dtype=torch.int32))
+    else:
+        lens = [Tn] * B
+    q = inp["q"][0]
+    res = run_decode(cache, q, Pt, k, out_dtype=torch_dtype(out), scores=True)
+    Kt = oracle_cache(k_all, P64, kv, d_store)
+    V = v_all.transpose(0, 2, 1, 3).astype(np.float64)
+    ref = O.decode(q, P64, Kt, V, lens, k, m=d_store, out_dtype=out)
+    return cache, res, ref, lens
+
+
+def _check_outputs(res, ref, out, lens):
+    tol = TOL_BF16_OUT if out == "bf16" else TOL_F32_OUT
+    err = rel_err_rows(res["out"], ref["out"])
+    assert np.max(err) <= tol, f"max rel err {np.max(err):.3e} > {tol}"
+    np.testing.assert_allclose(res["lse"], ref["lse"], rtol=1e-5, atol=1e-5)
+
+
+def test_decode_fp32_tiny_config():
+    """1 sequence, 4 query heads over 1 KV head, T = 1024, k = 96, f32 throughout."""
+    cache, res, ref, lens = _decode_case(1, 4, 1, 1023, 96, kv="f32", out="f32")
+    _check_outputs(res, ref, "f32", lens)
+    near = check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 96)
+    assert near == 0
+
+
+@pytest.mark.parametrize("k", [128, 96, 64, 32, 1])
+def test_decode_bf16_k_sweep(k):
+    cache, res, ref, lens = _decode_case(2, 8, 2, 700, k)
+    _check_outputs(res, ref, "bf16", lens)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], k)
+
+
+@pytest.mark.parametrize("T", [0, 1, 15, 127, 128, 129, 1000])
+def test_decode_bf16_ragged_lengths(T):
+    # several tiles, a ragged tail, and a history shorter than one tile
+    cache, res, ref, lens = _decode_case(2, 8, 2, T, 96)
+    _check_outputs(res, ref, "bf16", lens)
+
+
+def test_decode_bf16_per_sequence_lengths_and_empty():
+    lens = [1000, 37, 0, 513]
+    cache, res, ref, _ = _decode_case(4, 8, 2, 1000, 64, lens=lens)
+    live = [i for i, L in enumerate(lens) if L > 0]
+    _check_outputs({"out": res["out"][live], "lse": res["lse"][live]},
+                   {"out": ref["out"][live], "lse": ref["lse"][live]}, "bf16", None)
+    assert np.all(res["out"][2] == 0.0)
+    assert np.all(np.isneginf(res["lse"][2]))
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_decode_group_sizes(G):
+    Hkv = 2
+    cache, res, ref, lens = _decode_case(1, G * Hkv, Hkv, 300, 48)
+    _check_outputs(res, ref, "bf16", lens)
+
+
+def test_decode_f32_output_from_bf16_cache():
+    cache, res, ref, lens = _decode_case(2, 8, 2, 900, 96, out="f32")
+    _check_outputs(res, ref, "f32", lens)
+
+
+def test_decode_truncated_cache():
+    """AQUA-Memory: only the first m = 96 projected dims are stored; k = 64 chosen within them."""
+    cache, res, ref, lens = _decode_case(2, 8, 2, 640, 64, d_store=96)
+    _check_outputs(res, ref, "bf16", lens)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 64, m=96)
+    assert res["sel"].max() < 96
+
+
+def test_decode_scores_match_oracle():
+    cache, res, ref, lens = _decode_case(1, 4, 1, 200, 96, kv="f32", out="f32")
+    T = lens[0]
+    for h in range(4):
+        p = np.exp(res["scores"][0, h, :T] - res["lse"][0, h])
+        np.testing.assert_allclose(p, ref["probs"][0][h], rtol=2e-5, atol=1e-9)
+
+
+def test_decode_adversarial_ties():
+    """Identity projection and magnitudes with exact ties and +- pairs: ties go to the lower index."""
+    B, Hq, Hkv, T, k = 1, 4, 1, 64, 5
+    P32 = np.eye(128, dtype=np.float32)[None]
+    rng = np.random.default_rng(5)
+    q = np.zeros((B, Hq, 128), dtype=np.float32)
+    q[0, 0, [3, 9, 20, 40, 41, 90, 100]] = [2, -2, 2, 1, -1, 1, 1]      # 3 tied at 2, 4 tied at 1
+    q[0, 1, :] = 1.0                                                      # all tied
+    q[0, 2, ::2] = -0.5
+    q[0, 2, 1::2] = 0.5
+    q[0, 3] = rng.integers(-2, 3, 128)
+    k_tok = synth.cast_bf16(rng.standard_normal((B, T, Hkv, 128)).astype(np.float32))
+    v_tok = synth.cast_bf16(rng.standard_normal((B, T, Hkv, 128)).astype(np.float32))
+    q = synth.cast_bf16(q)
+    cache = aq.AquaCache(B, Hkv, 64)
+    Pt = fill_cache(cache, k_tok, v_tok, P32)
+    res = run_decode(cache, q, Pt, k)
+    for h in range(Hq):
+        ref_sel = O.select_dims(q[0, h].astype(np.float64), k)
+        np.testing.assert_array_equal(res["sel"][0, h], ref_sel)
+    assert list(res["sel"][0, 0]) == [3, 9, 20, 40, 41]
+    assert list(res["sel"][0, 1]) == [0, 1, 2, 3, 4]
+    ref = O.decode(q, P32.astype(np.float64), oracle_cache(k_tok, P32.astype(np.float64), "bf16"),
+                   v_tok.transpose(0, 2, 1, 3), [T], k, out_dtype="bf16")
+    assert np.max(rel_err_rows(res["out"], ref["out"])) <= TOL_BF16_OUT
+
+
+def test_key_cache_storage_rounding():
+    """Stored K~ equals the oracle's bf16 RNE of k P, except where the exact value lies within
+    f32 rounding of a bf16 midpoint (then the two neighbours are both acceptable)."""
+    B, Hkv, T = 2, 2, 200
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, 4, Hkv, T, bf16=True, steps=1)
+    cache = aq.AquaCache(B, Hkv, 208)
+    fill_cache(cache, inp["k_hist"], inp["v_hist"], P32, chunk=64)
+    got = cache.k_proj.float().cpu().numpy()[..., :T].transpose(0, 1, 3, 2).astype(np.float64)   # [B,Hkv,T,d]
+    exact = np.einsum("btgi,gij->bgtj", inp["k_hist"].astype(np.float64), P64)
+    ref = O.round_bf16(exact)
+    diff = got != ref
+    if diff.any():
+        e, g = exact[diff], got[diff]
+        r = ref[diff]
+        mid = (g + r) / 2
+        assert np.all(np.abs(e - mid) <= 1e-6 * np.abs(e) + 1e-30)
+    assert diff.mean() < 1e-3
+    np.testing.assert_array_equal(cache.v.float().cpu().numpy()[:, :, :T].transpose(0, 2, 1, 3), inp["v_hist"])
+    assert cache.len.cpu().tolist() == [T, T] and cache.max_len == T
+
+
+def test_chunked_append_equals_single_append():
+    B, Hkv, T = 1, 2, 300
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, 4, Hkv, T, bf16=True, steps=1)
+    c1 = aq.AquaCache(B, Hkv, 304)
+    c2 = aq.AquaCache(B, Hkv, 304)
+    fill_cache(c1, inp["k_hist"], inp["v_hist"], P32)
+    fill_cache(c2, inp["k_hist"], inp["v_hist"], P32, chunk=7)
+    assert torch.equal(c1.k_proj, c2.k_proj) and torch.equal(c1.v, c2.v)
+    assert torch.equal(c1.len, c2.len)
+
+
+def test_repeated_calls_are_deterministic_and_status_clean():
+    cache, res, ref, lens = _decode_case(2, 8, 2, 2000, 96)
+    P64, P32 = calib_P(2)
+    q = synth.decode_inputs(2, 8, 2, 2000, steps=1)["q"][0]
+    r2 = run_decode(cache, q, tdev(P32), 96)
+    np.testing.assert_array_equal(res["out"], r2["out"])
+    assert aq.aqua_status(cache.desc) == aq.AQUA_OK
+    assert int(cache.ctrl[1:].abs().sum().item()) == 0      # tickets back at zero
+
+
+def test_snapshot_restore_resumes_identically():
+    cache, res, ref, lens = _decode_case(1, 4, 1, 500, 96)
+    snap = cache.snapshot()
+    P64, P32 = calib_P(1)
+    q = synth.decode_inputs(1, 4, 1, 500, steps=1)["q"][0]
+    cache.k_proj.zero_()
+    cache.v.zero_()
+    cache.restore(snap)
+    r2 = run_decode(cache, q, tdev(P32), 96)
+    np.testing.assert_array_equal(res["out"], r2["out"])
+
+
+def test_long_context_split_k_sampled():
+    """B = 1, 32/8 heads, 131072 cached tokens, k = 96: the split-K path with
+    many partials per unit, checked on every head against the oracle."""
+    B, Hq, Hkv, T, k = 1, 32, 8, 131071, 96
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, Hq, Hkv, T, bf16=True, steps=1)
+    k_all = np.concatenate([inp["k_hist"], inp["k_new"].transpose(1, 0, 2, 3)], axis=1)
+    v_all = np.concatenate([inp["v_hist"], inp["v_new"].transpose(1, 0, 2, 3)], axis=1)
+    cache = aq.AquaCache(B, Hkv, T + 1)
+    Pt = fill_cache(cache, k_all, v_all, P32, chunk=16384)
+    q = inp["q"][0]
+    res = run_decode(cache, q, Pt, k, out_dtype=torch.float32)
+    for g in (0, 5):
+        Kt = O.build_key_cache(k_all[:, :, g:g + 1], P64[g:g + 1], "bf16").transpose(0, 2, 1, 3)
+        ref = O.decode(q[:, g * 4:(g + 1) * 4], P64[g:g + 1], Kt, v_all[:, :, g:g + 1].transpose(0, 2, 1, 3),
+                       [T + 1], k)
+        err = rel_err_rows(res["out"][:, g * 4:(g + 1) * 4], ref["out"])
+        assert np.max(err) <= TOL_F32_OUT * 3, np.max(err)
