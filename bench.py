@@ -3,8 +3,9 @@
 measured B200 copy bandwidth) on a Llama-3.1-8B-shaped attention layer.
 
 A step is one pass of the decode hot path over one batch: the new tokens' key
-projection + append (aqua_project_keys), then query projection + magnitude
-top-k + sparse-dimension split-K attention with its combine (aqua_decode_attn).
+projection + append, query projection + magnitude top-k, and the
+sparse-dimension split-K attention with its combine -- one aqua_decode_attn
+call carrying the step's k_new/v_new (two kernel launches).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl aqua|reference]
 
@@ -164,8 +165,8 @@ class DecodeBench:
         torch.cuda.synchronize()
         del inp["k_hist"], inp["v_hist"]
         self.q_h = torch.from_numpy(inp["q"]).to(self.dt).pin_memory()                       # [S, B, Hq, d]
-        self.k_h = torch.from_numpy(inp["k_new"][:, :, None]).to(self.dt).pin_memory()       # [S, B, 1, Hkv, d]
-        self.v_h = torch.from_numpy(inp["v_new"][:, :, None]).to(self.dt).pin_memory()
+        self.k_h = torch.from_numpy(inp["k_new"]).to(self.dt).pin_memory()                   # [S, B, Hkv, d]
+        self.v_h = torch.from_numpy(inp["v_new"]).to(self.dt).pin_memory()
         self.q_d = self.q_h.cuda()
         self.k_d = self.k_h.cuda()
         self.v_d = self.v_h.cuda()
@@ -181,8 +182,13 @@ class DecodeBench:
 
     def step(self, s: int, k: int, sel=None):
         aq, wl = self.aq, self.wl
-        aq.aqua_project_keys(self.cache.desc, self.k_d[s], self.v_d[s], self.P, 1)
-        aq.aqua_decode_attn(self.cache.desc, self.q_d[s], self.P, wl["Hq"], k, self.out, self.ws, sel_out=sel)
+        aq.aqua_decode_attn(self.cache.desc, self.q_d[s], self.P, wl["Hq"], k, self.out, self.ws,
+                            k_new=self.k_d[s], v_new=self.v_d[s], sel_out=sel)
+
+    def step_unfused(self, s: int, k: int):
+        aq, wl = self.aq, self.wl
+        aq.aqua_project_keys(self.cache.desc, self.k_d[s][:, None], self.v_d[s][:, None], self.P, 1)
+        aq.aqua_decode_attn(self.cache.desc, self.q_d[s], self.P, wl["Hq"], k, self.out, self.ws)
 
     def union_sizes(self, k: int, n: int):
         """|U| per (b, g) for the first n steps' queries (selection depends on q and P only)."""
@@ -211,6 +217,22 @@ class DecodeBench:
         wl, e = self.wl, self.esize
         return float(wl["B"] * wl["Hkv"] * 128 * e * 4)    # read k, v; write k~ column, v row
 
+    def timed_unfused(self, K: int, W: int, k: int):
+        """The same steps as two public calls (aqua_project_keys, then aqua_decode_attn)."""
+        torch = self.torch
+        self.rewind()
+        for s in range(W):
+            self.step_unfused(s % self.n_in, k)
+        torch.cuda.synchronize()
+        self.rewind()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(K):
+            self.step_unfused(s % self.n_in, k)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
     def timed(self, K: int, W: int, k: int, world: int, clocks: bool):
         torch = self.torch
         st = torch.cuda.current_stream()
@@ -221,7 +243,6 @@ class DecodeBench:
         torch.cuda.synchronize()
         self.rewind()
         ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        ev_m = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
@@ -232,19 +253,15 @@ class DecodeBench:
         e0.record(st)
         for s in range(K):
             ev_s[s].record(st)
-            self.aq.aqua_project_keys(self.cache.desc, self.k_d[s % self.n_in], self.v_d[s % self.n_in], self.P, 1)
-            ev_m[s].record(st)
-            self.aq.aqua_decode_attn(self.cache.desc, self.q_d[s % self.n_in], self.P, self.wl["Hq"], k, self.out,
-                                     self.ws)
+            self.step(s % self.n_in, k)
             ev_e[s].record(st)
         e1.record(st)
         torch.cuda.synchronize()
         barrier(world)
         clk = sampler.stop() if sampler else None
         total_ms = e0.elapsed_time(e1)
-        dec_ms = [ev_m[s].elapsed_time(ev_e[s]) for s in range(K)]
-        app_ms = [ev_s[s].elapsed_time(ev_m[s]) for s in range(K)]
-        return total_ms, dec_ms, app_ms, clk
+        step_ms = [ev_s[s].elapsed_time(ev_e[s]) for s in range(K)]
+        return total_ms, step_ms, clk
 
     def e2e(self, K: int, k: int):
         """Same steps through the public API from pinned host buffers: per step H2D of q,
@@ -268,8 +285,8 @@ class DecodeBench:
             qd.copy_(self.q_h[i], non_blocking=True)
             kd.copy_(self.k_h[i], non_blocking=True)
             vd.copy_(self.v_h[i], non_blocking=True)
-            self.aq.aqua_project_keys(self.cache.desc, kd, vd, self.P, 1)
-            self.aq.aqua_decode_attn(self.cache.desc, qd, self.P, wl["Hq"], k, self.out, self.ws)
+            self.aq.aqua_decode_attn(self.cache.desc, qd, self.P, wl["Hq"], k, self.out, self.ws, k_new=kd,
+                                     v_new=vd)
             self.out_h.copy_(self.out, non_blocking=True)
         e1.record(st)
         torch.cuda.synchronize()
@@ -376,14 +393,15 @@ def main():
 
     bench = DecodeBench(wl, K, W)
     usz = bench.union_sizes(wl["k"], min(K, bench.n_in))                       # [K, B, Hkv]
-    total_ms, dec_ms, app_ms, clk = bench.timed(K, W, wl["k"], world, clocks=(rank == 0))
+    total_ms, step_ms, clk = bench.timed(K, W, wl["k"], world, clocks=(rank == 0))
     total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / K
     value = world * wl["B"] * K / (total_ms / 1e3)
     T_steps = [wl["T"] + s for s in range(K)]
     dec_bytes = [bench.bytes_decode(usz[s % usz.shape[0]], T_steps[s]) for s in range(K)]
-    achieved = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
+    achieved = (sum(dec_bytes) + K * bench.bytes_append()) / (sum(step_ms) / 1e3) / 1e9
     step_gbs = (sum(dec_bytes) + K * bench.bytes_append()) / (total_ms / 1e3) / 1e9
+    unfused_ms = bench.timed_unfused(min(K, 100), W, wl["k"])
     e2e_ms, h2d, d2h = bench.e2e(K, wl["k"])
     e2e_ms = max_over_ranks(e2e_ms, world)
     line = {
@@ -400,21 +418,22 @@ def main():
         "mean_union": float(usz.mean()),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": None,
-                     "kernel": "aqua_decode_attn call (qproj_topk_kernel + decode_attn_kernel)",
+                     "kernel": "aqua_decode_attn step (qproj_topk_kernel with fused append + decode_attn_bf16_kernel)",
                      "peak_source": peak_kind,
-                     "decode_us": 1e3 * statistics.mean(dec_ms), "append_us": 1e3 * statistics.mean(app_ms)},
+                     "step_us": 1e3 * statistics.mean(step_ms)},
+        "unfused_step_us": 1e3 * unfused_ms,
         "e2e": {"value": world * wl["B"] * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 2 * K,
         "clocks": clk,
     }
     if not args.no_extras:
         sweep = []
         for kk in (128, 96, 64, 32):
             u = bench.union_sizes(kk, min(K, 8))
-            t_ms, d_ms, _, _ = bench.timed(K, W, kk, world, clocks=False)
+            t_ms, d_ms, _ = bench.timed(K, W, kk, world, clocks=False)
             t_ms = max_over_ranks(t_ms, world)
-            by = [bench.bytes_decode(u[s % u.shape[0]], T_steps[s]) for s in range(K)]
+            by = [bench.bytes_decode(u[s % u.shape[0]], T_steps[s]) + bench.bytes_append() for s in range(K)]
             sweep.append({"k": kk, "queries_per_s": world * wl["B"] * K / (t_ms / 1e3), "ms_per_step": t_ms / K,
                           "decode_us": 1e3 * statistics.mean(d_ms), "mean_union": float(u.mean()),
                           "decode_gbs": sum(by) / (sum(d_ms) / 1e3) / 1e9})
@@ -428,9 +447,9 @@ def main():
         lb = DecodeBench(lwl, min(K, 50), W)
         lu = lb.union_sizes(lwl["k"], min(K, 50, lb.n_in))
         Kl = min(K, 50)
-        t_ms, d_ms, _, _ = lb.timed(Kl, W, lwl["k"], world, clocks=False)
+        t_ms, d_ms, _ = lb.timed(Kl, W, lwl["k"], world, clocks=False)
         t_ms = max_over_ranks(t_ms, world)
-        by = [lb.bytes_decode(lu[s % lu.shape[0]], lwl["T"] + s) for s in range(Kl)]
+        by = [lb.bytes_decode(lu[s % lu.shape[0]], lwl["T"] + s) + lb.bytes_append() for s in range(Kl)]
         ach = sum(by) / (sum(d_ms) / 1e3) / 1e9
         line["long_context"] = {"workload": "long-context-decode", "B": 1, "T": lwl["T"], "k": lwl["k"],
                                 "queries_per_s": world * Kl / (t_ms / 1e3), "ms_per_step": t_ms / Kl,

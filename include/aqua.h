@@ -145,8 +145,14 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
 
 /*
  * One decode step of AQUA attention for every sequence and query head, over
- * the len[b] cached tokens (the step's own key must already be appended).
+ * the len[b] cached tokens.
  *   q          [B][Hq][d]  cache dtype; query head h uses KV head h / (Hq/Hkv)
+ *   k_new, v_new  nullable [B][Hkv][d] cache dtype: the step's new key and
+ *              value.  When given they are appended first, exactly as
+ *              aqua_project_keys(cache, k_new, v_new, P, 1) would (slot len[b],
+ *              len[b] += 1, cache->max_len += 1), inside the same launch that
+ *              projects the queries, so the step sees its own token.  When NULL
+ *              the caller appended the step's key beforehand.
  *   P          [Hkv][d][d] f32
  *   k          dimensions kept per query head, 1 <= k <= d_store
  *   scale      score scale; <= 0 selects 1/sqrt(d) (d = full head dim)
@@ -157,12 +163,13 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  *   lse_out    nullable [B][Hq] f32: log-sum-exp of the scores
  * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4}.  A sequence with
  * len[b] = 0 gets a zero output and lse = -inf.
+ * Errors: AQUA_ERR_ARG if only one of k_new, v_new is given or the cache is full.
  */
 AQUA_API size_t aqua_decode_workspace_size(const aqua_cache* cache, int Hq);
-AQUA_API int aqua_decode_attn(const aqua_cache* cache, const void* q, const float* P, int Hq, int k,
-                     float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out,
-                     float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
-                     aqua_stream_t stream);
+AQUA_API int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_new, const void* v_new,
+                              const float* P, int Hq, int k, float scale, void* out, int out_dtype,
+                              int32_t* sel_out, float* qproj_out, float* scores_out, float* lse_out,
+                              void* workspace, size_t workspace_bytes, aqua_stream_t stream);
 
 /*
  * Causal AQUA attention for a chunk of L prompt tokens at absolute positions

@@ -140,6 +140,9 @@ def attend_one(qt, k: int, Kt, V, scale: float, m: int | None = None):
     unprojected values V [T, d].
     """
     S = select_dims(qt, k, m)
+    if len(Kt) == 0:
+        # no visible token: the weighted sum is empty (zero) and log(sum exp) = -inf
+        return np.zeros(np.shape(V)[-1]), np.zeros(0), -np.inf, S
     s = sparse_scores(qt, S, Kt, scale)
     p, lse = softmax(s)
     return p @ np.asarray(V, dtype=np.float64), p, lse, S

@@ -73,7 +73,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "aqua_calibrate": (c_int, [P, c_int, c_int, P, P, P, c_size_t, P]),
         "aqua_project_keys": (c_int, [C, P, P, P, c_int, P]),
         "aqua_decode_workspace_size": (c_size_t, [C, c_int]),
-        "aqua_decode_attn": (c_int, [C, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
+        "aqua_decode_attn": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
         "aqua_prefill_workspace_size": (c_size_t, [C, c_int, c_int]),
         "aqua_prefill_attn": (c_int, [C, P, c_int, c_int, P, c_int, c_int, c_float, P, c_int, P, P, c_size_t, P]),
         "aqua_h2o_update": (c_int, [C, P, P, c_int, c_int, c_int, P, P]),
@@ -142,11 +142,13 @@ def aqua_decode_workspace_size(cache: aqua_cache, Hq: int) -> int:
 
 
 def aqua_decode_attn(cache: aqua_cache, q, P, Hq: int, k: int, out, workspace, scale: float = 0.0,
-                     sel_out=None, qproj_out=None, scores_out=None, lse_out=None, stream=None) -> None:
+                     k_new=None, v_new=None, sel_out=None, qproj_out=None, scores_out=None, lse_out=None,
+                     stream=None) -> None:
+    """One decode step; with k_new/v_new ([B, Hkv, d]) the step's token is appended first."""
     out_dtype = AQUA_BF16 if str(out.dtype) == "torch.bfloat16" else AQUA_F32
     _check(load_library().aqua_decode_attn(
-        ctypes.byref(cache), _ptr(q), _ptr(P), Hq, k, scale, _ptr(out), out_dtype, _ptr(sel_out),
-        _ptr(qproj_out), _ptr(scores_out), _ptr(lse_out), _ptr(workspace),
+        ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(P), Hq, k, scale, _ptr(out), out_dtype,
+        _ptr(sel_out), _ptr(qproj_out), _ptr(scores_out), _ptr(lse_out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

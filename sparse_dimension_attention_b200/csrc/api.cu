@@ -5,6 +5,9 @@
 #include <cstdint>
 #include <cstdio>
 
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "aqua_internal.cuh"
 
 namespace aqua {
@@ -36,13 +39,37 @@ int device_sm_count() {
   return n;
 }
 
+int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                        uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (encode == nullptr) return set_error(AQUA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(AQUA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return AQUA_OK;
+}
+
 // launchers (defined next to their kernels)
 int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
                         cudaStream_t st);
 size_t decode_workspace_bytes(int n_units, int G);
 int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale,
                   void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
-                  float* lse_out, void* ws, cudaStream_t st);
+                  float* lse_out, const void* k_new, const void* v_new, void* ws, cudaStream_t st);
 size_t prefill_workspace_bytes(const aqua_cache* c, int Hq, int L);
 int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const float* P, int Hq, int k,
                    float scale, void* out, int out_dtype, int32_t* sel_out, void* ws, cudaStream_t st);
@@ -94,7 +121,7 @@ extern "C" {
 
 const char* aqua_last_error(void) { return aqua::g_err; }
 
-int aqua_version(void) { return 1; }
+int aqua_version(void) { return 2; }
 
 int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream) {
   if (cache == nullptr || cache->ctrl == nullptr || status_out == nullptr)
@@ -156,9 +183,10 @@ size_t aqua_decode_workspace_size(const aqua_cache* cache, int Hq) {
   return aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv);
 }
 
-int aqua_decode_attn(const aqua_cache* cache, const void* q, const float* P, int Hq, int k, float scale,
-                     void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
-                     float* lse_out, void* workspace, size_t workspace_bytes, aqua_stream_t stream) {
+int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_new, const void* v_new, const float* P,
+                     int Hq, int k, float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out,
+                     float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
+                     aqua_stream_t stream) {
   aqua::g_err[0] = '\0';
   int rc = validate_cache(cache);
   if (rc != AQUA_OK) return rc;
@@ -177,9 +205,20 @@ int aqua_decode_attn(const aqua_cache* cache, const void* q, const float* P, int
   const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, G);
   if (workspace_bytes < need)
     return set_error(AQUA_ERR_WORKSPACE, "aqua_decode_attn: workspace %zu < %zu bytes", workspace_bytes, need);
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k_new and v_new must both be given or both be NULL");
+  if (k_new != nullptr) {
+    if ((long long)cache->max_len + 1 > cache->Tcap)
+      return set_error(AQUA_ERR_ARG, "aqua_decode_attn: appending to a full cache (max_len %d, Tcap %d)",
+                       cache->max_len, cache->Tcap);
+    if (!aligned(k_new, 16) || !aligned(v_new, 16))
+      return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k_new, v_new must be 16-byte aligned");
+  }
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)cache->d);
-  return aqua::launch_decode(cache, q, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, scores_out, lse_out,
-                             workspace, reinterpret_cast<cudaStream_t>(stream));
+  rc = aqua::launch_decode(cache, q, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, scores_out, lse_out,
+                           k_new, v_new, workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (rc == AQUA_OK && k_new != nullptr) cache->max_len += 1;
+  return rc;
 }
 
 size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L) {

@@ -1,24 +1,36 @@
 // AQUA decode step on sm_100a.
 //
-// Kernel 1 (qproj_topk_kernel), one CTA per (sequence b, KV head g), one warp
-// per query head of the group:
-//   q~ = q P                                  (abstract: "project query ... vectors")
-//   S_h = k largest |q~_j|, ties to lower j  (edgentiq, Online Inference: "highest
-//                                             'magnitude' in the projected query")
-//   U_g = union of the group's S_h, and the masked, pre-scaled query rows
-//   qm[r][h] = (j_r in S_h) ? q~_h[j_r] * scale * log2(e) : 0 for j_r = U_g[r].
+// qproj_topk_kernel -- one CTA per (sequence b, KV head g), one warp per query
+// head of the group (P[g] staged in shared memory by one bulk copy), plus one
+// warp that appends the step's new key and value when the call carries them
+// (k~ = k P rounded to the cache type, written at slot len[b]; the last CTA
+// advances the lengths):
+//   q~ = q P                                  (abstract: "project query and key vectors")
+//   S_h = k largest |q~_j|, ties to lower j  (edgentiq, Online Inference: the dimensions
+//                                             with the highest "magnitude" in the projected query)
+//   U_g = union of the group's S_h and the masked, pre-scaled query rows
+//   qm[r][h] = (U_r in S_h) ? q~_h[U_r] * scale * log2(e) : 0.
 //
-// Kernel 2 (decode_attn_kernel), persistent, one CTA per SM.  The cached
-// tokens of all (b, g) units are cut into tiles of TT tokens and the flat tile
-// sequence is split evenly over the CTAs.  Per tile a producer warp gathers the
-// |U_g| selected rows of the dimension-major K~ cache and the V tile into shared
-// memory with bulk asynchronous copies (one union read per GQA group), three
-// stages deep; eight consumer warps compute
-//   s_{h,t} = sum_{r} qm[r][h] K~[U_r][t]       (scores on the selected dims only)
-// followed by an online softmax and o_h += p_{h,t} V_t (unprojected V).  A CTA
-// that finishes a partial unit writes (m, l, o) and takes a ticket; the last
-// CTA of a unit merges the partials (log-sum-exp) and writes the output.  No
-// CTA ever waits for another.
+// decode_attn_*_kernel -- persistent, one CTA per SM.  The cached tokens of all
+// (b, g) units are cut into tiles of TT tokens and the flat tile sequence is
+// split evenly over the CTAs.  Per tile a producer warp gathers the |U_g|
+// selected rows of the dimension-major K~ cache (one union read per GQA group)
+// and the V tile into shared memory with asynchronous bulk / tensor copies,
+// three stages deep.  Consumer warps compute the scores on the selected
+// dimensions only, s_{h,t} = sum_r qm[r][h] K~[U_r][t], an online softmax, and
+// o_h += p_{h,t} V_t over the unprojected values (AQUA abstract; edgentiq,
+// "How AQUA Works").  A CTA that ends inside a unit writes (m, l, o) and takes
+// a ticket; the unit's last CTA merges the partials (log-sum-exp).  No CTA
+// ever waits for another.
+//
+// bf16 caches: the consumers use the tensor cores (mma.sync m16n8k16, bf16 in,
+// f32 accumulate).  q~ and p are split into bf16 high and low parts (rows
+// 0..G-1 and 8..8+G-1 of the 16-row A operand), so the products keep ~16
+// significant bits; each warp owns 16 tokens of every tile and keeps its own
+// running max, merged at the end of a segment.  The K~ rows are gathered with
+// 16-byte cp.async by four producer warps (many small bulk copies from one warp
+// cannot keep HBM busy); the V tile arrives by a 128B-swizzled tensor copy.
+// f32 caches: CUDA-core FMA consumers (exact f32 products).
 #include <math.h>
 
 #include "aqua_internal.cuh"
@@ -32,8 +44,12 @@ constexpr int NCW = 8;                 // consumer warps
 constexpr int NCT = NCW * 32;          // consumer threads
 constexpr int NTHREADS = NCT + 32;     // + one producer warp
 constexpr int NSTAGE = 3;
-constexpr int RMAX = D / NCW;          // union rows per consumer warp
+constexpr int RMAX = D / NCW;          // union rows per consumer warp (f32 kernel)
 constexpr int kMaxCtas = 1024;
+constexpr int KROW_BF16 = 272;         // padded byte stride of a K~ row in shared memory (bf16 kernel)
+constexpr float kLazyRescale = 8.0f;   // running max is raised only when exceeded by 2^8
+constexpr int NPW_BF16 = 4;            // producer warps of the bf16 kernel (K~ gather by 16-byte cp.async)
+constexpr int NTHREADS_BF16 = NCT + NPW_BF16 * 32;
 
 struct DecodeParams {
   const void* q;
@@ -53,33 +69,17 @@ struct DecodeParams {
   float* scores_out;
   float* lse_out;
   int32_t* ctrl;
+  // optional fused append of the step's new token (k_new == nullptr: none)
+  const void* k_new;      // [B][Hkv][D] cache dtype
+  const void* v_new;      // [B][Hkv][D]
+  int32_t* len_w;         // == len, written by the append ticket
+  int32_t* n_abs;
+  int32_t* pos;
+  float* score;
   int B, Hq, Hkv, d_store, Tcap, k;
   int out_bf16;
   float scale_log2;
 };
-
-template <typename T> struct Tile;
-template <> struct Tile<__nv_bfloat16> { static constexpr int TT = 128; };
-template <> struct Tile<float> { static constexpr int TT = 64; };
-
-// ------------------------------------------------------------------ small loads
-template <typename T, int N>
-__device__ __forceinline__ void load_row(const T* p, float (&f)[N]);
-template <>
-__device__ __forceinline__ void load_row<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&f)[4]) {
-  const uint2 w = *reinterpret_cast<const uint2*>(p);
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-}
-template <>
-__device__ __forceinline__ void load_row<float, 4>(const float* p, float (&f)[4]) {
-  const float4 v = *reinterpret_cast<const float4*>(p);
-  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void load_row<float, 2>(const float* p, float (&f)[2]) {
-  const float2 v = *reinterpret_cast<const float2*>(p);
-  f[0] = v.x; f[1] = v.y;
-}
 
 // cached tokens of sequence b, clamped to the cache capacity (lengths are caller-owned device data)
 __device__ __forceinline__ int seq_len(const int32_t* len, int b, int Tcap) { return min(max(len[b], 0), Tcap); }
@@ -95,125 +95,180 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
+__device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, float v) {
+  if (p.out_bf16)
+    static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+  else
+    static_cast<float*>(p.out)[idx] = v;
+}
+
 // ============================================================================
-// Kernel 1: query projection + magnitude top-k + group union
+// query projection + magnitude top-k + group union
 // ============================================================================
 template <typename T, int G>
-__global__ void __launch_bounds__(G * 32) qproj_topk_kernel(DecodeParams p) {
+__global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p) {
+  extern __shared__ __align__(128) float Ps[];   // P[g], [D][D]
   __shared__ float qs[G][D];
   __shared__ uint32_t masks[G][4];
+  __shared__ __align__(8) uint64_t pbar;
+  __shared__ int is_last;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, g = u % p.Hkv;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = g * G + w;
+  const int h = g * G + (w < G ? w : 0);
   const int m = p.d_store;
+  const bool append = p.k_new != nullptr;
+  const int len_before = __ldcg(p.len + b);   // read before the append ticket below
 
+  if (threadIdx.x == 0) {
+    mbar_init(&pbar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&pbar, D * D * 4);
+    bulk_g2s_plain(Ps, p.P + (size_t)g * D * D, D * D * 4, &pbar);
+  }
   const T* qrow = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D;
   float qv[4];
 #pragma unroll
   for (int s = 0; s < 4; ++s) qv[s] = Elem<T>::load(qrow + 4 * lane + s);
-
-  // q~_j for j = 4*lane + s
-  float qt[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* Pg = p.P + (size_t)g * D * D;
-#pragma unroll 8
-  for (int i = 0; i < D; ++i) {
-    const float qi = __shfl_sync(0xffffffffu, qv[i & 3], i >> 2);
-    const float4 pr = __ldg(reinterpret_cast<const float4*>(Pg + (size_t)i * D) + lane);
-    qt[0] = fmaf(qi, pr.x, qt[0]);
-    qt[1] = fmaf(qi, pr.y, qt[1]);
-    qt[2] = fmaf(qi, pr.z, qt[2]);
-    qt[3] = fmaf(qi, pr.w, qt[3]);
+  const bool ok = mbar_wait_bounded(&pbar, 0);
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+    return;
   }
 
-  // Keys: magnitude bits + 1 for candidate dims (j < m), 0 otherwise, so that
-  // unsigned order equals |q~| order and non-candidates rank below everything.
-  uint32_t key[4];
+  if (w == G) {
+    // ---- fused append of the new token of unit (b, g)
+    if (append) {
+      const int slot = len_before;
+      if (slot < 0 || slot >= p.Tcap) {
+        if (lane == 0) record_status(p.ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
+      } else {
+        const T* kr = static_cast<const T*>(p.k_new) + (size_t)u * D;
+        float kv[4];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int j = 4 * lane + s;
-    key[s] = (j < m) ? (__float_as_uint(fabsf(qt[s])) + 1u) : 0u;
-  }
-  // Radix select of the k-th largest key: the largest tau with #{key >= tau} >= k.
-  uint32_t tau = 0;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = tau | (1u << bit);
-    int c = 0;
+        for (int s2 = 0; s2 < 4; ++s2) kv[s2] = Elem<T>::load(kr + 4 * lane + s2);
+        float kt[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+        for (int i = 0; i < D; ++i) {
+          const float ki = __shfl_sync(0xffffffffu, kv[i & 3], i >> 2);
+          const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
+          kt[0] = fmaf(ki, pr.x, kt[0]);
+          kt[1] = fmaf(ki, pr.y, kt[1]);
+          kt[2] = fmaf(ki, pr.z, kt[2]);
+          kt[3] = fmaf(ki, pr.w, kt[3]);
+        }
+        T* kp = const_cast<T*>(static_cast<const T*>(p.kproj)) + (size_t)u * p.d_store * p.Tcap + slot;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) c += (key[s] >= cand);
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= p.k) tau = cand;
-  }
-  int ngt = 0, neq = 0;
+        for (int s2 = 0; s2 < 4; ++s2) {
+          const int jd = 4 * lane + s2;
+          if (jd < p.d_store) kp[(size_t)jd * p.Tcap] = Elem<T>::from_f32(kt[s2]);
+        }
+        T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * D;
+        const T* vr = static_cast<const T*>(p.v_new) + (size_t)u * D;
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    ngt += (key[s] > tau);
-    neq += (key[s] == tau);
-  }
-  const int need = p.k - __reduce_add_sync(0xffffffffu, ngt);  // ties to take, lowest index first
-  // exclusive prefix of equal-key counts over lanes (index order = lane-major)
-  int incl = neq;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  int rank = incl - neq;
-  bool sel[4];
-  int nsel = 0;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    sel[s] = key[s] > tau;
-    if (key[s] == tau) {
-      sel[s] = rank < need;
-      ++rank;
+        for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = vr[4 * lane + s2];
+        if (p.pos != nullptr && lane == 0) {
+          p.pos[(size_t)u * p.Tcap + slot] = __ldcg(p.n_abs + b);
+          p.score[(size_t)u * p.Tcap + slot] = 0.f;
+        }
+      }
     }
-    nsel += sel[s];
-  }
-  // ascending output position of each selected dim
-  int pincl = nsel;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, pincl, o);
-    if (lane >= o) pincl += y;
-  }
-  int opos = pincl - nsel;
-  const size_t bh = (size_t)b * p.Hq + h;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int j = 4 * lane + s;
-    if (sel[s]) {
-      if (p.sel_out) p.sel_out[bh * p.k + opos] = j;
-      ++opos;
+  } else {
+    // q~_j for j = 4*lane + s
+    float qt[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll 16
+    for (int i = 0; i < D; ++i) {
+      const float qi = __shfl_sync(0xffffffffu, qv[i & 3], i >> 2);
+      const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
+      qt[0] = fmaf(qi, pr.x, qt[0]);
+      qt[1] = fmaf(qi, pr.y, qt[1]);
+      qt[2] = fmaf(qi, pr.z, qt[2]);
+      qt[3] = fmaf(qi, pr.w, qt[3]);
     }
-    if (p.qproj_out) p.qproj_out[bh * D + j] = qt[s];
-    qs[w][j] = sel[s] ? qt[s] * p.scale_log2 : 0.f;
-  }
-  // 128-bit selection mask of this head
-  const uint32_t nib = (uint32_t)sel[0] | ((uint32_t)sel[1] << 1) | ((uint32_t)sel[2] << 2) |
-                       ((uint32_t)sel[3] << 3);
-  const uint32_t shifted = nib << (4 * (lane & 7));
-#pragma unroll
-  for (int wd = 0; wd < 4; ++wd) {
-    const uint32_t word = __reduce_or_sync(0xffffffffu, (lane >> 3) == wd ? shifted : 0u);
-    if (lane == 0) masks[w][wd] = word;
+
+    // Keys: magnitude bits + 1 for candidate dims (j < m), 0 otherwise, so that
+    // unsigned order equals |q~| order and non-candidates rank below everything.
+    uint32_t key[4];
+  #pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int j = 4 * lane + s;
+      key[s] = (j < m) ? (__float_as_uint(fabsf(qt[s])) + 1u) : 0u;
+    }
+    // Radix select of the k-th largest key: the largest tau with #{key >= tau} >= k.
+    uint32_t tau = 0;
+  #pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = tau | (1u << bit);
+      int c = 0;
+  #pragma unroll
+      for (int s = 0; s < 4; ++s) c += (key[s] >= cand);
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= p.k) tau = cand;
+    }
+    int ngt = 0, neq = 0;
+  #pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      ngt += (key[s] > tau);
+      neq += (key[s] == tau);
+    }
+    const int need = p.k - __reduce_add_sync(0xffffffffu, ngt);  // ties to take, lowest index first
+    int incl = neq;
+  #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int rank = incl - neq;
+    bool sel[4];
+    int nsel = 0;
+  #pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      sel[s] = key[s] > tau;
+      if (key[s] == tau) {
+        sel[s] = rank < need;
+        ++rank;
+      }
+      nsel += sel[s];
+    }
+    int pincl = nsel;
+  #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, pincl, o);
+      if (lane >= o) pincl += y;
+    }
+    int opos = pincl - nsel;
+    const size_t bh = (size_t)b * p.Hq + h;
+  #pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int j = 4 * lane + s;
+      if (sel[s]) {
+        if (p.sel_out) p.sel_out[bh * p.k + opos] = j;
+        ++opos;
+      }
+      if (p.qproj_out) p.qproj_out[bh * D + j] = qt[s];
+      qs[w][j] = sel[s] ? qt[s] * p.scale_log2 : 0.f;
+    }
+    const uint32_t nib = (uint32_t)sel[0] | ((uint32_t)sel[1] << 1) | ((uint32_t)sel[2] << 2) |
+                         ((uint32_t)sel[3] << 3);
+    const uint32_t shifted = nib << (4 * (lane & 7));
+  #pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      const uint32_t word = __reduce_or_sync(0xffffffffu, (lane >> 3) == wd ? shifted : 0u);
+      if (lane == 0) masks[w][wd] = word;
+    }
   }
 
   // sequences with no tokens: zero output, lse = -inf
-  const int T_b = seq_len(p.len, b, p.Tcap);
-  if (T_b <= 0) {
-    for (int j = lane; j < D; j += 32) {
-      if (p.out_bf16)
-        static_cast<__nv_bfloat16*>(p.out)[bh * D + j] = __float2bfloat16_rn(0.f);
-      else
-        static_cast<float*>(p.out)[bh * D + j] = 0.f;
-    }
+  if (w < G && !append && seq_len(p.len, b, p.Tcap) <= 0) {
+    const size_t bh = (size_t)b * p.Hq + h;
+    for (int j = lane; j < D; j += 32) store_val(p, bh * D + j, 0.f);
     if (p.lse_out && lane == 0) p.lse_out[bh] = -INFINITY;
   }
   __syncthreads();
 
-  // group union U_g (ascending) and the masked query rows over it
   uint32_t um[4];
 #pragma unroll
   for (int wd = 0; wd < 4; ++wd) {
@@ -222,7 +277,7 @@ __global__ void __launch_bounds__(G * 32) qproj_topk_kernel(DecodeParams p) {
     for (int hh = 0; hh < G; ++hh) x |= masks[hh][wd];
     um[wd] = x;
   }
-  for (int j = threadIdx.x; j < D; j += G * 32) {
+  for (int j = threadIdx.x; j < D; j += blockDim.x) {
     const int wd = j >> 5, bit = j & 31;
     if ((um[wd] >> bit) & 1u) {
       int r = __popc(um[wd] & ((1u << bit) - 1u));
@@ -237,10 +292,26 @@ __global__ void __launch_bounds__(G * 32) qproj_topk_kernel(DecodeParams p) {
     p.ucount[u] = __popc(um[0]) + __popc(um[1]) + __popc(um[2]) + __popc(um[3]);
     p.counters[u] = 0;
   }
+  if (!append) return;
+  // every CTA has read len[b]; the last one advances the lengths
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    is_last = (atomicAdd(p.ctrl + kCtrlAppendTicket, 1) == (int)gridDim.x - 1);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int bb = threadIdx.x; bb < p.B; bb += blockDim.x) {
+      p.len_w[bb] += 1;
+      if (p.n_abs) p.n_abs[bb] += 1;
+    }
+    if (threadIdx.x == 0) p.ctrl[kCtrlAppendTicket] = 0;
+  }
 }
 
 // ============================================================================
-// Kernel 2: persistent split-K sparse-dimension attention
+// shared pieces of the attention kernels
 // ============================================================================
 struct StageHdr {
   int u;       // unit b*Hkv + g
@@ -260,10 +331,12 @@ __device__ __forceinline__ int cta_of_tile(long long t, long long N, int C) {
   return (int)(c < C - 1 ? c : C - 1);
 }
 
-// exclusive scan over all NTHREADS threads; *total receives the sum
+// exclusive scan over all NT threads of the block; *total receives the sum
+template <int NT>
 __device__ __forceinline__ long long block_excl_scan(long long v, long long* sh, long long* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int NW = NTHREADS / 32;
+  constexpr int NW = NT / 32;
+  static_assert(NW <= 32, "scan uses one warp for the warp totals");
   long long x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -289,62 +362,31 @@ __device__ __forceinline__ long long block_excl_scan(long long v, long long* sh,
   return excl;
 }
 
-template <typename T, int G>
-struct DecodeSmem {
-  static constexpr int TT = Tile<T>::TT;
-  static constexpr int KBYTES = D * TT * (int)sizeof(T);
-  static constexpr int VBYTES = TT * D * (int)sizeof(T);
-  static constexpr int STAGE = KBYTES + VBYTES;
-  static constexpr int RW = TT > D ? TT : D;
-  static constexpr int SLOTS = (G * TT + NCT - 1) / NCT;
-  static constexpr int OFF_RED = NSTAGE * STAGE;
-  static constexpr int OFF_PSM = OFF_RED + NCW * G * RW * 4;
-  static constexpr int OFF_WST = OFF_PSM + TT * G * 4;
-  static constexpr int OFF_HDR = OFF_WST + 2 * SLOTS * NCW * 4;
-  static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
-  static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int BYTES = OFF_SCH + 16 * 8;
+struct Sched {
+  long long N, my_start, my_end;
+  int C;
+  int u0;
+  long long ts0, sb0;
 };
 
-template <typename T, int G>
-__global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p) {
-  using S = DecodeSmem<T, G>;
-  constexpr int TT = S::TT;
-  constexpr int TPL = TT / 32;        // tokens per lane in the score pass
-  constexpr int TPW = TT / NCW;       // tokens per warp in the PV pass
-  constexpr int EPV = 16 / (int)sizeof(T);   // elements per 16-byte vector
-
-  extern __shared__ __align__(1024) unsigned char smem[];
-  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
-  float* psm = reinterpret_cast<float*>(smem + S::OFF_PSM);
-  float* wmax = reinterpret_cast<float*>(smem + S::OFF_WST);
-  float* wsum = wmax + S::SLOTS * NCW;
-  StageHdr* hdr = reinterpret_cast<StageHdr*>(smem + S::OFF_HDR);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-  uint64_t* empty = full + NSTAGE;
-  long long* sch = reinterpret_cast<long long*>(smem + S::OFF_SCH);
-
+// Flat tile range of this CTA and its first unit.  Returns false (for the
+// whole CTA) when the CTA has no tile.  `scratch` needs 32 long longs.
+template <int TT, int NT>
+__device__ bool make_schedule(const DecodeParams& p, long long* scratch, long long* sch, Sched& S) {
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
   const int n_units = p.B * p.Hkv;
-  const int C = gridDim.x, c = blockIdx.x;
-
-  if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NCW);
-    }
-    fence_barrier_init();
-  }
-
-  // ---------------- schedule: flat tile range of this CTA and its first unit
-  long long* scan_sh = reinterpret_cast<long long*>(smem);  // stage memory is free until the producer starts
-  const int chunk = (n_units + NTHREADS - 1) / NTHREADS;
+  const int c = blockIdx.x;
+  const int chunk = (n_units + NT - 1) / NT;
   const int u_lo = min(n_units, tid * chunk), u_hi = min(n_units, u_lo + chunk);
   long long my_tiles = 0;
   for (int u = u_lo; u < u_hi; ++u) my_tiles += (seq_len(p.len, u / p.Hkv, p.Tcap) + TT - 1) / TT;
   long long N;
-  const long long t_excl = block_excl_scan(my_tiles, scan_sh, &N);
+  const long long t_excl = block_excl_scan<NT>(my_tiles, scratch, &N);
+  // Effective grid: never more CTAs than tiles, so every CTA owns at least one
+  // tile and the CTAs covering a unit are consecutive (the ticket count relies
+  // on it).  The host sizes the grid from an upper bound of the lengths.
+  const int C = (int)min((long long)gridDim.x, N);
+  if (c >= C) return false;
   const long long my_start = (long long)c * N / C, my_end = (long long)(c + 1) * N / C;
   long long my_segs = 0;
   {
@@ -356,7 +398,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
     }
   }
   long long NS;
-  const long long s_excl = block_excl_scan(my_segs, scan_sh, &NS);
+  const long long s_excl = block_excl_scan<NT>(my_segs, scratch, &NS);
   {
     long long ts = t_excl, sb = s_excl;
     for (int u = u_lo; u < u_hi; ++u) {
@@ -371,48 +413,211 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
     }
   }
   __syncthreads();
-  if (my_start >= my_end) return;
-  const int n_tiles = (int)(my_end - my_start);
+  S.N = N;
+  S.C = C;
+  S.my_start = my_start;
+  S.my_end = my_end;
+  S.u0 = (int)sch[0];
+  S.ts0 = sch[1];
+  S.sb0 = sch[2];
+  return true;
+}
 
-  if (warp == NCW) {
-    // ======================= producer warp =======================
-    const uint64_t pol = policy_evict_first();
-    int u = (int)sch[0];
-    long long ts = sch[1], sb = sch[2];
-    int b = u / p.Hkv;
-    int Tb = seq_len(p.len, b, p.Tcap);
-    long long te = ts + (Tb + TT - 1) / TT;
-    int cf = cta_of_tile(ts, N, C);
-    int nseg = cta_of_tile(te - 1, N, C) - cf + 1;
-    int nU = p.ucount[u];
-    int urow[D / 32];
+// Walks the units of this CTA's tile range; one instance per producer warp.
+struct UnitWalker {
+  int u, b, Tb, nU, nseg, cf;
+  long long ts, te, sb;
+  template <int TT>
+  __device__ void start(const DecodeParams& p, const Sched& S) {
+    u = S.u0;
+    ts = S.ts0;
+    sb = S.sb0;
+    b = u / p.Hkv;
+    Tb = seq_len(p.len, b, p.Tcap);
+    te = ts + (Tb + TT - 1) / TT;
+    cf = cta_of_tile(ts, S.N, S.C);
+    nseg = cta_of_tile(te - 1, S.N, S.C) - cf + 1;
+    nU = p.ucount[u];
+  }
+  // advance to the unit holding flat tile t; true when the unit changed
+  template <int TT>
+  __device__ bool seek(const DecodeParams& p, const Sched& S, long long t) {
+    bool changed = false;
+    while (t >= te) {
+      sb += nseg;
+      ++u;
+      b = u / p.Hkv;
+      Tb = seq_len(p.len, b, p.Tcap);
+      ts = te;
+      te = ts + (Tb + TT - 1) / TT;
+      if (te > ts) {
+        cf = cta_of_tile(ts, S.N, S.C);
+        nseg = cta_of_tile(te - 1, S.N, S.C) - cf + 1;
+        nU = p.ucount[u];
+      } else {
+        nseg = 0;
+      }
+      changed = true;
+    }
+    return changed;
+  }
+  __device__ StageHdr header(const Sched& S, long long t, int TT) const {
+    StageHdr hh;
+    hh.u = u;
+    hh.t0 = (int)(t - ts) * TT;
+    hh.nvalid = min(TT, Tb - hh.t0);
+    hh.nU = nU;
+    hh.flags = ((t == S.my_start || t == ts) ? kFirst : 0) | ((t == S.my_end - 1 || t == te - 1) ? kLast : 0);
+    hh.seg = nseg > 1 ? (int)(sb + (blockIdx.x - cf)) : -1;
+    hh.nseg = nseg;
+    hh.seg0 = (int)sb;
+    return hh;
+  }
+};
+
+// Segment result (M, L per head; O unnormalised in shared memory, [G][D]) ->
+// output, or partial + ticket + merge by the unit's last CTA.  Called by all
+// consumer threads; thread idx handles (h, dim) = (idx / D, idx % D).
+template <int G>
+__device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int tid, const float (&Mh)[G],
+                               const float (&Lh)[G], const float* Oacc, int* s_last) {
+  const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
+  const size_t bhq0 = (size_t)b * p.Hq + g * G;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = lane + 32 * i;
-      urow[i] = r < nU ? p.ulist[(size_t)u * D + r] : 0;
+  for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+    const int idx = tid + NCT * i;
+    if (idx < G * D) {
+      const int h = idx / D, dim = idx % D;
+      float lh = 0.f;
+#pragma unroll
+      for (int x = 0; x < G; ++x)
+        if (x == h) lh = Lh[x];
+      const float o = Oacc[h * D + dim];
+      if (hh.seg < 0)
+        store_val(p, (bhq0 + h) * D + dim, o / lh);
+      else
+        p.part_o[((size_t)hh.seg * G + h) * D + dim] = o;
+    }
+  }
+  if (tid < G) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      if (h == tid) {
+        if (hh.seg < 0) {
+          if (p.lse_out) p.lse_out[bhq0 + h] = (Mh[h] + log2f(Lh[h])) * kLn2;
+        } else {
+          p.part_ml[((size_t)hh.seg * G + h) * 2 + 0] = Mh[h];
+          p.part_ml[((size_t)hh.seg * G + h) * 2 + 1] = Lh[h];
+        }
+      }
+  }
+  if (hh.seg < 0) return;
+  // publish this partial, take a ticket; the unit's last arrival merges
+  __threadfence();
+  named_bar_sync(1, NCT);
+  if (tid == 0) *s_last = (atomicAdd(p.counters + hh.u, 1) == hh.nseg - 1);
+  named_bar_sync(1, NCT);
+  if (!*s_last) return;
+  __threadfence();
+#pragma unroll 1
+  for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+    const int idx = tid + NCT * i;
+    if (idx >= G * D) break;
+    const int h = idx / D, dim = idx % D;
+    float M = -INFINITY;
+#pragma unroll 1
+    for (int sg = 0; sg < hh.nseg; ++sg) M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(hh.seg0 + sg) * G + h) * 2));
+    float Lsum = 0.f, O = 0.f;
+#pragma unroll 1
+    for (int sg = 0; sg < hh.nseg; ++sg) {
+      const size_t slot = (size_t)(hh.seg0 + sg) * G + h;
+      const float f = exp2f(__ldcg(p.part_ml + slot * 2) - M);
+      Lsum = fmaf(f, __ldcg(p.part_ml + slot * 2 + 1), Lsum);
+      O = fmaf(f, __ldcg(p.part_o + slot * D + dim), O);
+    }
+    store_val(p, (bhq0 + h) * D + dim, O / Lsum);
+    if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M + log2f(Lsum)) * kLn2;
+  }
+  if (tid == 0) p.counters[hh.u] = 0;
+}
+
+// ============================================================================
+// bf16 cache: tensor-core consumers
+// ============================================================================
+template <int G>
+struct SmemBF16 {
+  static constexpr int TT = 128;
+  static constexpr int VHALF = TT * 128;                // [TT tokens][64 dims] bf16, 128B-swizzled
+  static constexpr int KBYTES = D * KROW_BF16;          // [128 rows][272 B]
+  static constexpr int STAGE = 2 * VHALF + KBYTES;      // multiple of 1024
+  static constexpr int OFF_RED = NSTAGE * STAGE;        // [NCW][G][D] f32
+  static constexpr int OFF_ML = OFF_RED + NCW * G * D * 4;   // [NCW][G][2] f32
+  static constexpr int OFF_HDR = OFF_ML + NCW * G * 2 * 4;
+  static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
+  static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
+  static constexpr int OFF_MISC = OFF_SCH + 36 * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+};
+
+template <int G>
+__global__ void __launch_bounds__(NTHREADS_BF16, 1)
+    decode_attn_bf16_kernel(const __grid_constant__ CUtensorMap tmap_v, DecodeParams p) {
+  using S = SmemBF16<G>;
+  constexpr int TT = S::TT;
+  static_assert(G <= 8, "head rows 0..G-1 (high parts) and 8..8+G-1 (low parts)");
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
+  float* mlb = reinterpret_cast<float*>(smem + S::OFF_ML);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* empty = full + NSTAGE;
+  long long* sch = reinterpret_cast<long long*>(smem + S::OFF_SCH);
+  int* s_last = reinterpret_cast<int*>(smem + S::OFF_MISC);   // [0]: merge ticket, [1]: timeout flag
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) s_last[1] = 0;
+
+  // shared memory starts zeroed: padding rows and never-copied tokens must be finite
+  for (int i = tid; i < NSTAGE * S::STAGE / 16; i += NTHREADS_BF16)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      // arrivals: one cp.async arrival per producer thread + the V tensor-copy arrival
+      mbar_init(&full[s], NPW_BF16 * 32 + 1);
+      mbar_init(&empty[s], NCW);
+    }
+    fence_barrier_init();
+  }
+  Sched Sd;
+  if (!make_schedule<TT, NTHREADS_BF16>(p, sch + 4, sch, Sd)) return;
+  fence_proxy_async_smem();
+  __syncthreads();
+  const int n_tiles = (int)(Sd.my_end - Sd.my_start);
+
+  if (warp >= NCW) {
+    // ======================= producer warps =======================
+    // Thread pt copies 16-byte chunk (pt & 15) of union rows (pt >> 4) + 8 j,
+    // j = 0..15, of every tile; producer thread 0 also issues the V tile.
+    const int pt = tid - NCT;
+    const int chunk = pt & 15, r0 = pt >> 4;
+    const uint64_t pol = policy_evict_first();
+    if (pt == 0) prefetch_tmap(&tmap_v);
+    UnitWalker W;
+    W.start<TT>(p, Sd);
+    int urow[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int r = r0 + 8 * j;
+      urow[j] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
     }
     for (int it = 0; it < n_tiles; ++it) {
-      const long long t = my_start + it;
-      while (t >= te) {  // next non-empty unit
-        sb += nseg;
-        ++u;
-        b = u / p.Hkv;
-        Tb = seq_len(p.len, b, p.Tcap);
-        ts = te;
-        te = ts + (Tb + TT - 1) / TT;
-        if (te > ts) {
-          cf = cta_of_tile(ts, N, C);
-          nseg = cta_of_tile(te - 1, N, C) - cf + 1;
-        } else {
-          nseg = 0;
-        }
-        if (te > ts) {
-          nU = p.ucount[u];
+      const long long t = Sd.my_start + it;
+      if (W.seek<TT>(p, Sd, t)) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = lane + 32 * i;
-            urow[i] = r < nU ? p.ulist[(size_t)u * D + r] : 0;
-          }
+        for (int j = 0; j < 16; ++j) {
+          const int r = r0 + 8 * j;
+          urow[j] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
         }
       }
       const int s = it % NSTAGE;
@@ -425,42 +630,367 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
           return;
         }
       }
-      const int t0 = (int)(t - ts) * TT;
-      const int nvalid = min(TT, Tb - t0);
-      const int kvec = (nvalid + EPV - 1) / EPV * EPV;          // row copy in 16-byte units
-      const uint32_t kbytes = (uint32_t)kvec * sizeof(T);
-      const uint32_t vbytes = (uint32_t)nvalid * D * sizeof(T);
+      const StageHdr hh = W.header(Sd, t, TT);
+      unsigned char* st = smem + (size_t)s * S::STAGE;
+      if (pt == 0) {
+        mbar_arrive_expect_tx(&full[s], 2 * S::VHALF);
+        const int row = hh.u * p.Tcap + hh.t0;
+        tma_load_2d(st, &tmap_v, 0, row, &full[s], pol);
+        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[s], pol);
+      }
+      const int nch = (hh.nvalid + 7) / 8;                  // 16-byte groups of 8 tokens
+      if (chunk < nch) {
+        const __nv_bfloat16* kbase =
+            static_cast<const __nv_bfloat16*>(p.kproj) + (size_t)hh.u * p.d_store * p.Tcap + hh.t0 + chunk * 8;
+        unsigned char* ks = st + 2 * S::VHALF + chunk * 16;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int r = r0 + 8 * j;
+          if (r < hh.nU) cp_async16(ks + r * KROW_BF16, kbase + (size_t)urow[j] * p.Tcap, pol);
+        }
+      }
+      cp_async_arrive_noinc(&full[s]);
+    }
+    return;
+  }
+
+  // ======================= consumer warps =======================
+  // A-operand rows: row h < G carries the bf16 high part of head h, row 8 + h
+  // its low part; the thread holding row grp also holds row grp + 8.
+  const int grp = lane >> 2, q4 = lane & 3;    // mma fragment coordinates
+  const int tb = 16 * warp;                     // this warp's tokens in every tile
+  const bool head_row = grp < G;
+  uint32_t afr[8][4];
+  float o[16][4];
+  float mu = -INFINITY, ell = 0.f;
+  int cur_u = -1, nks = 0;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) afr[kk][0] = afr[kk][1] = afr[kk][2] = afr[kk][3] = 0u;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  // Every consumer warp walks the schedule itself, so all warps agree on the
+  // segment ends (where they synchronise) whatever happens to the data.  A
+  // warp whose wait runs out records the error, stops computing and keeps
+  // taking part in the segment-end barriers; the other warps follow it.
+  UnitWalker W;
+  W.start<TT>(p, Sd);
+  volatile int* dead_flag = s_last + 1;
+  bool dead = false;
+
+  for (int it = 0; it < n_tiles; ++it) {
+    const int s = it % NSTAGE;
+    const long long t = Sd.my_start + it;
+    W.seek<TT>(p, Sd, t);
+    const StageHdr hh = W.header(Sd, t, TT);
+    if (!dead) {
+      const bool ok = mbar_wait_bounded(&full[s], (it / NSTAGE) & 1);
+      const bool timed_out = __any_sync(0xffffffffu, !ok);     // warp-uniform decision
+      if (timed_out && lane == 0) {
+        *dead_flag = 1;
+        record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+      }
+      dead = timed_out || __any_sync(0xffffffffu, *dead_flag != 0);
+    }
+    unsigned char* st = smem + (size_t)s * S::STAGE;
+    const unsigned char* ks_base = st + 2 * S::VHALF;
+
+    if (!dead && (hh.flags & kFirst)) {
+      if (hh.u != cur_u) {
+        cur_u = hh.u;
+        nks = (hh.nU + 15) / 16;
+        const float* qmu = p.qm + (size_t)hh.u * D * G;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float hi2[2], lo2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = kk * 16 + half * 8 + 2 * q4 + e;
+              const float x = (head_row && col < hh.nU) ? __ldg(qmu + (size_t)col * G + grp) : 0.f;
+              split_bf16(x, hi2[e], lo2[e]);
+            }
+            afr[kk][half * 2] = pack_bf16(hi2[0], hi2[1]);       // row grp
+            afr[kk][half * 2 + 1] = pack_bf16(lo2[0], lo2[1]);   // row grp + 8
+          }
+        }
+      }
+      mu = -INFINITY;
+      ell = 0.f;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    }
+
+    bool wrote_smem = false;
+    if (!dead && tb < hh.nvalid) {
+      if (tb + 16 > hh.nvalid) {
+        // zero the V rows of this warp's tokens past the end (p = 0 there, V must be finite)
+        for (int i = lane; i < 16 * 16; i += 32) {
+          const int row = tb + (i >> 4), chunk = i & 15;
+          if (row >= hh.nvalid)
+            *reinterpret_cast<uint4*>(st + (chunk >> 3) * S::VHALF + row * 128 + (chunk & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        wrote_smem = true;
+        __syncwarp();
+      }
+      // ---- scores S[row][token] for this warp's 16 tokens (two accumulator
+      // chains per n-tile: even and odd k-steps)
+      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int mtx = lane >> 3, r8 = lane & 7;
+        const unsigned char* a0 = ks_base + ((mtx & 1) * 8 + r8) * KROW_BF16 + (tb + (mtx >> 1) * 8) * 2;
+#pragma unroll
+        for (int kk = 0; kk < 8; kk += 2) {
+          if (kk < nks) {
+            uint32_t bfr[4];
+            ldsm_x4_trans(bfr, a0 + kk * 16 * KROW_BF16);
+            mma_bf16_16816(c0, afr[kk], bfr[0], bfr[1]);
+            mma_bf16_16816(c1, afr[kk], bfr[2], bfr[3]);
+          }
+          if (kk + 1 < nks) {
+            uint32_t bfr[4];
+            ldsm_x4_trans(bfr, a0 + (kk + 1) * 16 * KROW_BF16);
+            mma_bf16_16816(d0, afr[kk + 1], bfr[0], bfr[1]);
+            mma_bf16_16816(d1, afr[kk + 1], bfr[2], bfr[3]);
+          }
+        }
+      }
+      // high + low parts; tokens tb + {2q, 2q+1, 8+2q, 9+2q}
+      float sc[4] = {(c0[0] + c0[2]) + (d0[0] + d0[2]), (c0[1] + c0[3]) + (d0[1] + d0[3]),
+                     (c1[0] + c1[2]) + (d1[0] + d1[2]), (c1[1] + c1[3]) + (d1[1] + d1[3])};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = tb + (e >> 1) * 8 + 2 * q4 + (e & 1);
+        if (tok >= hh.nvalid) sc[e] = -INFINITY;
+      }
+      if (p.scores_out != nullptr && head_row) {
+        const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
+        float* dst = p.scores_out + ((size_t)b * p.Hq + g * G + grp) * p.Tcap + hh.t0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = tb + (e >> 1) * 8 + 2 * q4 + (e & 1);
+          if (tok < hh.nvalid) dst[tok] = sc[e] * kLn2;
+        }
+      }
+      // ---- online softmax over this warp's tokens (lazy rescale)
+      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const bool upd = head_row && mx > mu + kLazyRescale;
+      if (__any_sync(0xffffffffu, upd)) {
+        float alpha = 1.f;
+        if (upd) {
+          alpha = exp2f(mu - mx);
+          mu = mx;
+        }
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          o[n][0] *= alpha;
+          o[n][1] *= alpha;
+          o[n][2] *= alpha;
+          o[n][3] *= alpha;
+        }
+        ell *= alpha;
+      }
+      float pv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pv[e] = head_row ? exp2f(sc[e] - mu) : 0.f;
+      float rs = (pv[0] + pv[1]) + (pv[2] + pv[3]);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+      rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+      ell += rs;
+      // A fragments of P: high parts in row grp, low parts in row grp + 8
+      float ph[4], pl[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) split_bf16(pv[e], ph[e], pl[e]);
+      const uint32_t pa[4] = {pack_bf16(ph[0], ph[1]), pack_bf16(pl[0], pl[1]), pack_bf16(ph[2], ph[3]),
+                              pack_bf16(pl[2], pl[3])};
+      // ---- o += P V over 128 dims (16 n-tiles of 8)
+      {
+        const int mtx = lane >> 3, r8 = lane & 7;
+        const int tok = tb + (mtx & 1) * 8 + r8;
+        const unsigned char* vrow = st + tok * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int dim0 = 16 * j + (mtx >> 1) * 8;
+          const int chunk = (dim0 & 63) >> 3;
+          uint32_t bfr[4];
+          ldsm_x4_trans(bfr, vrow + (dim0 >> 6) * S::VHALF + ((chunk ^ (tok & 7)) << 4));
+          mma_bf16_16816(o[2 * j], pa, bfr[0], bfr[1]);
+          mma_bf16_16816(o[2 * j + 1], pa, bfr[2], bfr[3]);
+        }
+      }
+    }
+    if (wrote_smem) fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+
+    if (!(hh.flags & kLast)) continue;
+
+    // ---- end of a segment: merge the warps' (m, l, o), then output or partial
+    if (head_row) {
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        *reinterpret_cast<float2*>(red + ((size_t)warp * G + grp) * D + 8 * n + 2 * q4) =
+            make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
+      if (q4 == 0) {
+        mlb[(warp * G + grp) * 2 + 0] = mu;
+        mlb[(warp * G + grp) * 2 + 1] = ell;
+      }
+    }
+    named_bar_sync(1, NCT);
+    float Mh[G], Lh[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < NCW; ++w2) M = fmaxf(M, mlb[(w2 * G + h) * 2]);
+      float L = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < NCW; ++w2) L = fmaf(exp2f(mlb[(w2 * G + h) * 2] - M), mlb[(w2 * G + h) * 2 + 1], L);
+      Mh[h] = M;
+      Lh[h] = L;
+    }
+    float merged[(G * D + NCT - 1) / NCT];
+#pragma unroll
+    for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+      const int idx = tid + NCT * i;
+      merged[i] = 0.f;
+      if (idx < G * D) {
+        const int h = idx / D, dim = idx % D;
+        float mh = 0.f;
+#pragma unroll
+        for (int x = 0; x < G; ++x)
+          if (x == h) mh = Mh[x];
+        float acc = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NCW; ++w2) {
+          const float f = exp2f(mlb[(w2 * G + h) * 2] - mh);
+          acc = fmaf(f, red[((size_t)w2 * G + h) * D + dim], acc);
+        }
+        merged[i] = acc;
+      }
+    }
+    named_bar_sync(1, NCT);
+#pragma unroll
+    for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+      const int idx = tid + NCT * i;
+      if (idx < G * D) red[idx] = merged[i];
+    }
+    named_bar_sync(1, NCT);
+    finish_segment<G>(p, hh, tid, Mh, Lh, red, s_last);
+    named_bar_sync(1, NCT);
+  }
+}
+
+// ============================================================================
+// f32 cache: CUDA-core consumers
+// ============================================================================
+template <int G>
+struct SmemF32 {
+  static constexpr int TT = 64;
+  static constexpr int KBYTES = D * TT * 4;
+  static constexpr int VBYTES = TT * D * 4;
+  static constexpr int STAGE = KBYTES + VBYTES;
+  static constexpr int RW = D;
+  static constexpr int SLOTS = (G * TT + NCT - 1) / NCT;
+  static constexpr int OFF_RED = NSTAGE * STAGE;
+  static constexpr int OFF_PSM = OFF_RED + NCW * G * RW * 4;
+  static constexpr int OFF_WST = OFF_PSM + TT * G * 4;
+  static constexpr int OFF_HDR = OFF_WST + 2 * SLOTS * NCW * 4;
+  static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
+  static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
+  static constexpr int OFF_MISC = OFF_SCH + 36 * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+};
+
+template <int G>
+__global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodeParams p) {
+  using S = SmemF32<G>;
+  constexpr int TT = S::TT;
+  constexpr int TPL = TT / 32;        // tokens per lane in the score pass
+  constexpr int TPW = TT / NCW;       // tokens per warp in the PV pass
+  static_assert(TPL == 2, "score pass loads two f32 tokens per lane");
+
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
+  float* psm = reinterpret_cast<float*>(smem + S::OFF_PSM);
+  float* wmax = reinterpret_cast<float*>(smem + S::OFF_WST);
+  float* wsum = wmax + S::SLOTS * NCW;
+  StageHdr* hdr = reinterpret_cast<StageHdr*>(smem + S::OFF_HDR);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  uint64_t* empty = full + NSTAGE;
+  long long* sch = reinterpret_cast<long long*>(smem + S::OFF_SCH);
+  int* s_last = reinterpret_cast<int*>(smem + S::OFF_MISC);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    fence_barrier_init();
+  }
+  Sched Sd;
+  if (!make_schedule<TT, NTHREADS>(p, sch + 4, sch, Sd)) return;
+  const int n_tiles = (int)(Sd.my_end - Sd.my_start);
+
+  if (warp == NCW) {
+    const uint64_t pol = policy_evict_first();
+    UnitWalker W;
+    W.start<TT>(p, Sd);
+    int urow[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+      const int r = lane + 32 * i;
+      urow[i] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
+    }
+    for (int it = 0; it < n_tiles; ++it) {
+      const long long t = Sd.my_start + it;
+      if (W.seek<TT>(p, Sd, t)) {
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+          const int r = lane + 32 * i;
+          urow[i] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
+        }
+      }
+      const int s = it % NSTAGE;
+      if (it >= NSTAGE) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(&empty[s], ((it / NSTAGE) & 1) ^ 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+          return;
+        }
+      }
+      const StageHdr hh = W.header(Sd, t, TT);
+      const uint32_t kbytes = (uint32_t)((hh.nvalid + 3) / 4 * 16);
+      const uint32_t vbytes = (uint32_t)hh.nvalid * D * 4;
       unsigned char* st = smem + (size_t)s * S::STAGE;
       if (lane == 0) {
-        StageHdr hh;
-        hh.u = u;
-        hh.t0 = t0;
-        hh.nvalid = nvalid;
-        hh.nU = nU;
-        hh.flags = ((t == my_start || t == ts) ? kFirst : 0) | ((t == my_end - 1 || t == te - 1) ? kLast : 0);
-        hh.seg = nseg > 1 ? (int)(sb + (c - cf)) : -1;
-        hh.nseg = nseg;
-        hh.seg0 = (int)sb;
         hdr[s] = hh;
-        mbar_arrive_expect_tx(&full[s], kbytes * nU + vbytes);
+        mbar_arrive_expect_tx(&full[s], kbytes * hh.nU + vbytes);
       }
       __syncwarp();
-      const T* kbase = static_cast<const T*>(p.kproj) + (size_t)u * p.d_store * p.Tcap + t0;
+      const float* kbase = static_cast<const float*>(p.kproj) + (size_t)hh.u * p.d_store * p.Tcap + hh.t0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < D / 32; ++i) {
         const int r = lane + 32 * i;
-        if (r < nU)
-          bulk_g2s(st + (size_t)r * TT * sizeof(T), kbase + (size_t)urow[i] * p.Tcap, kbytes, &full[s], pol);
+        if (r < hh.nU) bulk_g2s(st + (size_t)r * TT * 4, kbase + (size_t)urow[i] * p.Tcap, kbytes, &full[s], pol);
       }
       if (lane == 0) {
-        const T* vsrc = static_cast<const T*>(p.v) + ((size_t)u * p.Tcap + t0) * D;
+        const float* vsrc = static_cast<const float*>(p.v) + ((size_t)hh.u * p.Tcap + hh.t0) * D;
         bulk_g2s(st + S::KBYTES, vsrc, vbytes, &full[s], pol);
       }
     }
     return;
   }
 
-  // ======================= consumer warps =======================
   float qreg[RMAX][G];
   float oacc[G][4];
   float m_run[G], l_run[G];
@@ -477,14 +1007,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
 #pragma unroll
     for (int h = 0; h < G; ++h) qreg[i][h] = 0.f;
 
-  __shared__ int s_last;
   for (int it = 0; it < n_tiles; ++it) {
     const int s = it % NSTAGE;
     const bool ok = mbar_wait_bounded(&full[s], (it / NSTAGE) & 1);
     const StageHdr hh = hdr[s];
     const unsigned char* st = smem + (size_t)s * S::STAGE;
-    const T* Ks = reinterpret_cast<const T*>(st);
-    const T* Vs = reinterpret_cast<const T*>(st + S::KBYTES);
+    const float* Ks = reinterpret_cast<const float*>(st);
+    const float* Vs = reinterpret_cast<const float*>(st + S::KBYTES);
     const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
 
     if (ok && (hh.flags & kFirst)) {
@@ -507,7 +1036,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
       }
     }
 
-    // ---- partial scores over this warp's union rows
     if (ok) {
       float sacc[G][TPL];
 #pragma unroll
@@ -518,12 +1046,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
       for (int i = 0; i < RMAX; ++i) {
         const int r = warp + NCW * i;
         if (r < hh.nU) {
-          float kf[TPL];
-          load_row<T, TPL>(Ks + (size_t)r * TT + TPL * lane, kf);
+          const float2 kf = *reinterpret_cast<const float2*>(Ks + (size_t)r * TT + TPL * lane);
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < TPL; ++e) sacc[h][e] = fmaf(qreg[i][h], kf[e], sacc[h][e]);
+          for (int h = 0; h < G; ++h) {
+            sacc[h][0] = fmaf(qreg[i][h], kf.x, sacc[h][0]);
+            sacc[h][1] = fmaf(qreg[i][h], kf.y, sacc[h][1]);
+          }
         }
       }
 #pragma unroll
@@ -536,7 +1064,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
       return;
     }
 
-    // ---- reduce over warps, mask, tile maxima
     float sv[S::SLOTS];
 #pragma unroll
     for (int i = 0; i < S::SLOTS; ++i) {
@@ -564,8 +1091,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
         if (idx < G * TT) {
           const int h = idx / TT;
 #pragma unroll
-          for (int hh2 = 0; hh2 < G; ++hh2)
-            if (hh2 == h) mnew[hh2] = fmaxf(mnew[hh2], wmax[i * NCW + w2]);
+          for (int x = 0; x < G; ++x)
+            if (x == h) mnew[x] = fmaxf(mnew[x], wmax[i * NCW + w2]);
         }
       }
 #pragma unroll
@@ -577,8 +1104,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
         const int h = idx / TT, tok = idx % TT;
         float mh = 0.f;
 #pragma unroll
-        for (int hh2 = 0; hh2 < G; ++hh2)
-          if (hh2 == h) mh = mnew[hh2];
+        for (int x = 0; x < G; ++x)
+          if (x == h) mh = mnew[x];
         const float pr = exp2f(sv[i] - mh);
         psm[tok * G + h] = pr;
         const float sm = warp_sum(pr);
@@ -598,14 +1125,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
         if (idx < G * TT) {
           const int h = idx / TT;
 #pragma unroll
-          for (int hh2 = 0; hh2 < G; ++hh2)
-            if (hh2 == h) l_run[hh2] += wsum[i * NCW + w2];
+          for (int x = 0; x < G; ++x)
+            if (x == h) l_run[x] += wsum[i * NCW + w2];
         }
       }
 #pragma unroll
     for (int h = 0; h < G; ++h) m_run[h] = mnew[h];
 
-    // ---- o += p V over this warp's tokens
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -614,15 +1140,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
     for (int j = 0; j < TPW; ++j) {
       const int tok = warp * TPW + j;
       if (tok < hh.nvalid) {
-        float vf[4];
-        load_row<T, 4>(Vs + (size_t)tok * D + 4 * lane, vf);
+        const float4 vf = *reinterpret_cast<const float4*>(Vs + (size_t)tok * D + 4 * lane);
         float pv[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) pv[h] = psm[tok * G + h];
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) oacc[h][e] = fmaf(pv[h], vf[e], oacc[h][e]);
+        for (int h = 0; h < G; ++h) {
+          oacc[h][0] = fmaf(pv[h], vf.x, oacc[h][0]);
+          oacc[h][1] = fmaf(pv[h], vf.y, oacc[h][1]);
+          oacc[h][2] = fmaf(pv[h], vf.z, oacc[h][2]);
+          oacc[h][3] = fmaf(pv[h], vf.w, oacc[h][3]);
+        }
       }
     }
     __syncwarp();
@@ -630,102 +1158,84 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_kernel(DecodeParams p
 
     if (!(hh.flags & kLast)) continue;
 
-    // ---- end of a segment: reduce o over warps, then output or partial
 #pragma unroll
     for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) red[((size_t)warp * G + h) * S::RW + 4 * lane + e] = oacc[h][e];
+      *reinterpret_cast<float4*>(red + ((size_t)warp * G + h) * S::RW + 4 * lane) =
+          make_float4(oacc[h][0], oacc[h][1], oacc[h][2], oacc[h][3]);
     named_bar_sync(1, NCT);
-    const size_t bhq0 = (size_t)b * p.Hq + g * G;
+    float merged[(G * D + NCT - 1) / NCT];
 #pragma unroll
     for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
       const int idx = tid + NCT * i;
+      merged[i] = 0.f;
       if (idx < G * D) {
         const int h = idx / D, dim = idx % D;
-        float o = 0.f;
+        float acc = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < NCW; ++w2) o += red[((size_t)w2 * G + h) * S::RW + dim];
-        float lh = 0.f;
-#pragma unroll
-        for (int hh2 = 0; hh2 < G; ++hh2)
-          if (hh2 == h) lh = l_run[hh2];
-        if (hh.seg < 0) {
-          const float val = o / lh;
-          if (p.out_bf16)
-            static_cast<__nv_bfloat16*>(p.out)[(bhq0 + h) * D + dim] = __float2bfloat16_rn(val);
-          else
-            static_cast<float*>(p.out)[(bhq0 + h) * D + dim] = val;
-        } else {
-          p.part_o[((size_t)hh.seg * G + h) * D + dim] = o;
-        }
+        for (int w2 = 0; w2 < NCW; ++w2) acc += red[((size_t)w2 * G + h) * S::RW + dim];
+        merged[i] = acc;
       }
     }
-    if (tid < G) {
+    named_bar_sync(1, NCT);
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-        if (h == tid) {
-          if (hh.seg < 0) {
-            if (p.lse_out) p.lse_out[bhq0 + h] = (m_run[h] + log2f(l_run[h])) * kLn2;
-          } else {
-            p.part_ml[((size_t)hh.seg * G + h) * 2 + 0] = m_run[h];
-            p.part_ml[((size_t)hh.seg * G + h) * 2 + 1] = l_run[h];
-          }
-        }
+    for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+      const int idx = tid + NCT * i;
+      if (idx < G * D) red[idx] = merged[i];
     }
-    if (hh.seg >= 0) {
-      // publish this partial, take a ticket; the unit's last arrival merges
-      __threadfence();
-      named_bar_sync(1, NCT);
-      if (tid == 0) s_last = (atomicAdd(p.counters + hh.u, 1) == hh.nseg - 1);
-      named_bar_sync(1, NCT);
-      if (s_last) {
-        __threadfence();
-#pragma unroll 1
-        for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
-          const int idx = tid + NCT * i;
-          if (idx >= G * D) break;
-          const int h = idx / D, dim = idx % D;
-          float M = -INFINITY;
-#pragma unroll 1
-          for (int sg = 0; sg < hh.nseg; ++sg)
-            M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(hh.seg0 + sg) * G + h) * 2));
-          float Lsum = 0.f, O = 0.f;
-#pragma unroll 1
-          for (int sg = 0; sg < hh.nseg; ++sg) {
-            const size_t slot = (size_t)(hh.seg0 + sg) * G + h;
-            const float f = exp2f(__ldcg(p.part_ml + slot * 2) - M);
-            Lsum = fmaf(f, __ldcg(p.part_ml + slot * 2 + 1), Lsum);
-            O = fmaf(f, __ldcg(p.part_o + slot * D + dim), O);
-          }
-          const float val = O / Lsum;
-          if (p.out_bf16)
-            static_cast<__nv_bfloat16*>(p.out)[(bhq0 + h) * D + dim] = __float2bfloat16_rn(val);
-          else
-            static_cast<float*>(p.out)[(bhq0 + h) * D + dim] = val;
-          if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M + log2f(Lsum)) * kLn2;
-        }
-        if (tid == 0) p.counters[hh.u] = 0;
-      }
-    }
+    named_bar_sync(1, NCT);
+    finish_segment<G>(p, hh, tid, m_run, l_run, red, s_last);
     named_bar_sync(1, NCT);
   }
 }
 
+// ============================================================================
+// host launch
+// ============================================================================
 template <typename T, int G>
-int launch_decode_t(const DecodeParams& p, int n_units, int C, cudaStream_t st) {
-  using S = DecodeSmem<T, G>;
+int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(decode_attn_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::BYTES) != cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(decode_attn_kernel)");
+    if (cudaFuncSetAttribute(qproj_topk_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, D * D * 4) !=
+        cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(qproj_topk_kernel)");
     configured = true;
   }
-  qproj_topk_kernel<T, G><<<n_units, G * 32, 0, st>>>(p);
-  int rc = check_launch("qproj_topk_kernel");
+  qproj_topk_kernel<T, G><<<n_units, (G + 1) * 32, D * D * 4, st>>>(p);
+  return check_launch("qproj_topk_kernel");
+}
+
+template <int G>
+int launch_decode_bf16(const aqua_cache* c, const DecodeParams& p, int n_units, int C, cudaStream_t st) {
+  using S = SmemBF16<G>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(decode_attn_bf16_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES) !=
+        cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(decode_attn_bf16_kernel)");
+    configured = true;
+  }
+  CUtensorMap tmap;
+  int rc = encode_tmap_bf16_2d(&tmap, c->v, D, (uint64_t)c->B * c->Hkv * c->Tcap, D * 2, 64, S::TT, true);
   if (rc != AQUA_OK) return rc;
-  decode_attn_kernel<T, G><<<C, NTHREADS, S::BYTES, st>>>(p);
-  return check_launch("decode_attn_kernel");
+  if ((rc = launch_qproj<__nv_bfloat16, G>(p, n_units, st)) != AQUA_OK) return rc;
+  decode_attn_bf16_kernel<G><<<C, NTHREADS_BF16, S::BYTES, st>>>(tmap, p);
+  return check_launch("decode_attn_bf16_kernel");
+}
+
+template <int G>
+int launch_decode_f32(const DecodeParams& p, int n_units, int C, cudaStream_t st) {
+  using S = SmemF32<G>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(decode_attn_f32_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES) !=
+        cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(decode_attn_f32_kernel)");
+    configured = true;
+  }
+  int rc = launch_qproj<float, G>(p, n_units, st);
+  if (rc != AQUA_OK) return rc;
+  decode_attn_f32_kernel<G><<<C, NTHREADS, S::BYTES, st>>>(p);
+  return check_launch("decode_attn_f32_kernel");
 }
 
 }  // namespace
@@ -745,7 +1255,7 @@ size_t decode_workspace_bytes(int n_units, int G) {
 
 int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale,
                   void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
-                  float* lse_out, void* ws, cudaStream_t st) {
+                  float* lse_out, const void* k_new, const void* v_new, void* ws, cudaStream_t st) {
   const int G = Hq / c->Hkv;
   const int n_units = c->B * c->Hkv;
   DecodeParams p;
@@ -774,6 +1284,12 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.scores_out = scores_out;
   p.lse_out = lse_out;
   p.ctrl = c->ctrl;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.len_w = c->len;
+  p.n_abs = c->n_abs;
+  p.pos = c->pos;
+  p.score = c->score;
   p.B = c->B;
   p.Hq = Hq;
   p.Hkv = c->Hkv;
@@ -782,20 +1298,18 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.k = k;
   p.out_bf16 = out_dtype == AQUA_BF16;
   p.scale_log2 = scale * kLog2e;
-  const int TT = c->dtype == AQUA_BF16 ? Tile<__nv_bfloat16>::TT : Tile<float>::TT;
-  const long long tiles_ub = (long long)n_units * ((c->max_len + TT - 1) / TT);
+  const bool bf = c->dtype == AQUA_BF16;
+  const int TT = bf ? SmemBF16<1>::TT : SmemF32<1>::TT;
+  const int max_len = c->max_len + (k_new != nullptr ? 1 : 0);
+  const long long tiles_ub = (long long)n_units * ((max_len + TT - 1) / TT);
   long long C = device_sm_count();
   if (C > tiles_ub) C = tiles_ub;
   if (C < 1) C = 1;
   if (C > kMaxCtas) C = kMaxCtas;
-  const bool bf = c->dtype == AQUA_BF16;
   switch (G) {
-    case 1: return bf ? launch_decode_t<__nv_bfloat16, 1>(p, n_units, (int)C, st)
-                      : launch_decode_t<float, 1>(p, n_units, (int)C, st);
-    case 2: return bf ? launch_decode_t<__nv_bfloat16, 2>(p, n_units, (int)C, st)
-                      : launch_decode_t<float, 2>(p, n_units, (int)C, st);
-    case 4: return bf ? launch_decode_t<__nv_bfloat16, 4>(p, n_units, (int)C, st)
-                      : launch_decode_t<float, 4>(p, n_units, (int)C, st);
+    case 1: return bf ? launch_decode_bf16<1>(c, p, n_units, (int)C, st) : launch_decode_f32<1>(p, n_units, (int)C, st);
+    case 2: return bf ? launch_decode_bf16<2>(c, p, n_units, (int)C, st) : launch_decode_f32<2>(p, n_units, (int)C, st);
+    case 4: return bf ? launch_decode_bf16<4>(c, p, n_units, (int)C, st) : launch_decode_f32<4>(p, n_units, (int)C, st);
     default: return set_error(AQUA_ERR_UNSUPPORTED, "decode: Hq/Hkv = %d not in {1,2,4}", G);
   }
 }

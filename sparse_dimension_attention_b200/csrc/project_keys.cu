@@ -12,7 +12,7 @@ namespace aqua {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kTokPerCta = 8;  // one warp per token
+constexpr int kTokPerCta = 16;  // two tokens per warp
 
 template <typename T>
 __device__ __forceinline__ void load4(const T* p, float (&f)[4]);
@@ -38,7 +38,8 @@ __device__ __forceinline__ void copy4(__nv_bfloat16* dst, const __nv_bfloat16* s
   *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
 }
 
-// grid (ceil(L/8), Hkv, B), block 256: warp w projects token blockIdx.x*8+w of (b, g).
+// grid (ceil(L/16), Hkv, B), block 256: P[g] is staged in shared memory by one
+// bulk copy; warp w projects tokens blockIdx.x*16 + 2w and +1 of (b, g).
 template <typename T>
 __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__ k_new,
                                                            const T* __restrict__ v_new,
@@ -47,25 +48,43 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
                                                            int32_t* len, int32_t* n_abs, int32_t* pos,
                                                            float* score, int32_t* ctrl, int B, int L,
                                                            int Hkv, int d_store, int Tcap) {
+  extern __shared__ __align__(128) float Ps[];   // [D][D]
+  __shared__ __align__(8) uint64_t pbar;
+  __shared__ int is_last;
   const int g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int l = blockIdx.x * kTokPerCta + warp;
   // Lengths are read before this CTA takes its ticket below; the last CTA
   // advances them only after every CTA has taken one.
   const int base = __ldcg(len + b);
   const int abase = n_abs ? __ldcg(n_abs + b) : base;
-  if (l < L && (base < 0 || base + l >= Tcap)) {
-    if (lane == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
-  } else if (l < L) {
+  if (threadIdx.x == 0) {
+    mbar_init(&pbar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&pbar, D * D * 4);
+    bulk_g2s_plain(Ps, P + (size_t)g * D * D, D * D * 4, &pbar);
+  }
+  const bool ok = mbar_wait_bounded(&pbar, 0);
+  const bool bad = __syncthreads_or(!ok);
+  if (bad && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_TIMEOUT);
+#pragma unroll 1
+  for (int j = 0; j < kTokPerCta / 8 && !bad; ++j) {
+    const int l = blockIdx.x * kTokPerCta + warp * (kTokPerCta / 8) + j;
+    if (l >= L) break;
+    if (base < 0 || base + l >= Tcap) {
+      if (lane == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
+      break;
+    }
     const size_t row = ((size_t)b * L + l) * Hkv + g;
     float kv[4];
     load4<T>(k_new + row * D + 4 * lane, kv);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* Pg = P + (size_t)g * D * D;
-#pragma unroll 8
+#pragma unroll 16
     for (int i = 0; i < D; ++i) {
       const float ki = __shfl_sync(0xffffffffu, kv[i & 3], i >> 2);
-      const float4 pr = __ldg(reinterpret_cast<const float4*>(Pg + (size_t)i * D) + lane);
+      const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
       acc[0] = fmaf(ki, pr.x, acc[0]);
       acc[1] = fmaf(ki, pr.y, acc[1]);
       acc[2] = fmaf(ki, pr.z, acc[2]);
@@ -76,8 +95,8 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     T* kp = kproj + unit * d_store * (size_t)Tcap + slot;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      const int j = 4 * lane + s;
-      if (j < d_store) kp[(size_t)j * Tcap] = Elem<T>::from_f32(acc[s]);
+      const int jd = 4 * lane + s;
+      if (jd < d_store) kp[(size_t)jd * Tcap] = Elem<T>::from_f32(acc[s]);
     }
     copy4<T>(vcache + (unit * Tcap + slot) * D + 4 * lane, v_new + row * D + 4 * lane);
     if (pos != nullptr && lane == 0) {
@@ -85,7 +104,6 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
       score[unit * Tcap + slot] = 0.f;
     }
   }
-  __shared__ int is_last;
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -108,13 +126,28 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
 int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
                         cudaStream_t st) {
   dim3 grid((L + kTokPerCta - 1) / kTokPerCta, c->Hkv, c->B);
+  const int smem = D * D * 4;
   if (c->dtype == AQUA_BF16) {
-    project_keys_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+    static bool configured = false;
+    if (!configured) {
+      if (cudaFuncSetAttribute(project_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem) != cudaSuccess)
+        return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
+      configured = true;
+    }
+    project_keys_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
         static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), P,
         static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs,
         c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
   } else {
-    project_keys_kernel<float><<<grid, 256, 0, st>>>(
+    static bool configured = false;
+    if (!configured) {
+      if (cudaFuncSetAttribute(project_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
+      configured = true;
+    }
+    project_keys_kernel<float><<<grid, 256, smem, st>>>(
         static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
         static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score,
         c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);

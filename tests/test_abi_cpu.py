@@ -49,7 +49,7 @@ def test_struct_layout():
 
 
 def test_version(lib):
-    assert aq.aqua_version() == 1
+    assert aq.aqua_version() == 2
 
 
 def _desc(**kw):
@@ -88,9 +88,9 @@ def test_decode_argument_checks(lib):
     ws = lib.aqua_decode_workspace_size(ctypes.byref(c), 8)
     assert ws > 0
     call = lambda **kw: lib.aqua_decode_attn(
-        ctypes.byref(kw.get("c", c)), kw.get("q", 0x5000), 0x7000, kw.get("Hq", 8), kw.get("k", 96), 0.0,
-        0x8000, kw.get("od", abi.AQUA_BF16), None, None, None, None, kw.get("ws", 0x10000),
-        kw.get("wsb", ws), None)
+        ctypes.byref(kw.get("c", c)), kw.get("q", 0x5000), kw.get("kn", None), kw.get("vn", None), 0x7000,
+        kw.get("Hq", 8), kw.get("k", 96), 0.0, 0x8000, kw.get("od", abi.AQUA_BF16), None, None, None, None,
+        kw.get("ws", 0x10000), kw.get("wsb", ws), None)
     assert call(Hq=7) == abi.AQUA_ERR_ARG                 # not a multiple of Hkv
     assert call(Hq=16) == abi.AQUA_ERR_UNSUPPORTED        # group of 8
     assert call(k=0) == abi.AQUA_ERR_ARG
@@ -100,6 +100,10 @@ def test_decode_argument_checks(lib):
     assert call(od=5) == abi.AQUA_ERR_UNSUPPORTED
     assert call(wsb=ws - 1) == abi.AQUA_ERR_WORKSPACE
     assert call(ws=0x10010) == abi.AQUA_ERR_ARG           # workspace alignment
+    assert call(kn=0x9000) == abi.AQUA_ERR_ARG            # k_new without v_new
+    full = _desc(max_len=64)
+    assert call(c=full, kn=0x9000, vn=0x9100) == abi.AQUA_ERR_ARG   # no room to append
+    assert full.max_len == 64
 
 
 def test_decode_workspace_grows_with_units(lib):

@@ -13,7 +13,12 @@ from aqua_testlib import (calib_P, check_selection, fill_cache, oracle_cache, re
 pytestmark = pytest.mark.gpu
 
 TOL_BF16_OUT = 2e-3   # bf16 output vs the oracle output rounded to bf16
-TOL_F32_OUT = 1e-5
+TOL_F32_OUT = 1e-5    # f32 output, f32 cache
+# f32 output from a bf16 cache: the stored K~ is the bf16 rounding of an f32
+# projection; where the exact value lies within the f32 rounding error of a
+# bf16 midpoint (about 2e-4 of the elements on these inputs) the two sides
+# store neighbouring bf16 values, which perturbs a few scores by ~1e-4.
+TOL_F32_OUT_BF16_CACHE = 1e-4
 
 
 def _decode_case(B, Hq, Hkv, T, k, kv="bf16", out="bf16", lens=None, d_store=None, Tcap=None, chunk=None):
@@ -36,8 +41,8 @@ def _decode_case(B, Hq, Hkv, T, k, kv="bf16", out="bf16", lens=None, d_store=Non
     return cache, res, ref, lens
 
 
-def _check_outputs(res, ref, out, lens):
-    tol = TOL_BF16_OUT if out == "bf16" else TOL_F32_OUT
+def _check_outputs(res, ref, out, lens, kv="bf16"):
+    tol = TOL_BF16_OUT if out == "bf16" else (TOL_F32_OUT if kv == "f32" else TOL_F32_OUT_BF16_CACHE)
     err = rel_err_rows(res["out"], ref["out"])
     assert np.max(err) <= tol, f"max rel err {np.max(err):.3e} > {tol}"
     np.testing.assert_allclose(res["lse"], ref["lse"], rtol=1e-5, atol=1e-5)
@@ -46,7 +51,7 @@ def _check_outputs(res, ref, out, lens):
 def test_decode_fp32_tiny_config():
     """1 sequence, 4 query heads over 1 KV head, T = 1024, k = 96, f32 throughout."""
     cache, res, ref, lens = _decode_case(1, 4, 1, 1023, 96, kv="f32", out="f32")
-    _check_outputs(res, ref, "f32", lens)
+    _check_outputs(res, ref, "f32", lens, kv="f32")
     near = check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 96)
     assert near == 0
 
@@ -71,6 +76,7 @@ def test_decode_bf16_per_sequence_lengths_and_empty():
     live = [i for i, L in enumerate(lens) if L > 0]
     _check_outputs({"out": res["out"][live], "lse": res["lse"][live]},
                    {"out": ref["out"][live], "lse": ref["lse"][live]}, "bf16", None)
+    assert np.all(ref["out"][2] == 0.0) and np.all(np.isneginf(ref["lse"][2]))
     assert np.all(res["out"][2] == 0.0)
     assert np.all(np.isneginf(res["lse"][2]))
 
@@ -98,6 +104,7 @@ def test_decode_truncated_cache():
 def test_decode_scores_match_oracle():
     cache, res, ref, lens = _decode_case(1, 4, 1, 200, 96, kv="f32", out="f32")
     T = lens[0]
+    _check_outputs(res, ref, "f32", lens, kv="f32")
     for h in range(4):
         p = np.exp(res["scores"][0, h, :T] - res["lse"][0, h])
         np.testing.assert_allclose(p, ref["probs"][0][h], rtol=2e-5, atol=1e-9)
@@ -131,23 +138,26 @@ def test_decode_adversarial_ties():
 
 
 def test_key_cache_storage_rounding():
-    """Stored K~ equals the oracle's bf16 RNE of k P, except where the exact value lies within
-    f32 rounding of a bf16 midpoint (then the two neighbours are both acceptable)."""
+    """Stored K~ equals the oracle's bf16 RNE of k P, except where the exact value lies
+    within the f32 projection's rounding-error bound (gamma_128 * sum_i |k_i P_ij|) of a
+    bf16 midpoint; there both neighbours are correct roundings of an f32 result."""
     B, Hkv, T = 2, 2, 200
     P64, P32 = calib_P(Hkv)
     inp = synth.decode_inputs(B, 4, Hkv, T, bf16=True, steps=1)
     cache = aq.AquaCache(B, Hkv, 208)
     fill_cache(cache, inp["k_hist"], inp["v_hist"], P32, chunk=64)
     got = cache.k_proj.float().cpu().numpy()[..., :T].transpose(0, 1, 3, 2).astype(np.float64)   # [B,Hkv,T,d]
-    exact = np.einsum("btgi,gij->bgtj", inp["k_hist"].astype(np.float64), P64)
+    kk = inp["k_hist"].astype(np.float64)
+    exact = np.einsum("btgi,gij->bgtj", kk, P64)
+    bound = 128 * 2.0 ** -24 * np.einsum("btgi,gij->bgtj", np.abs(kk), np.abs(P64))
     ref = O.round_bf16(exact)
     diff = got != ref
     if diff.any():
-        e, g = exact[diff], got[diff]
-        r = ref[diff]
+        e, g, r, bd = exact[diff], got[diff], ref[diff], bound[diff]
         mid = (g + r) / 2
-        assert np.all(np.abs(e - mid) <= 1e-6 * np.abs(e) + 1e-30)
-    assert diff.mean() < 1e-3
+        assert np.all(O.round_bf16(g) == g)                    # a bf16 value
+        assert np.all(np.abs(e - mid) <= bd)                   # only at a midpoint within f32 error
+    assert diff.mean() < 2e-3
     np.testing.assert_array_equal(cache.v.float().cpu().numpy()[:, :, :T].transpose(0, 2, 1, 3), inp["v_hist"])
     assert cache.len.cpu().tolist() == [T, T] and cache.max_len == T
 
@@ -203,4 +213,42 @@ def test_long_context_split_k_sampled():
         ref = O.decode(q[:, g * 4:(g + 1) * 4], P64[g:g + 1], Kt, v_all[:, :, g:g + 1].transpose(0, 2, 1, 3),
                        [T + 1], k)
         err = rel_err_rows(res["out"][:, g * 4:(g + 1) * 4], ref["out"])
-        assert np.max(err) <= TOL_F32_OUT * 3, np.max(err)
+        assert np.max(err) <= TOL_F32_OUT_BF16_CACHE, np.max(err)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "f32"])
+def test_fused_append_equals_separate_append(kv):
+    """aqua_decode_attn with k_new/v_new == aqua_project_keys(L=1) then aqua_decode_attn."""
+    B, Hq, Hkv, T, k = 3, 8, 2, 300, 64
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, Hq, Hkv, T, bf16=(kv == "bf16"), steps=2)
+    dt = torch_dtype(kv)
+    caches = [aq.AquaCache(B, Hkv, 320, dtype=dt) for _ in range(2)]
+    for c in caches:
+        Pt = fill_cache(c, inp["k_hist"], inp["v_hist"], P32)
+    outs = []
+    for mode, c in enumerate(caches):
+        ws = torch.empty(aq.aqua_decode_workspace_size(c.desc, Hq), dtype=torch.uint8, device="cuda")
+        res = []
+        for s in range(2):
+            q = tdev(inp["q"][s], dt)
+            kn, vn = tdev(inp["k_new"][s], dt), tdev(inp["v_new"][s], dt)
+            out = torch.empty((B, Hq, 128), dtype=torch.float32, device="cuda")
+            if mode == 0:
+                aq.aqua_project_keys(c.desc, kn, vn, Pt, 1)
+                aq.aqua_decode_attn(c.desc, q, Pt, Hq, k, out, ws)
+            else:
+                aq.aqua_decode_attn(c.desc, q, Pt, Hq, k, out, ws, k_new=kn, v_new=vn)
+            res.append(out.cpu())
+        torch.cuda.synchronize()
+        outs.append(res)
+    for s in range(2):
+        assert torch.equal(outs[0][s], outs[1][s])
+    assert torch.equal(caches[0].k_proj, caches[1].k_proj) and torch.equal(caches[0].v, caches[1].v)
+    assert torch.equal(caches[0].len, caches[1].len) and caches[0].max_len == caches[1].max_len == T + 2
+    # and both equal the oracle
+    k_all = np.concatenate([inp["k_hist"], inp["k_new"].transpose(1, 0, 2, 3)], axis=1)
+    v_all = np.concatenate([inp["v_hist"], inp["v_new"].transpose(1, 0, 2, 3)], axis=1)
+    ref = O.decode(inp["q"][1], P64, oracle_cache(k_all, P64, kv), v_all.transpose(0, 2, 1, 3), [T + 2] * B, k)
+    err = rel_err_rows(outs[1][1].numpy().astype(np.float64), ref["out"])
+    assert np.max(err) <= (TOL_F32_OUT if kv == "f32" else TOL_F32_OUT_BF16_CACHE)

@@ -111,6 +111,11 @@ def test_select_identity_projection_is_raw_topk():
         np.testing.assert_array_equal(O.select_dims(qt, k), ref)
 
 
+def test_attend_over_no_tokens_is_empty_sum():
+    o, p, lse, S = O.attend_one(np.ones(8), 2, np.zeros((0, 8)), np.zeros((0, 8)), 1.0)
+    assert np.all(o == 0) and p.size == 0 and lse == -np.inf and list(S) == [0, 1]
+
+
 def test_select_rejects_bad_k():
     with pytest.raises(ValueError):
         O.select_dims(np.ones(8), 0)
