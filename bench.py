@@ -233,17 +233,29 @@ class DecodeBench:
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / K
 
-    def timed(self, K: int, W: int, k: int, world: int, clocks: bool):
+    def timed(self, K: int, W: int, k: int, world: int, clocks: bool, graph: bool = True):
+        """K decode steps after W warm-up steps.  With graph=True the K steps are
+        captured once into a CUDA graph and timed as one replay (the way a serving
+        loop issues them); otherwise each step is issued from Python."""
         torch = self.torch
         st = torch.cuda.current_stream()
         self.rewind()
         for s in range(W):
             self.step(s % self.n_in, k)
-        # soak so the clock sampler sees the GPU under this load
         torch.cuda.synchronize()
         self.rewind()
-        ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        g = None
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for s in range(K):
+                    self.step(s % self.n_in, k)
+            torch.cuda.synchronize()
+            self.rewind()
+            g.replay()          # one untimed replay (uploads the graph)
+            torch.cuda.synchronize()
+            self.rewind()
+            torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(torch.cuda.current_device()) if clocks else None
         if sampler:
@@ -251,36 +263,31 @@ class DecodeBench:
         barrier(world)
         torch.cuda.synchronize()
         e0.record(st)
-        for s in range(K):
-            ev_s[s].record(st)
-            self.step(s % self.n_in, k)
-            ev_e[s].record(st)
+        if g is not None:
+            g.replay()
+        else:
+            for s in range(K):
+                self.step(s % self.n_in, k)
         e1.record(st)
         torch.cuda.synchronize()
         barrier(world)
         clk = sampler.stop() if sampler else None
         total_ms = e0.elapsed_time(e1)
-        step_ms = [ev_s[s].elapsed_time(ev_e[s]) for s in range(K)]
-        return total_ms, step_ms, clk
+        del g
+        return total_ms, [total_ms / K] * K, clk
 
     def e2e(self, K: int, k: int):
-        """Same steps through the public API from pinned host buffers: per step H2D of q,
-        k_new, v_new and D2H of the output inside the timed region."""
+        """Same steps through the public API from pinned host buffers: per step the
+        H2D copies of q, k_new, v_new and the D2H copy of the output are part of
+        the timed region (captured with the calls into one CUDA graph)."""
         torch = self.torch
         st = torch.cuda.current_stream()
         wl = self.wl
         qd = torch.empty_like(self.q_d[0])
         kd = torch.empty_like(self.k_d[0])
         vd = torch.empty_like(self.v_d[0])
-        for s in range(3):   # warm-up
-            qd.copy_(self.q_h[s % self.n_in], non_blocking=True)
-            self.step(s % self.n_in, k)
-        torch.cuda.synchronize()
-        self.rewind()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(st)
-        for s in range(K):
+
+        def one(s):
             i = s % self.n_in
             qd.copy_(self.q_h[i], non_blocking=True)
             kd.copy_(self.k_h[i], non_blocking=True)
@@ -288,9 +295,29 @@ class DecodeBench:
             self.aq.aqua_decode_attn(self.cache.desc, qd, self.P, wl["Hq"], k, self.out, self.ws, k_new=kd,
                                      v_new=vd)
             self.out_h.copy_(self.out, non_blocking=True)
+
+        self.rewind()
+        for s in range(3):
+            one(s)
+        torch.cuda.synchronize()
+        self.rewind()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s in range(K):
+                one(s)
+        torch.cuda.synchronize()
+        self.rewind()
+        g.replay()
+        torch.cuda.synchronize()
+        self.rewind()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        g.replay()
         e1.record(st)
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1)
+        del g
         h2d = (self.q_h[0].numel() + self.k_h[0].numel() + self.v_h[0].numel()) * self.esize
         d2h = self.out.numel() * self.esize
         return ms, h2d, d2h
@@ -402,6 +429,7 @@ def main():
     achieved = (sum(dec_bytes) + K * bench.bytes_append()) / (sum(step_ms) / 1e3) / 1e9
     step_gbs = (sum(dec_bytes) + K * bench.bytes_append()) / (total_ms / 1e3) / 1e9
     unfused_ms = bench.timed_unfused(min(K, 100), W, wl["k"])
+    eager_ms, _, _ = bench.timed(min(K, 100), W, wl["k"], world, clocks=False, graph=False)
     e2e_ms, h2d, d2h = bench.e2e(K, wl["k"])
     e2e_ms = max_over_ranks(e2e_ms, world)
     line = {
@@ -411,6 +439,7 @@ def main():
         "config": {"workload": args.workload, "B": wl["B"], "Hq": wl["Hq"], "Hkv": wl["Hkv"], "d": 128,
                    "T": wl["T"], "T_range": [T_steps[0], T_steps[-1]], "k": wl["k"], "kv_cache": wl["kv"],
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "launch": "cuda graph",
                    "l2": "no flush: each step streams %.0f MB of K~/V, above the 126 MB L2"
                          % (dec_bytes[0] / 1e6),
                    "inputs": "synthetic anisotropic Q/K (Llama-3.1-8B shape), P from GPU SVD calibration"},
@@ -421,6 +450,8 @@ def main():
                      "kernel": "aqua_decode_attn step (qproj_topk_kernel with fused append + decode_attn_bf16_kernel)",
                      "peak_source": peak_kind,
                      "step_us": 1e3 * statistics.mean(step_ms)},
+        "launch": "K steps captured in one CUDA graph (kernels chained with programmatic dependent launch)",
+        "eager_step_us": 1e3 * eager_ms / min(K, 100),
         "unfused_step_us": 1e3 * unfused_ms,
         "e2e": {"value": world * wl["B"] * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},

@@ -7,6 +7,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "aqua.h"
 
 namespace aqua {
@@ -30,6 +32,25 @@ int device_sm_count();
 int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel in the stream is still running; it must call pdl_wait()
+// before reading or writing anything that kernel may touch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- element access
 template <typename T> struct Elem;
 template <> struct Elem<float> {
@@ -44,6 +65,28 @@ template <> struct Elem<__nv_bfloat16> {
 // bf16 pair packed in a 32-bit word -> two exact floats (low half first)
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// y = x P for one row vector x (shared memory, kHeadDim floats, 16-byte aligned)
+// and P in shared memory ([kHeadDim][kHeadDim], row i = input dim i); lane
+// computes outputs 4*lane .. 4*lane+3.  Every projection in the library (keys
+// appended by either entry point, queries) uses this one summation order.
+__device__ __forceinline__ void project_row_smem(const float* Ps, const float* xs, int lane, float (&y)[4]) {
+  float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int i = 0; i < kHeadDim; i += 4) {
+    const float4 x4 = *reinterpret_cast<const float4*>(xs + i);
+    const float4 p0 = reinterpret_cast<const float4*>(Ps + (i + 0) * kHeadDim)[lane];
+    const float4 p1 = reinterpret_cast<const float4*>(Ps + (i + 1) * kHeadDim)[lane];
+    const float4 p2 = reinterpret_cast<const float4*>(Ps + (i + 2) * kHeadDim)[lane];
+    const float4 p3 = reinterpret_cast<const float4*>(Ps + (i + 3) * kHeadDim)[lane];
+    a[0] = fmaf(x4.x, p0.x, a[0]); a[1] = fmaf(x4.x, p0.y, a[1]); a[2] = fmaf(x4.x, p0.z, a[2]); a[3] = fmaf(x4.x, p0.w, a[3]);
+    b[0] = fmaf(x4.y, p1.x, b[0]); b[1] = fmaf(x4.y, p1.y, b[1]); b[2] = fmaf(x4.y, p1.z, b[2]); b[3] = fmaf(x4.y, p1.w, b[3]);
+    a[0] = fmaf(x4.z, p2.x, a[0]); a[1] = fmaf(x4.z, p2.y, a[1]); a[2] = fmaf(x4.z, p2.z, a[2]); a[3] = fmaf(x4.z, p2.w, a[3]);
+    b[0] = fmaf(x4.w, p3.x, b[0]); b[1] = fmaf(x4.w, p3.y, b[1]); b[2] = fmaf(x4.w, p3.z, b[2]); b[3] = fmaf(x4.w, p3.w, b[3]);
+  }
+#pragma unroll
+  for (int s = 0; s < 4; ++s) y[s] = a[s] + b[s];
+}
 
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }
 __device__ __forceinline__ void store_out(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
@@ -206,6 +249,13 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
       : "memory");
   return r != 0;
 }
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now / wait until every prerequisite grid has completed and its
+// memory is visible.  Both are no-ops for kernels launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void record_status(int32_t* ctrl, int code) {
   if (ctrl) atomicCAS(ctrl + kCtrlStatus, 0, code);

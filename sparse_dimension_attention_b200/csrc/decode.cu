@@ -108,7 +108,8 @@ __device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, flo
 template <typename T, int G>
 __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p) {
   extern __shared__ __align__(128) float Ps[];   // P[g], [D][D]
-  __shared__ float qs[G][D];
+  __shared__ __align__(16) float qs[G][D];
+  __shared__ __align__(16) float knew_s[D];
   __shared__ uint32_t masks[G][4];
   __shared__ __align__(8) uint64_t pbar;
   __shared__ int is_last;
@@ -118,12 +119,13 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
   const int h = g * G + (w < G ? w : 0);
   const int m = p.d_store;
   const bool append = p.k_new != nullptr;
-  const int len_before = __ldcg(p.len + b);   // read before the append ticket below
 
   if (threadIdx.x == 0) {
     mbar_init(&pbar, 1);
     fence_barrier_init();
   }
+  pdl_launch_dependents();   // the attention kernel may take free SMs for its prologue
+  pdl_wait();                // inputs and the cache may come from the previous kernel
   __syncthreads();
   if (threadIdx.x == 0) {
     mbar_arrive_expect_tx(&pbar, D * D * 4);
@@ -139,6 +141,7 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
     return;
   }
 
+  const int len_before = __ldcg(p.len + b);   // read before the append ticket below
   if (w == G) {
     // ---- fused append of the new token of unit (b, g)
     if (append) {
@@ -147,19 +150,11 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
         if (lane == 0) record_status(p.ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
       } else {
         const T* kr = static_cast<const T*>(p.k_new) + (size_t)u * D;
-        float kv[4];
 #pragma unroll
-        for (int s2 = 0; s2 < 4; ++s2) kv[s2] = Elem<T>::load(kr + 4 * lane + s2);
-        float kt[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-        for (int i = 0; i < D; ++i) {
-          const float ki = __shfl_sync(0xffffffffu, kv[i & 3], i >> 2);
-          const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
-          kt[0] = fmaf(ki, pr.x, kt[0]);
-          kt[1] = fmaf(ki, pr.y, kt[1]);
-          kt[2] = fmaf(ki, pr.z, kt[2]);
-          kt[3] = fmaf(ki, pr.w, kt[3]);
-        }
+        for (int s2 = 0; s2 < 4; ++s2) knew_s[4 * lane + s2] = Elem<T>::load(kr + 4 * lane + s2);
+        __syncwarp();
+        float kt[4];
+        project_row_smem(Ps, knew_s, lane, kt);
         T* kp = const_cast<T*>(static_cast<const T*>(p.kproj)) + (size_t)u * p.d_store * p.Tcap + slot;
 #pragma unroll
         for (int s2 = 0; s2 < 4; ++s2) {
@@ -177,44 +172,44 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
       }
     }
   } else {
-    // q~_j for j = 4*lane + s
-    float qt[4] = {0.f, 0.f, 0.f, 0.f};
-  #pragma unroll 16
-    for (int i = 0; i < D; ++i) {
-      const float qi = __shfl_sync(0xffffffffu, qv[i & 3], i >> 2);
-      const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
-      qt[0] = fmaf(qi, pr.x, qt[0]);
-      qt[1] = fmaf(qi, pr.y, qt[1]);
-      qt[2] = fmaf(qi, pr.z, qt[2]);
-      qt[3] = fmaf(qi, pr.w, qt[3]);
-    }
+    // q~_j for j = 4*lane + s; q is read back from shared memory as a broadcast,
+    // two accumulator chains (even / odd input dims)
+    qs[w][4 * lane + 0] = qv[0];
+    qs[w][4 * lane + 1] = qv[1];
+    qs[w][4 * lane + 2] = qv[2];
+    qs[w][4 * lane + 3] = qv[3];
+    __syncwarp();
+    float qt[4];
+    project_row_smem(Ps, qs[w], lane, qt);
+    __syncwarp();
 
     // Keys: magnitude bits + 1 for candidate dims (j < m), 0 otherwise, so that
     // unsigned order equals |q~| order and non-candidates rank below everything.
     uint32_t key[4];
-  #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int j = 4 * lane + s;
-      key[s] = (j < m) ? (__float_as_uint(fabsf(qt[s])) + 1u) : 0u;
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) {
+      const int j = 4 * lane + s2;
+      key[s2] = (j < m) ? (__float_as_uint(fabsf(qt[s2])) + 1u) : 0u;
     }
-    // Radix select of the k-th largest key: the largest tau with #{key >= tau} >= k.
+    // Radix select of the k-th largest key: the largest tau with
+    // #{key >= tau} >= k, one bit per round; counts by ballot + popc.
     uint32_t tau = 0;
-  #pragma unroll 1
+#pragma unroll 4
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = tau | (1u << bit);
-      int c = 0;
-  #pragma unroll
-      for (int s = 0; s < 4; ++s) c += (key[s] >= cand);
-      c = __reduce_add_sync(0xffffffffu, c);
+      const int c = __popc(__ballot_sync(0xffffffffu, key[0] >= cand)) +
+                    __popc(__ballot_sync(0xffffffffu, key[1] >= cand)) +
+                    __popc(__ballot_sync(0xffffffffu, key[2] >= cand)) +
+                    __popc(__ballot_sync(0xffffffffu, key[3] >= cand));
       if (c >= p.k) tau = cand;
     }
     int ngt = 0, neq = 0;
   #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      ngt += (key[s] > tau);
+      ngt += __popc(__ballot_sync(0xffffffffu, key[s] > tau));
       neq += (key[s] == tau);
     }
-    const int need = p.k - __reduce_add_sync(0xffffffffu, ngt);  // ties to take, lowest index first
+    const int need = p.k - ngt;  // ties to take, lowest index first
     int incl = neq;
   #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -279,9 +274,11 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
   }
   for (int j = threadIdx.x; j < D; j += blockDim.x) {
     const int wd = j >> 5, bit = j & 31;
-    if ((um[wd] >> bit) & 1u) {
-      int r = __popc(um[wd] & ((1u << bit) - 1u));
-      for (int x = 0; x < wd; ++x) r += __popc(um[x]);
+    // register selects instead of a run-time index into um[]
+    const uint32_t word = wd == 0 ? um[0] : (wd == 1 ? um[1] : (wd == 2 ? um[2] : um[3]));
+    if ((word >> bit) & 1u) {
+      int r = __popc(word & ((1u << bit) - 1u));
+      r += (wd > 0 ? __popc(um[0]) : 0) + (wd > 1 ? __popc(um[1]) : 0) + (wd > 2 ? __popc(um[2]) : 0);
       p.ulist[(size_t)u * D + r] = j;
       float* dst = p.qm + ((size_t)u * D + r) * G;
 #pragma unroll
@@ -512,13 +509,18 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
       }
   }
   if (hh.seg < 0) return;
-  // publish this partial, take a ticket; the unit's last arrival merges
-  __threadfence();
+  // publish this partial and take a ticket; the unit's last arrival merges.
+  // The barrier orders every thread's partial stores before thread 0's
+  // GPU-scope fence (fences are cumulative), which precedes the ticket.
   named_bar_sync(1, NCT);
-  if (tid == 0) *s_last = (atomicAdd(p.counters + hh.u, 1) == hh.nseg - 1);
+  if (tid == 0) {
+    __threadfence();
+    *s_last = (atomicAdd(p.counters + hh.u, 1) == hh.nseg - 1);
+  }
   named_bar_sync(1, NCT);
   if (!*s_last) return;
   __threadfence();
+  constexpr int MB = 8;   // partials fetched per round, loads in flight together
 #pragma unroll 1
   for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
     const int idx = tid + NCT * i;
@@ -526,15 +528,35 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
     const int h = idx / D, dim = idx % D;
     float M = -INFINITY;
 #pragma unroll 1
-    for (int sg = 0; sg < hh.nseg; ++sg) M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(hh.seg0 + sg) * G + h) * 2));
+    for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
+      float mv[MB];
+#pragma unroll
+      for (int j = 0; j < MB; ++j)
+        mv[j] = (s0 + j < hh.nseg) ? __ldcg(p.part_ml + ((size_t)(hh.seg0 + s0 + j) * G + h) * 2) : -INFINITY;
+#pragma unroll
+      for (int j = 0; j < MB; ++j) M = fmaxf(M, mv[j]);
+    }
     float Lsum = 0.f, O = 0.f;
 #pragma unroll 1
-    for (int sg = 0; sg < hh.nseg; ++sg) {
-      const size_t slot = (size_t)(hh.seg0 + sg) * G + h;
-      const float f = exp2f(__ldcg(p.part_ml + slot * 2) - M);
-      Lsum = fmaf(f, __ldcg(p.part_ml + slot * 2 + 1), Lsum);
-      O = fmaf(f, __ldcg(p.part_o + slot * D + dim), O);
+    for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
+      float mv[MB], lv[MB], ov[MB];
+#pragma unroll
+      for (int j = 0; j < MB; ++j) {
+        const bool in = s0 + j < hh.nseg;
+        const size_t slot = (size_t)(hh.seg0 + s0 + j) * G + h;
+        mv[j] = in ? __ldcg(p.part_ml + slot * 2) : -INFINITY;
+        lv[j] = in ? __ldcg(p.part_ml + slot * 2 + 1) : 0.f;
+        ov[j] = in ? __ldcg(p.part_o + slot * D + dim) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < MB; ++j) {
+        const float f = exp2f(mv[j] - M);
+        Lsum = fmaf(f, lv[j], Lsum);
+        O = fmaf(f, ov[j], O);
+      }
     }
+    const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
+    const size_t bhq0 = (size_t)b * p.Hq + g * G;
     store_val(p, (bhq0 + h) * D + dim, O / Lsum);
     if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M + log2f(Lsum)) * kLn2;
   }
@@ -551,8 +573,8 @@ struct SmemBF16 {
   static constexpr int KBYTES = D * KROW_BF16;          // [128 rows][272 B]
   static constexpr int STAGE = 2 * VHALF + KBYTES;      // multiple of 1024
   static constexpr int OFF_RED = NSTAGE * STAGE;        // [NCW][G][D] f32
-  static constexpr int OFF_ML = OFF_RED + NCW * G * D * 4;   // [NCW][G][2] f32
-  static constexpr int OFF_HDR = OFF_ML + NCW * G * 2 * 4;
+  static constexpr int OFF_ML = OFF_RED + NCW * G * D * 4;   // [NCW][G][2] f32, [NCW][G] factors, [2][G]
+  static constexpr int OFF_HDR = OFF_ML + (NCW * G * 3 + 2 * G) * 4;
   static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
   static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
   static constexpr int OFF_MISC = OFF_SCH + 36 * 8;
@@ -589,6 +611,9 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     }
     fence_barrier_init();
   }
+  if (tid == NCT) prefetch_tmap(&tmap_v);
+  pdl_launch_dependents();
+  pdl_wait();   // the projection kernel (and any append) must be complete
   Sched Sd;
   if (!make_schedule<TT, NTHREADS_BF16>(p, sch + 4, sch, Sd)) return;
   fence_proxy_async_smem();
@@ -602,9 +627,23 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     const int pt = tid - NCT;
     const int chunk = pt & 15, r0 = pt >> 4;
     const uint64_t pol = policy_evict_first();
-    if (pt == 0) prefetch_tmap(&tmap_v);
     UnitWalker W;
     W.start<TT>(p, Sd);
+    if (pt == 0) {
+      // V tiles of the first stages do not depend on the union list: issue
+      // them before the union rows are fetched
+      UnitWalker W0 = W;
+      for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
+        const long long t = Sd.my_start + it;
+        W0.seek<TT>(p, Sd, t);
+        const StageHdr h0 = W0.header(Sd, t, TT);
+        unsigned char* st = smem + (size_t)it * S::STAGE;
+        mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
+        const int row = h0.u * p.Tcap + h0.t0;
+        tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
+        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
+      }
+    }
     int urow[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
@@ -632,7 +671,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       }
       const StageHdr hh = W.header(Sd, t, TT);
       unsigned char* st = smem + (size_t)s * S::STAGE;
-      if (pt == 0) {
+      if (pt == 0 && it >= NSTAGE) {
         mbar_arrive_expect_tx(&full[s], 2 * S::VHALF);
         const int row = hh.u * p.Tcap + hh.t0;
         tma_load_2d(st, &tmap_v, 0, row, &full[s], pol);
@@ -841,17 +880,29 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       }
     }
     named_bar_sync(1, NCT);
-    float Mh[G], Lh[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
+    // per-head running max over the warps and each warp's scale factor, once
+    float* fac = mlb + NCW * G * 2;          // [NCW][G] scale factors, then [G] M and [G] L
+    if (tid < G) {
+      const int h = tid;
       float M = -INFINITY;
 #pragma unroll
       for (int w2 = 0; w2 < NCW; ++w2) M = fmaxf(M, mlb[(w2 * G + h) * 2]);
       float L = 0.f;
 #pragma unroll
-      for (int w2 = 0; w2 < NCW; ++w2) L = fmaf(exp2f(mlb[(w2 * G + h) * 2] - M), mlb[(w2 * G + h) * 2 + 1], L);
-      Mh[h] = M;
-      Lh[h] = L;
+      for (int w2 = 0; w2 < NCW; ++w2) {
+        const float f = exp2f(mlb[(w2 * G + h) * 2] - M);
+        fac[w2 * G + h] = f;
+        L = fmaf(f, mlb[(w2 * G + h) * 2 + 1], L);
+      }
+      fac[NCW * G + h] = M;
+      fac[NCW * G + G + h] = L;
+    }
+    named_bar_sync(1, NCT);
+    float Mh[G], Lh[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      Mh[h] = fac[NCW * G + h];
+      Lh[h] = fac[NCW * G + G + h];
     }
     float merged[(G * D + NCT - 1) / NCT];
 #pragma unroll
@@ -860,20 +911,12 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       merged[i] = 0.f;
       if (idx < G * D) {
         const int h = idx / D, dim = idx % D;
-        float mh = 0.f;
-#pragma unroll
-        for (int x = 0; x < G; ++x)
-          if (x == h) mh = Mh[x];
         float acc = 0.f;
 #pragma unroll
-        for (int w2 = 0; w2 < NCW; ++w2) {
-          const float f = exp2f(mlb[(w2 * G + h) * 2] - mh);
-          acc = fmaf(f, red[((size_t)w2 * G + h) * D + dim], acc);
-        }
+        for (int w2 = 0; w2 < NCW; ++w2) acc = fmaf(fac[w2 * G + h], red[((size_t)w2 * G + h) * D + dim], acc);
         merged[i] = acc;
       }
-    }
-    named_bar_sync(1, NCT);
+    }    named_bar_sync(1, NCT);
 #pragma unroll
     for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
       const int idx = tid + NCT * i;
@@ -935,6 +978,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
     }
     fence_barrier_init();
   }
+  pdl_launch_dependents();
+  pdl_wait();
   Sched Sd;
   if (!make_schedule<TT, NTHREADS>(p, sch + 4, sch, Sd)) return;
   const int n_tiles = (int)(Sd.my_end - Sd.my_start);
@@ -1200,7 +1245,8 @@ int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
       return check_launch("cudaFuncSetAttribute(qproj_topk_kernel)");
     configured = true;
   }
-  qproj_topk_kernel<T, G><<<n_units, (G + 1) * 32, D * D * 4, st>>>(p);
+  const cudaError_t e = launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3((G + 1) * 32), D * D * 4, st, p);
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
   return check_launch("qproj_topk_kernel");
 }
 
@@ -1214,11 +1260,21 @@ int launch_decode_bf16(const aqua_cache* c, const DecodeParams& p, int n_units, 
       return check_launch("cudaFuncSetAttribute(decode_attn_bf16_kernel)");
     configured = true;
   }
-  CUtensorMap tmap;
-  int rc = encode_tmap_bf16_2d(&tmap, c->v, D, (uint64_t)c->B * c->Hkv * c->Tcap, D * 2, 64, S::TT, true);
-  if (rc != AQUA_OK) return rc;
+  // The tensor map depends only on the V buffer and its row count; reuse the
+  // last encoding while they are unchanged (encoding costs host time every step).
+  static thread_local const void* last_base = nullptr;
+  static thread_local uint64_t last_rows = 0;
+  static thread_local CUtensorMap tmap;
+  const uint64_t rows = (uint64_t)c->B * c->Hkv * c->Tcap;
+  int rc = AQUA_OK;
+  if (last_base != c->v || last_rows != rows) {
+    if ((rc = encode_tmap_bf16_2d(&tmap, c->v, D, rows, D * 2, 64, S::TT, true)) != AQUA_OK) return rc;
+    last_base = c->v;
+    last_rows = rows;
+  }
   if ((rc = launch_qproj<__nv_bfloat16, G>(p, n_units, st)) != AQUA_OK) return rc;
-  decode_attn_bf16_kernel<G><<<C, NTHREADS_BF16, S::BYTES, st>>>(tmap, p);
+  const cudaError_t e = launch_pdl(decode_attn_bf16_kernel<G>, dim3(C), dim3(NTHREADS_BF16), S::BYTES, st, tmap, p);
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_bf16_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attn_bf16_kernel");
 }
 
@@ -1234,7 +1290,8 @@ int launch_decode_f32(const DecodeParams& p, int n_units, int C, cudaStream_t st
   }
   int rc = launch_qproj<float, G>(p, n_units, st);
   if (rc != AQUA_OK) return rc;
-  decode_attn_f32_kernel<G><<<C, NTHREADS, S::BYTES, st>>>(p);
+  const cudaError_t e = launch_pdl(decode_attn_f32_kernel<G>, dim3(C), dim3(NTHREADS), S::BYTES, st, p);
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_f32_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attn_f32_kernel");
 }
 

@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
                                                            float* score, int32_t* ctrl, int B, int L,
                                                            int Hkv, int d_store, int Tcap) {
   extern __shared__ __align__(128) float Ps[];   // [D][D]
+  __shared__ __align__(16) float xs[8][D];        // one key row per warp
   __shared__ __align__(8) uint64_t pbar;
   __shared__ int is_last;
   const int g = blockIdx.y, b = blockIdx.z;
@@ -80,16 +81,11 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     const size_t row = ((size_t)b * L + l) * Hkv + g;
     float kv[4];
     load4<T>(k_new + row * D + 4 * lane, kv);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-    for (int i = 0; i < D; ++i) {
-      const float ki = __shfl_sync(0xffffffffu, kv[i & 3], i >> 2);
-      const float4 pr = reinterpret_cast<const float4*>(Ps + i * D)[lane];
-      acc[0] = fmaf(ki, pr.x, acc[0]);
-      acc[1] = fmaf(ki, pr.y, acc[1]);
-      acc[2] = fmaf(ki, pr.z, acc[2]);
-      acc[3] = fmaf(ki, pr.w, acc[3]);
-    }
+    *reinterpret_cast<float4*>(&xs[warp][4 * lane]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+    __syncwarp();
+    float acc[4];
+    project_row_smem(Ps, xs[warp], lane, acc);
+    __syncwarp();
     const int slot = base + l;
     const size_t unit = (size_t)b * Hkv + g;
     T* kp = kproj + unit * d_store * (size_t)Tcap + slot;
