@@ -45,6 +45,25 @@ DEFAULT_WORKLOAD = "llama3.1-8b-decode"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def profile_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
+    or None when the kernel source changed since that capture."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "decode_attn_bf16_llama3.1-8b-decode.md")
+    src = os.path.join(ROOT, "sparse_dimension_attention_b200", "csrc", "decode.cu")
+    try:
+        txt = open(prof).read()
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if ("source sha256: " + digest) not in txt:
+            return None
+        for ln in txt.splitlines():
+            if ln.startswith("traffic_bytes_per_launch:"):
+                return int(ln.split(":")[1])
+    except Exception:
+        return None
+    return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -446,7 +465,9 @@ def main():
         "hbm_gbs": step_gbs,
         "mean_union": float(usz.mean()),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
+                     "frac": achieved / hbm_peak, "traffic": profile_traffic(),
+                     "traffic_note": "ncu DRAM read+write bytes of one decode_attn_bf16_kernel launch "
+                                     "(profiles/decode_attn_bf16_llama3.1-8b-decode.md); null if the kernel changed",
                      "kernel": "aqua_decode_attn step (qproj_topk_kernel with fused append + decode_attn_bf16_kernel)",
                      "peak_source": peak_kind,
                      "step_us": 1e3 * statistics.mean(step_ms)},
