@@ -172,6 +172,29 @@ AQUA_API int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_ne
                               void* workspace, size_t workspace_bytes, aqua_stream_t stream);
 
 /*
+ * The decode step of aqua_decode_attn for callers that cannot provide device
+ * scratch memory: their device memory belongs to another allocator they may
+ * not bypass with cudaMalloc (a framework pool, a fixed memory budget), or
+ * their interface has no place for a workspace buffer.  The paper has no
+ * counterpart to this entry point; it is an interface convenience.
+ *   - Arguments and results as aqua_decode_attn, without workspace and
+ *     workspace_bytes.  Nothing is allocated or freed.
+ *   - The scratch is an 8 MiB array inside the library's device image; every
+ *     GPU that loads the library keeps it until the library is unloaded.
+ *     AQUA_ERR_WORKSPACE if the shape needs more (aqua_decode_workspace_size
+ *     gives the need); nothing is launched then.
+ *   - The first call on a device looks up the array's address on that device;
+ *     make that first call before any stream capture.
+ *   - All calls share the array, which keeps the previous call's contents; the
+ *     kernels re-initialise what they depend on.  Calls that overlap on the GPU
+ *     (e.g. on two streams) race on it and must be ordered by the caller.
+ */
+AQUA_API int aqua_decode_attn_static(aqua_cache* cache, const void* q, const void* k_new, const void* v_new,
+                                     const float* P, int Hq, int k, float scale, void* out, int out_dtype,
+                                     int32_t* sel_out, float* qproj_out, float* scores_out, float* lse_out,
+                                     aqua_stream_t stream);
+
+/*
  * Causal AQUA attention for a chunk of L prompt tokens at absolute positions
  * pos0 .. pos0+L-1 of every sequence (their keys must already be appended, so
  * len[b] >= pos0 + L).  Row i of sequence b attends to slots 0 .. pos0+i; each

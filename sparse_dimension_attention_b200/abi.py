@@ -28,7 +28,7 @@ EXPORTED = (
     "aqua_last_error", "aqua_version", "aqua_status",
     "aqua_calibrate_workspace_size", "aqua_calibrate",
     "aqua_project_keys",
-    "aqua_decode_workspace_size", "aqua_decode_attn",
+    "aqua_decode_workspace_size", "aqua_decode_attn", "aqua_decode_attn_static",
     "aqua_prefill_workspace_size", "aqua_prefill_attn",
     "aqua_h2o_update",
 )
@@ -74,6 +74,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "aqua_project_keys": (c_int, [C, P, P, P, c_int, P]),
         "aqua_decode_workspace_size": (c_size_t, [C, c_int]),
         "aqua_decode_attn": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
+        "aqua_decode_attn_static": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P]),
         "aqua_prefill_workspace_size": (c_size_t, [C, c_int, c_int]),
         "aqua_prefill_attn": (c_int, [C, P, c_int, c_int, P, c_int, c_int, c_float, P, c_int, P, P, c_size_t, P]),
         "aqua_h2o_update": (c_int, [C, P, P, c_int, c_int, c_int, P, P]),
@@ -150,6 +151,17 @@ def aqua_decode_attn(cache: aqua_cache, q, P, Hq: int, k: int, out, workspace, s
         ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(P), Hq, k, scale, _ptr(out), out_dtype,
         _ptr(sel_out), _ptr(qproj_out), _ptr(scores_out), _ptr(lse_out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def aqua_decode_attn_static(cache: aqua_cache, q, P, Hq: int, k: int, out, scale: float = 0.0, k_new=None,
+                            v_new=None, sel_out=None, qproj_out=None, scores_out=None, lse_out=None,
+                            stream=None) -> None:
+    """The decode step without a workspace argument, for callers that cannot allocate
+    device scratch: the library's built-in 8 MiB scratch array is used instead."""
+    out_dtype = AQUA_BF16 if str(out.dtype) == "torch.bfloat16" else AQUA_F32
+    _check(load_library().aqua_decode_attn_static(
+        ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(P), Hq, k, scale, _ptr(out), out_dtype,
+        _ptr(sel_out), _ptr(qproj_out), _ptr(scores_out), _ptr(lse_out), _stream(stream)))
 
 
 def aqua_prefill_workspace_size(cache: aqua_cache, Hq: int, L: int) -> int:
