@@ -24,7 +24,7 @@ def calib_P(Hkv: int = 1, n_q: int = 8192, n_k: int = 8192) -> tuple[np.ndarray,
 
 
 def tdev(x: np.ndarray, dtype=torch.float32) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(x)).to(dtype).cuda()
+    return torch.from_numpy(np.array(x, order="C", copy=True)).to(dtype).cuda()
 
 
 def torch_dtype(kv: str):
