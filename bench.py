@@ -42,6 +42,11 @@ WORKLOADS = {
     "tiny-f32-decode": dict(B=1, Hq=4, Hkv=1, T=1024, k=96, kv="f32", d_store=128),
 }
 DEFAULT_WORKLOAD = "llama3.1-8b-decode"
+# chunked causal prefill: a 4096-token prompt in 512-token chunks (Llama-3.1-8B heads)
+PREFILL = dict(B=1, Hq=32, Hkv=8, L_total=4096, chunk=512, k=96)
+# truncated cache (first m projected dims stored), k within them, H2O budget of
+# `recent` newest + heavy hitters; absolute length runs from `budget` to T_end
+H2O_WL = dict(B=32, Hq=32, Hkv=8, m=96, k=64, budget=2048, recent=256, T_end=32768)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -342,6 +347,190 @@ class DecodeBench:
         return ms, h2d, d2h
 
 
+class PrefillBench:
+    """A prompt pass = for every chunk: aqua_project_keys (append the chunk's keys
+    and values), then aqua_prefill_attn (selection + tcgen05 attention)."""
+
+    def __init__(self, wl: dict, P):
+        import torch
+        import sparse_dimension_attention_b200 as aq
+        self.aq, self.torch, self.wl, self.P = aq, torch, wl, P[:wl["Hkv"]].contiguous()
+        inp = synth.prefill_inputs(wl["L_total"], wl["Hq"], wl["Hkv"], bf16=True, B=wl["B"])
+        bf = torch.bfloat16
+        self.q = torch.from_numpy(inp["q"]).to(bf).cuda()          # [B, L, Hq, d]
+        self.k = torch.from_numpy(inp["k"]).to(bf).cuda()          # [B, L, Hkv, d]
+        self.v = torch.from_numpy(inp["v"]).to(bf).cuda()
+        self.cache = aq.AquaCache(wl["B"], wl["Hkv"], wl["L_total"] + 128)
+        self.out = torch.empty((wl["B"], wl["chunk"], wl["Hq"], 128), dtype=bf, device="cuda")
+        self.ws = torch.empty(aq.aqua_prefill_workspace_size(self.cache.desc, wl["Hq"], wl["chunk"]),
+                              dtype=torch.uint8, device="cuda")
+        self.n_chunks = wl["L_total"] // wl["chunk"]
+
+    def one_pass(self, k: int, ev=None):
+        aq, wl, C = self.aq, self.wl, self.wl["chunk"]
+        self.cache.reset()
+        for c in range(self.n_chunks):
+            s = c * C
+            aq.aqua_project_keys(self.cache.desc, self.k[:, s:s + C], self.v[:, s:s + C], self.P, C)
+            if ev is not None:
+                ev[c][0].record()
+            aq.aqua_prefill_attn(self.cache.desc, self.q[:, s:s + C], s, C, self.P, wl["Hq"], k, self.out, self.ws)
+            if ev is not None:
+                ev[c][1].record()
+
+    def flops(self, pos0: int):
+        """(dense causal flops, tensor-core flops issued) of one aqua_prefill_attn chunk call.
+        Dense causal: 2 d flops for q.k and 2 d for p.v per visible (row, token) per
+        query head.  Issued: the kernel's MMAs, bf16 high+low parts of the masked
+        query and of P, over every 128-token tile each 128-row CTA visits."""
+        wl, C, d = self.wl, self.wl["chunk"], 128
+        G = wl["Hq"] // wl["Hkv"]
+        pairs = C * pos0 + C * (C + 1) // 2
+        dense = pairs * wl["Hq"] * 4.0 * d
+        rpb = 128 // G
+        tiles = sum(-(-(pos0 + min(C, (qb + 1) * rpb)) // 128) for qb in range(-(-C // rpb)))
+        issued = tiles * wl["Hkv"] * wl["B"] * (2 * 2.0 * 128 * 128 * d + 2 * 2.0 * 128 * 128 * 128)
+        return dense, issued
+
+    def timed(self, K: int, W: int, k: int):
+        torch = self.torch
+        for _ in range(W):
+            self.one_pass(k)
+        torch.cuda.synchronize()
+        E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        passes, attn = [], np.zeros(self.n_chunks)
+        for _ in range(K):
+            ev = [(E(), E()) for _ in range(self.n_chunks)]
+            p0, p1 = E(), E()
+            p0.record()
+            self.one_pass(k, ev)
+            p1.record()
+            torch.cuda.synchronize()
+            passes.append(p0.elapsed_time(p1))
+            attn += np.array([a.elapsed_time(b) for a, b in ev])
+        return float(np.mean(passes)), attn / K                       # ms per prompt, ms per chunk call
+
+    def report(self, K: int, W: int, bf16_peak: float, peak_kind: str) -> dict:
+        wl = self.wl
+        prompt_ms, attn_ms = self.timed(K, W, wl["k"])
+        dense_ms, dense_attn = self.timed(K, W, 128)
+        fl = [self.flops(c * wl["chunk"]) for c in range(self.n_chunks)]
+        dense_f = sum(f[0] for f in fl)
+        issued_f = sum(f[1] for f in fl)
+        t_attn = float(attn_ms.sum()) / 1e3
+        alg = dense_f / t_attn / 1e12
+        return {"workload": "chunked-prefill-4096", **wl, "d": 128,
+                "prompt_ms": prompt_ms, "tokens_per_s": wl["B"] * wl["L_total"] / (prompt_ms / 1e3),
+                "attn_call_us": [round(1e3 * x, 2) for x in attn_ms],
+                "roofline": {"bound": "tensor", "achieved": alg, "peak": bf16_peak, "unit": "TFLOP/s",
+                             "frac": alg / bf16_peak, "peak_source": peak_kind + " bf16 burst",
+                             "achieved_note": "dense causal flops (4 d per visible pair and query head, "
+                                              "%.1f GFLOP per prompt) / summed aqua_prefill_attn call time "
+                                              "(selection + attention kernels)" % (dense_f / 1e9),
+                             "issued_tflops": issued_f / t_attn / 1e12,
+                             "issued_note": "tcgen05 flops issued (bf16 high+low splits, whole 128-token tiles)"},
+                "dense_k128_prompt_ms": dense_ms,
+                "speedup_vs_dense": dense_ms / prompt_ms,
+                "l2": "not flushed: a chunk's K~/V (<= 16 MB) were written by the append just before"}
+
+
+class H2OBench:
+    """Steady-state decode on a truncated cache with H2O eviction.  A step is
+    aqua_decode_attn (fused append of the step's key/value, scores and lse out)
+    followed by aqua_h2o_update (accumulate scores, evict one token): 3 launches."""
+
+    GRAPH_STEPS = 256
+
+    def __init__(self, wl: dict, P):
+        import torch
+        import sparse_dimension_attention_b200 as aq
+        self.aq, self.torch, self.wl = aq, torch, wl
+        self.P = P[:wl["Hkv"]].contiguous()
+        B, Hq, Hkv, n0 = wl["B"], wl["Hq"], wl["Hkv"], wl["budget"]
+        self.n_in = 64
+        inp = synth.decode_inputs(B, Hq, Hkv, n0, bf16=True, steps=self.n_in)
+        bf = torch.bfloat16
+        self.cache = aq.AquaCache(B, Hkv, n0 + 16, d_store=wl["m"], h2o=True)
+        for s0 in range(0, n0, 1024):                                       # warm-up fill: positions 0 .. budget-1
+            e0 = min(n0, s0 + 1024)
+            aq.aqua_project_keys(self.cache.desc, torch.from_numpy(np.ascontiguousarray(inp["k_hist"][:, s0:e0])).to(bf).cuda(),
+                                 torch.from_numpy(np.ascontiguousarray(inp["v_hist"][:, s0:e0])).to(bf).cuda(), self.P, e0 - s0)
+        self.q = torch.from_numpy(inp["q"]).to(bf).cuda()
+        self.kn = torch.from_numpy(inp["k_new"]).to(bf).cuda()
+        self.vn = torch.from_numpy(inp["v_new"]).to(bf).cuda()
+        Tc = self.cache.Tcap
+        self.sc = torch.zeros((B, Hq, Tc), dtype=torch.float32, device="cuda")
+        self.lse = torch.zeros((B, Hq), dtype=torch.float32, device="cuda")
+        self.out = torch.empty((B, Hq, 128), dtype=bf, device="cuda")
+        self.ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
+        self.ws = torch.empty(aq.aqua_decode_workspace_size(self.cache.desc, Hq), dtype=torch.uint8, device="cuda")
+        self.n_steps = 0
+        torch.cuda.synchronize()
+
+    def step(self, sel=None):
+        aq, wl, i = self.aq, self.wl, self.n_steps % self.n_in
+        aq.aqua_decode_attn(self.cache.desc, self.q[i], self.P, wl["Hq"], wl["k"], self.out, self.ws,
+                            k_new=self.kn[i], v_new=self.vn[i], scores_out=self.sc, lse_out=self.lse, sel_out=sel)
+        aq.aqua_h2o_update(self.cache.desc, self.sc, self.lse, wl["Hq"], wl["budget"], wl["recent"], self.ev)
+        self.n_steps += 1
+
+    def bytes_step(self, usz: float) -> float:
+        """Algorithmic HBM bytes of one step at n = budget+1 attended tokens per (b, g):
+        K~ union rows and V rows, the scores write and read-back, the cumulative
+        score/position arrays, the append, q and the output."""
+        wl = self.wl
+        B, Hq, Hkv, n = wl["B"], wl["Hq"], wl["Hkv"], wl["budget"] + 1
+        units = B * Hkv
+        attn = units * n * (2.0 * usz + 2 * 128)
+        scores = 2.0 * B * Hq * n * 4                       # written by the decode, read by the update
+        h2o = units * n * (4 + 4 + 4)                       # score read + write, pos read
+        move = units * (wl["m"] + 128) * 2 * 2              # victim slot <- last slot
+        append = units * (128 * 2 * 2 + wl["m"] * 2 + 128 * 2)
+        qo = B * Hq * 128 * 2 * 2
+        return attn + scores + h2o + move + append + qo
+
+    def report(self, W: int) -> dict:
+        torch, wl = self.torch, self.wl
+        G = wl["Hq"] // wl["Hkv"]
+        for _ in range(W):
+            self.step()
+        usz = []
+        for _ in range(4):
+            sel = torch.empty((wl["B"], wl["Hq"], wl["k"]), dtype=torch.int32, device="cuda")
+            self.step(sel)
+            m = torch.zeros((wl["B"], wl["Hq"], 128), dtype=torch.bool, device="cuda")
+            m.scatter_(2, sel.long(), True)
+            usz.append(float(m.view(wl["B"], wl["Hkv"], G, 128).any(2).sum(-1).float().mean()))
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(self.GRAPH_STEPS):
+                self.step()
+        g.replay()                                                           # upload; state advances
+        torch.cuda.synchronize()
+        t_abs0 = wl["budget"] + self.n_steps                               # tokens seen so far
+        reps = max(1, (wl["T_end"] - t_abs0) // self.GRAPH_STEPS)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        del g
+        K = reps * self.GRAPH_STEPS
+        n_len = int(self.cache.len[0].item())
+        status = self.aq.aqua_status(self.cache.desc)
+        by = self.bytes_step(float(np.mean(usz)))
+        return {"workload": "truncated-h2o-decode", **wl, "d": 128,
+                "steps": K, "T_abs_range": [t_abs0, t_abs0 + K], "cache_len_after": n_len, "status": status,
+                "queries_per_s": wl["B"] * K / (ms / 1e3), "ms_per_step": ms / K,
+                "mean_union": float(np.mean(usz)), "bytes_per_step": by,
+                "hbm_gbs": by * K / (ms / 1e3) / 1e9,
+                "launch": "%d-step CUDA graph replayed %d times; 3 launches per step" % (self.GRAPH_STEPS, reps),
+                "l2": "no flush: each step streams %.0f MB, above the 126 MB L2" % (by / 1e6)}
+
+
 def cpu_baseline(wl: dict, budget_s: float = 12.0) -> dict:
     """The oracle, as it stands, on the host cores: decode steps of one sequence
     (all its query heads) repeated until about budget_s seconds have run."""
@@ -435,7 +624,7 @@ def main():
     if args.k is not None:
         wl["k"] = args.k
     K, W = args.steps, args.warmup
-    hbm_peak, _, peak_kind = peaks()
+    hbm_peak, bf16_peak, peak_kind = peaks()
 
     bench = DecodeBench(wl, K, W)
     usz = bench.union_sizes(wl["k"], min(K, bench.n_in))                       # [K, B, Hkv]
@@ -507,7 +696,18 @@ def main():
                                 "queries_per_s": world * Kl / (t_ms / 1e3), "ms_per_step": t_ms / Kl,
                                 "decode_us": 1e3 * statistics.mean(d_ms), "decode_gbs": ach,
                                 "frac": ach / hbm_peak}
+        P = lb.P
         del lb
+        torch.cuda.empty_cache()
+        pb = PrefillBench(PREFILL, P)
+        line["prefill"] = pb.report(min(K, 20), W, bf16_peak, peak_kind)
+        del pb
+        torch.cuda.empty_cache()
+        hb = H2OBench(H2O_WL, P)
+        r = hb.report(W)
+        r["frac"] = r["hbm_gbs"] / hbm_peak
+        line["truncated_h2o"] = r
+        del hb
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

@@ -203,6 +203,12 @@ AQUA_API int aqua_decode_attn_static(aqua_cache* cache, const void* q, const voi
  *   q    [B][L][Hq][d] cache dtype (bf16 only)
  *   out  [B][L][Hq][d] out_dtype
  *   sel_out nullable [B][L][Hq][k] int32
+ *   workspace  device, 256-byte aligned, >= aqua_prefill_workspace_size bytes
+ *              (a small reserved block: projection, selection and attention
+ *              run in one kernel and keep their intermediates on chip)
+ * Requires Hq/Hkv in {1, 2, 4}, d_store a multiple of 16, k <= d_store.
+ * A wait that exceeds its time limit inside the kernel records
+ * AQUA_ERR_TIMEOUT in the cache's status word (aqua_status).
  */
 AQUA_API size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L);
 AQUA_API int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, const float* P,

@@ -39,8 +39,9 @@ int device_sm_count() {
   return n;
 }
 
-int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                        uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+namespace {
+// cuTensorMapEncodeTiled from the driver, resolved once through the runtime
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -50,17 +51,37 @@ int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint6
         q == cudaDriverEntryPointSuccess)
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
+  return encode;
+}
+
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                     const cuuint64_t* strides_bytes, const cuuint32_t* box, bool swizzle128) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tmap_encoder();
   if (encode == nullptr) return set_error(AQUA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                            strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(AQUA_ERR_CUDA, "cuTensorMapEncodeTiled (rank %d) failed (%d)", rank, (int)r);
+  return AQUA_OK;
+}
+}  // namespace
+
+int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                        uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {row_stride_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(AQUA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return AQUA_OK;
+  return encode_tmap_bf16(map, base, 2, dims, strides, box, swizzle128);
+}
+
+int encode_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
+                        const uint32_t box[3], bool swizzle128) {
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  return encode_tmap_bf16(map, base, 3, d, st, bx, swizzle128);
 }
 
 // launchers (defined next to their kernels)

@@ -31,6 +31,11 @@ int device_sm_count();
 // shared-memory swizzle.  Returns AQUA_OK or AQUA_ERR_CUDA.
 int encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                         uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+// 3-D tiled tensor map over a bf16 array with dims {d0 (contiguous), d1, d2},
+// byte strides of d1 and d2, and box {b0, b1, b2} (written to shared memory
+// with d0 fastest, then d1, then d2).
+int encode_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[3], const uint64_t strides_bytes[2],
+                        const uint32_t box[3], bool swizzle128);
 
 // Launch with programmatic stream serialization: the kernel may begin while
 // the previous kernel in the stream is still running; it must call pdl_wait()
@@ -86,6 +91,37 @@ __device__ __forceinline__ void project_row_smem(const float* Ps, const float* x
   }
 #pragma unroll
   for (int s = 0; s < 4; ++s) y[s] = a[s] + b[s];
+}
+
+// project_row_smem for NR row vectors at once (xs: NR rows of kHeadDim floats,
+// consecutive): every output element is summed in exactly the same order as
+// project_row_smem, so the results are bit-identical; P is read once per NR rows.
+template <int NR>
+__device__ __forceinline__ void project_rows_smem(const float* Ps, const float* xs, int lane, float (&y)[NR][4]) {
+  float a[NR][4], b[NR][4];
+#pragma unroll
+  for (int t = 0; t < NR; ++t)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) a[t][s] = b[t][s] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < kHeadDim; i += 4) {
+    const float4 p0 = reinterpret_cast<const float4*>(Ps + (i + 0) * kHeadDim)[lane];
+    const float4 p1 = reinterpret_cast<const float4*>(Ps + (i + 1) * kHeadDim)[lane];
+    const float4 p2 = reinterpret_cast<const float4*>(Ps + (i + 2) * kHeadDim)[lane];
+    const float4 p3 = reinterpret_cast<const float4*>(Ps + (i + 3) * kHeadDim)[lane];
+#pragma unroll
+    for (int t = 0; t < NR; ++t) {
+      const float4 x4 = *reinterpret_cast<const float4*>(xs + t * kHeadDim + i);
+      a[t][0] = fmaf(x4.x, p0.x, a[t][0]); a[t][1] = fmaf(x4.x, p0.y, a[t][1]); a[t][2] = fmaf(x4.x, p0.z, a[t][2]); a[t][3] = fmaf(x4.x, p0.w, a[t][3]);
+      b[t][0] = fmaf(x4.y, p1.x, b[t][0]); b[t][1] = fmaf(x4.y, p1.y, b[t][1]); b[t][2] = fmaf(x4.y, p1.z, b[t][2]); b[t][3] = fmaf(x4.y, p1.w, b[t][3]);
+      a[t][0] = fmaf(x4.z, p2.x, a[t][0]); a[t][1] = fmaf(x4.z, p2.y, a[t][1]); a[t][2] = fmaf(x4.z, p2.z, a[t][2]); a[t][3] = fmaf(x4.z, p2.w, a[t][3]);
+      b[t][0] = fmaf(x4.w, p3.x, b[t][0]); b[t][1] = fmaf(x4.w, p3.y, b[t][1]); b[t][2] = fmaf(x4.w, p3.z, b[t][2]); b[t][3] = fmaf(x4.w, p3.w, b[t][3]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NR; ++t)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) y[t][s] = a[t][s] + b[t][s];
 }
 
 __device__ __forceinline__ void store_out(float* p, float x) { *p = x; }

@@ -5,22 +5,27 @@
 // keeps its k largest |q~| dimensions (ties to the lower index), and attends
 // causally to tokens 0 .. pos0+i with scores on those dimensions only
 // (AQUA abstract; edgentiq, "How AQUA Works": project, select by query
-// magnitude, attend on the selected dimensions; the per-query mask makes the
-// score a dense contraction over a masked q~).
+// magnitude, attend on the selected dimensions).  The per-row mask turns the
+// score into a dense contraction over a masked q~, which runs on tcgen05.
 //
-// prefill_select_kernel: one warp per (row, head): q~ = q P[g] (f32, shared
-//   routine), radix select, masked q~ * scale * log2(e) split into bf16 high
-//   and low parts, written row-major in (b, g, row, head) order.
-// prefill_attn_kernel: one CTA per (b, g, block of 128/G rows), i.e. 128 query
-//   rows of one GQA group that share every K~/V tile.  Warp roles:
-//     warps 0-3  softmax (thread r <-> TMEM lane r <-> query row r)
-//     warp 4     TMEM allocation and the single thread issuing tcgen05.mma
-//     warp 5     TMA producer
-//   Per 128-token KV tile: S = Qh K~ + Ql K~ (M=128, N=128, K=d_store) into
-//   TMEM, causal mask, online softmax with a lazily raised running max,
-//   P split into bf16 high/low parts in shared memory, O += Ph V + Pl V
-//   (K=128 tokens, N=128 dims) into TMEM.  Operands are 128B-swizzled tiles:
-//   Q~m and P K-major, the dimension-major K~ and token-major V MN-major.
+// One kernel, one CTA per (sequence b, KV head g, block of 128/G prompt rows):
+// the 128 TMEM lanes are the 128 (row, head) query rows of one GQA group, which
+// share every K~/V tile.  Warp roles (320 threads):
+//   warps 0-3  softmax warpgroup 0: S columns 0-63 / O columns 0-63, and the
+//              per-row top-k selection in the prologue
+//   warps 4-7  softmax warpgroup 1: S columns 64-127 / O columns 64-127
+//   warp 8     TMEM allocation and the single thread issuing tcgen05.mma
+//   warp 9     TMA producer
+// Prologue: q~ = q P on the tensor cores (P split into three bf16 parts, f32
+// accumulation, so q~ carries ~24 bits), selection per row from TMEM, masked
+// q~ * scale * log2(e) written as bf16 high and low parts (K-major tiles).
+// Per 128-token KV tile j: S = Qh K~ + Ql K~ (M=128, N=128, K=d_store) into
+// TMEM; the softmax warps copy S to registers and release it, so S(j+1) is
+// computed while tile j's softmax runs (K~ and V tiles double-buffered); causal
+// mask on diagonal tiles, online softmax with a lazily raised running max, P
+// split into bf16 high/low parts written to tensor memory, O += Ph V + Pl V with
+// the A operand read from tensor memory (shared-memory bandwidth is the limit of
+// this loop: P never goes through it).
 #include <math.h>
 
 #include "aqua_internal.cuh"
@@ -32,9 +37,7 @@ namespace {
 constexpr int D = kHeadDim;
 constexpr int PM = 128;          // query rows per CTA (TMEM lanes)
 constexpr int PN = 128;          // tokens per KV tile
-constexpr int kSelWarps = 8;     // selection kernel: warps per CTA
-constexpr int kSelRows = 64;     // selection kernel: (row, head) pairs per CTA
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
 constexpr float kLazy = 8.0f;    // running max raised only when exceeded by 2^8
 
 // ------------------------------------------------------------------ tcgen05 wrappers
@@ -61,6 +64,18 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: A (M rows x K) read from tensor memory,
+// row i in lane i, 16-bit elements packed two per 32-bit column (K-major)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
       : "memory");
 }
 
@@ -118,9 +133,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 }
 
 struct PrefillParams {
-  const void* q;             // [B][L][Hq][D] bf16
   const float* P;            // [Hkv][D][D]
-  __nv_bfloat16* qm;         // [2][B*Hkv*L*G][D]: masked scaled q~, high part then low part
   void* out;                 // [B][L][Hq][D]
   int32_t* sel_out;          // nullable [B][L][Hq][k]
   int32_t* ctrl;
@@ -129,128 +142,110 @@ struct PrefillParams {
   float scale_log2;
 };
 
-// ============================================================================
-// selection: q~ = q P, top-k by |q~|, masked pre-scaled rows as bf16 hi / lo
-// ============================================================================
-template <int G>
-__global__ void __launch_bounds__(kSelWarps * 32) prefill_select_kernel(PrefillParams p) {
-  extern __shared__ __align__(128) float Ps[];
-  __shared__ __align__(16) float xs[kSelWarps][D];
-  __shared__ __align__(8) uint64_t pbar;
-  const int g = blockIdx.y, b = blockIdx.z;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t rows_total = (size_t)p.B * p.Hkv * p.L * G;
-  if (threadIdx.x == 0) {
-    mbar_init(&pbar, 1);
-    fence_barrier_init();
-  }
-  pdl_launch_dependents();
-  pdl_wait();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&pbar, D * D * 4);
-    bulk_g2s_plain(Ps, p.P + (size_t)g * D * D, D * D * 4, &pbar);
-  }
-  const bool ok = mbar_wait_bounded(&pbar, 0);
-  if (__syncthreads_or(!ok)) {
-    if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
-    return;
-  }
-  const int m = p.d_store;
-  for (int i = w; i < kSelRows; i += kSelWarps) {
-    const int pair = blockIdx.x * kSelRows + i;    // (row l, head hh) within this (b, g)
-    const int l = pair / G, hh = pair % G;
-    if (l >= p.L) break;
-    const int h = g * G + hh;
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (((size_t)b * p.L + l) * p.Hq + h) * D;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) xs[w][4 * lane + s] = __bfloat162float(qrow[4 * lane + s]);
-    __syncwarp();
-    float qt[4];
-    project_row_smem(Ps, xs[w], lane, qt);
-    __syncwarp();
-    uint32_t key[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int j = 4 * lane + s;
-      key[s] = (j < m) ? (__float_as_uint(fabsf(qt[s])) + 1u) : 0u;
-    }
-    uint32_t tau = 0;
-#pragma unroll 4
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      const int c = __popc(__ballot_sync(0xffffffffu, key[0] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[1] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[2] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[3] >= cand));
-      if (c >= p.k) tau = cand;
-    }
-    int ngt = 0, neq = 0;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      ngt += __popc(__ballot_sync(0xffffffffu, key[s] > tau));
-      neq += (key[s] == tau);
-    }
-    const int need = p.k - ngt;
-    int incl = neq;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int rank = incl - neq;
-    bool sel[4];
-    int nsel = 0;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      sel[s] = key[s] > tau;
-      if (key[s] == tau) {
-        sel[s] = rank < need;
-        ++rank;
-      }
-      nsel += sel[s];
-    }
-    if (p.sel_out) {
-      int pincl = nsel;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, pincl, o);
-        if (lane >= o) pincl += y;
-      }
-      int opos = pincl - nsel;
-      int32_t* so = p.sel_out + (((size_t)b * p.L + l) * p.Hq + h) * p.k;
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        if (sel[s]) so[opos++] = 4 * lane + s;
-    }
-    const size_t row = (((size_t)b * p.Hkv + g) * p.L + l) * G + hh;
-    __nv_bfloat16* hi_row = p.qm + row * D;
-    __nv_bfloat16* lo_row = p.qm + (rows_total + row) * D;
-    float hv[4], lv[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s) split_bf16(sel[s] ? qt[s] * p.scale_log2 : 0.f, hv[s], lv[s]);
-    *reinterpret_cast<uint2*>(hi_row + 4 * lane) = make_uint2(pack_bf16(hv[0], hv[1]), pack_bf16(hv[2], hv[3]));
-    *reinterpret_cast<uint2*>(lo_row + 4 * lane) = make_uint2(pack_bf16(lv[0], lv[1]), pack_bf16(lv[2], lv[3]));
-  }
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
 }
 
-// ============================================================================
-// causal attention on tcgen05
-// ============================================================================
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 2^x on the SFU; results below the normal range flush to zero (they are
+// softmax weights at least 2^-126 below the row's running maximum).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// x ~= hi + lo, both bf16 by truncation: hi = x with the low 16 bits cleared,
+// lo = (x - hi) likewise (x - hi is exact in f32).  |x - hi - lo| < 2^-14 |x|.
+// Returns hi and lo as f32 bit patterns with zero low halves; integer and
+// logic instructions only.
+__device__ __forceinline__ void split_trunc(float x, uint32_t& hi, uint32_t& lo) {
+  hi = __float_as_uint(x) & 0xffff0000u;
+  lo = __float_as_uint(x - __uint_as_float(hi)) & 0xffff0000u;
+}
+// two bf16 values held as f32 bit patterns with zero low halves -> one packed word (first in the low half)
+__device__ __forceinline__ uint32_t pack_hi_halves(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x7632); }
+
 struct AttnSmem {
-  static constexpr int TILE = PM * 128;              // 128 rows x 128 B = 16 KB (one 64-column half)
-  static constexpr int OFF_QH = 0;                   // [2 halves][128 rows][128 B]
-  static constexpr int OFF_QL = OFF_QH + 2 * TILE;
-  static constexpr int OFF_K = OFF_QL + 2 * TILE;    // [2 token halves][<=128 dims][128 B]
-  static constexpr int OFF_V = OFF_K + 2 * TILE;     // [2 dim halves][128 tokens][128 B]
-  static constexpr int OFF_PH = OFF_V + 2 * TILE;    // [2 token halves][128 rows][128 B]
-  static constexpr int OFF_PL = OFF_PH + 2 * TILE;
-  static constexpr int OFF_BAR = OFF_PL + 2 * TILE;  // 8 mbarriers
-  static constexpr int OFF_MISC = OFF_BAR + 8 * 8;
+  static constexpr int TILE = 128 * 128;             // 128 rows x 128 B = 16 KB (one 64-column half)
+  static constexpr int OFF_QH = 0;                   // [2 dim halves][128 rows][128 B]; prologue: P part 3
+  static constexpr int OFF_QL = OFF_QH + 2 * TILE;   // prologue: the raw query rows
+  static constexpr int OFF_K0 = OFF_QL + 2 * TILE;   // K~ buffer 0: [2 token halves][d_store rows][128 B]
+  static constexpr int OFF_K1 = OFF_K0 + 2 * TILE;   // K~ buffer 1
+  static constexpr int OFF_V0 = OFF_K1 + 2 * TILE;   // V buffer 0: [2 dim halves][128 tokens][128 B]
+  static constexpr int OFF_V1 = OFF_V0 + 2 * TILE;   // V buffer 1; prologue: P part 1
+  static constexpr int OFF_PP = OFF_V1 + 2 * TILE;   // prologue: P part 2
+  static constexpr int OFF_RED = OFF_PP + 2 * TILE;  // float [2][128]: row max / row sum exchange
+  static constexpr int OFF_BAR = OFF_RED + 2 * 128 * 4;
+  static constexpr int N_BAR = 24;
+  static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int USED = OFF_MISC + 64;
   static constexpr int BYTES = USED + 1024;          // + slack to align the base to the 1024-byte swizzle period
 };
-enum { BAR_Q = 0, BAR_K, BAR_V, BAR_S, BAR_P, BAR_O, BAR_DRAIN };
+enum {
+  BAR_Q = 0,     // raw query rows landed (TMA)
+  BAR_PS,        // P parts written (256 softmax threads)
+  BAR_QT,        // q~ = q P complete in TMEM (commit)
+  BAR_QM,        // masked q~ high/low parts written (128 threads of warpgroup 0)
+  BAR_KF0,       // K~ buffer 0 / 1 full (TMA)
+  BAR_KF1,
+  BAR_KE0,       // K~ buffer 0 / 1 free (commit after the QK MMAs reading it)
+  BAR_KE1,
+  BAR_VF0,       // V buffer 0 / 1 full (TMA)
+  BAR_VF1,
+  BAR_VE0,       // V buffer 0 / 1 free (commit after the P V MMAs reading it)
+  BAR_VE1,
+  BAR_S,         // S complete in TMEM (commit)
+  BAR_SF,        // S copied to registers by all 256 softmax threads
+  BAR_P,         // P written to TMEM, V tail zeroed (256 softmax threads)
+  BAR_O,         // O += P V complete (commit)
+  BAR_DRAIN,     // every MMA issued so far complete (commit)
+  BAR_COUNT
+};
+static_assert(BAR_COUNT <= AttnSmem::N_BAR, "barrier slots");
+static_assert(AttnSmem::BYTES <= 232448, "shared memory per CTA");
+constexpr int kSoftThreads = 256;
+constexpr int kMmaWarp = 8, kTmaWarp = 9;
+
+// Bounded wait that also gives up once another role raised the abort flag.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// S(j) = Qh K~(j) + Ql K~(j) into TMEM; then commits: K~ buffer j&1 free, S ready
+__device__ __forceinline__ void issue_qk(unsigned char* smem, uint32_t tm_S, int DS, int j, uint64_t* bars,
+                                         uint32_t idesc) {
+  using S = AttnSmem;
+  const int kb = (j & 1) ? S::OFF_K1 : S::OFF_K0;
+  int n = 0;
+  for (int part = 0; part < 2; ++part) {
+    const int qa = part == 0 ? S::OFF_QH : S::OFF_QL;
+    for (int ks = 0; ks < DS / 16; ++ks, ++n) {
+      const uint64_t ad = smem_desc_sw128(smem + qa + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
+      const uint64_t bd = smem_desc_sw128(smem + kb + ks * 16 * 128, DS * 128, 1024);
+      tc_mma(tm_S, ad, bd, idesc, n > 0);
+    }
+  }
+  tc_commit(&bars[BAR_KE0 + (j & 1)]);
+  tc_commit(&bars[BAR_S]);
+}
 
 template <int G>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -258,10 +253,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
   using S = AttnSmem;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // The 128B swizzle pattern (TMA, tcgen05 descriptors and the hand-written P
+  // The 128B swizzle pattern (TMA, tcgen05 descriptors and the hand-written
   // tiles) is a function of address bits 4-9: every tile starts on a 1024-byte boundary.
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::OFF_MISC + 4);
 
@@ -277,198 +273,385 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int unit = b * p.Hkv + g;
 
   if (tid == 0) {
-    for (int i = 0; i <= BAR_DRAIN; ++i) mbar_init(&bars[i], i == BAR_P ? 128 : 1);
+    for (int i = 0; i < BAR_COUNT; ++i) {
+      const int cnt = (i == BAR_PS || i == BAR_SF || i == BAR_P) ? kSoftThreads : (i == BAR_QM ? 128 : 1);
+      mbar_init(&bars[i], cnt);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
-    tmem_alloc(tmem_slot, 256);                       // S: columns [0,128), O: [128,256)
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);                       // S [0,128), P high/low [128,256), O (q~ first) [256,384)
     tmem_relinquish();
   }
-  if (tid == 160) {
+  if (tid == kTmaWarp * 32) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
   }
   pdl_launch_dependents();
-  pdl_wait();                                         // the selection kernel wrote q~m
+  pdl_wait();                                         // the previous kernel's appends are visible
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_S = tmem, tm_O = tmem + 128;
+  const uint32_t tm_S = tmem, tm_P = tmem + 128, tm_O = tmem + 256;
+  constexpr uint32_t idesc = idesc_bf16(PM, 128);
 
-  if (warp == 5) {
+  if (warp == kTmaWarp) {
     // ======================= TMA producer =======================
     if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      const int qrow = ((unit * p.L) + l0) * G;
-      const int rows_total = p.B * p.Hkv * p.L * G;
-      mbar_arrive_expect_tx(&bars[BAR_Q], 4 * S::TILE);
-      tma_load_2d(smem + S::OFF_QH, &tm_q, 0, qrow, &bars[BAR_Q], pol);
-      tma_load_2d(smem + S::OFF_QH + S::TILE, &tm_q, 64, qrow, &bars[BAR_Q], pol);
-      tma_load_2d(smem + S::OFF_QL, &tm_q, 0, rows_total + qrow, &bars[BAR_Q], pol);
-      tma_load_2d(smem + S::OFF_QL + S::TILE, &tm_q, 64, rows_total + qrow, &bars[BAR_Q], pol);
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_normal();  // every row block of this (b, g) re-reads the tiles
+      mbar_arrive_expect_tx(&bars[BAR_Q], 2 * S::TILE);
+      tma_load_3d(smem + S::OFF_QL, &tm_q, 0, g * G, b * p.L + l0, &bars[BAR_Q], pol_q);
+      tma_load_3d(smem + S::OFF_QL + S::TILE, &tm_q, 64, g * G, b * p.L + l0, &bars[BAR_Q], pol_q);
       const uint32_t kbytes = 2u * DS * 128u;
-      int nk = 0, nv = 0;                             // K~ and V tiles issued
-      for (int j = 0; j < n_tiles && !*abort_flag; ++j) {
-        const int t0 = j * PN;
-        if (j > 0 && !mbar_wait_bounded(&bars[BAR_S], (j - 1) & 1)) { *abort_flag = 1; break; }   // K~ buffer free
-        mbar_arrive_expect_tx(&bars[BAR_K], kbytes);
-        tma_load_2d(smem + S::OFF_K, &tm_k, t0, unit * DS, &bars[BAR_K], pol);
-        tma_load_2d(smem + S::OFF_K + DS * 128, &tm_k, t0 + 64, unit * DS, &bars[BAR_K], pol);
-        ++nk;
-        if (j > 0 && !mbar_wait_bounded(&bars[BAR_O], (j - 1) & 1)) { *abort_flag = 1; break; }   // V buffer free
-        mbar_arrive_expect_tx(&bars[BAR_V], 2 * S::TILE);
-        tma_load_2d(smem + S::OFF_V, &tm_v, 0, unit * p.Tcap + t0, &bars[BAR_V], pol);
-        tma_load_2d(smem + S::OFF_V + S::TILE, &tm_v, 64, unit * p.Tcap + t0, &bars[BAR_V], pol);
-        ++nv;
+      int jk = 0, jv = 0;                             // next K~ / V tile to load
+      unsigned long long t_last = globaltimer_ns();
+      while ((jk < n_tiles || jv < n_tiles) && !*abort_flag) {
+        bool progress = false;
+        // K~(jk) into buffer jk&1 once the QK MMAs of tile jk-2 are done with it
+        if (jk < n_tiles && (jk < 2 || mbar_try_wait(&bars[BAR_KE0 + (jk & 1)], ((jk - 2) >> 1) & 1))) {
+          unsigned char* kb = smem + ((jk & 1) ? S::OFF_K1 : S::OFF_K0);
+          uint64_t* kf = &bars[BAR_KF0 + (jk & 1)];
+          mbar_arrive_expect_tx(kf, kbytes);
+          tma_load_2d(kb, &tm_k, jk * PN, unit * DS, kf, pol_kv);
+          tma_load_2d(kb + DS * 128, &tm_k, jk * PN + 64, unit * DS, kf, pol_kv);
+          ++jk;
+          progress = true;
+        }
+        // V(jv) into buffer jv&1 once the P V MMAs of tile jv-2 are done with it (buffer 1
+        // holds a P part of the prologue until the projection MMAs have completed)
+        if (jv < n_tiles &&
+            (jv == 0 || (jv == 1 ? mbar_try_wait(&bars[BAR_QT], 0)
+                                 : mbar_try_wait(&bars[BAR_VE0 + (jv & 1)], ((jv - 2) >> 1) & 1)))) {
+          unsigned char* vb = smem + ((jv & 1) ? S::OFF_V1 : S::OFF_V0);
+          uint64_t* vf = &bars[BAR_VF0 + (jv & 1)];
+          mbar_arrive_expect_tx(vf, 2 * S::TILE);
+          tma_load_2d(vb, &tm_v, 0, unit * p.Tcap + jv * PN, vf, pol_kv);
+          tma_load_2d(vb + S::TILE, &tm_v, 64, unit * p.Tcap + jv * PN, vf, pol_kv);
+          ++jv;
+          progress = true;
+        }
+        const unsigned long long now = globaltimer_ns();
+        if (progress) t_last = now;
+        else if (now - t_last > kWaitLimitNs) *abort_flag = 1;
       }
-      // Before the CTA exits, every copy it issued must have landed (normally
-      // they all have been consumed already; after an abort this is the drain).
+      // every copy issued must have landed before the CTA exits
       bool drained = mbar_wait_bounded(&bars[BAR_Q], 0);
-      if (nk > 0) drained = mbar_wait_bounded(&bars[BAR_K], (nk - 1) & 1) && drained;
-      if (nv > 0) drained = mbar_wait_bounded(&bars[BAR_V], (nv - 1) & 1) && drained;
+      for (int t = max(0, jk - 2); t < jk; ++t)
+        drained = mbar_wait_bounded(&bars[BAR_KF0 + (t & 1)], (t >> 1) & 1) && drained;
+      for (int t = max(0, jv - 2); t < jv; ++t)
+        drained = mbar_wait_bounded(&bars[BAR_VF0 + (t & 1)], (t >> 1) & 1) && drained;
       if (!drained) *abort_flag = 1;
     }
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(PM, 128);
-      bool ok = mbar_wait_bounded(&bars[BAR_Q], 0);
+      bool ok = wait_or_abort(&bars[BAR_Q], 0, abort_flag) && wait_or_abort(&bars[BAR_PS], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        // q~ = q (P1 + P2 + P3): A = raw q rows (K-major), B = P parts (MN-major: input dim x output dim)
+        for (int part = 0; part < 3; ++part) {
+          const int part_off = part == 0 ? S::OFF_V1 : (part == 1 ? S::OFF_PP : S::OFF_QH);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = smem_desc_sw128(smem + S::OFF_QL + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(smem + part_off + ks * 16 * 128, S::TILE, 1024);
+            tc_mma(tm_O, ad, bd, idesc, part > 0 || ks > 0);
+          }
+        }
+        tc_commit(&bars[BAR_QT]);
+        ok = wait_or_abort(&bars[BAR_QM], 0, abort_flag);
+      }
+      if (ok) ok = wait_or_abort(&bars[BAR_KF0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(smem, tm_S, DS, 0, bars, idesc);
+      }
       for (int j = 0; j < n_tiles && ok; ++j) {
-        ok = mbar_wait_bounded(&bars[BAR_K], j & 1);
-        if (ok && j > 0) ok = mbar_wait_bounded(&bars[BAR_P], (j - 1) & 1);    // softmax done with S(j-1)
-        if (!ok) break;
-        tc_fence_after();
-        // S = Qh K~ + Ql K~: A K-major (32 B per k-step inside a 64-column half), B MN-major
-        int n = 0;
-        for (int part = 0; part < 2; ++part) {
-          const unsigned char* qa = smem + (part == 0 ? S::OFF_QH : S::OFF_QL);
-          for (int ks = 0; ks < DS / 16; ++ks, ++n) {
-            const uint64_t ad = smem_desc_sw128(qa + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(smem + S::OFF_K + ks * 16 * 128, DS * 128, 1024);
-            tc_mma(tm_S, ad, bd, idesc, n > 0);
-          }
+        if (j + 1 < n_tiles) {
+          // S is free once every softmax thread holds tile j's scores in registers
+          ok = wait_or_abort(&bars[BAR_SF], j & 1, abort_flag) &&
+               wait_or_abort(&bars[BAR_KF0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(smem, tm_S, DS, j + 1, bars, idesc);
         }
-        tc_commit(&bars[BAR_S]);
-        ok = mbar_wait_bounded(&bars[BAR_V], j & 1) && mbar_wait_bounded(&bars[BAR_P], j & 1);
+        ok = wait_or_abort(&bars[BAR_VF0 + (j & 1)], (j >> 1) & 1, abort_flag) &&
+             wait_or_abort(&bars[BAR_P], j & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // O += Ph V + Pl V
-        for (int part = 0; part < 2; ++part) {
-          const unsigned char* pa = smem + (part == 0 ? S::OFF_PH : S::OFF_PL);
+        // O += Ph V + Pl V, P (128 rows x 128 tokens, two tokens per column) from tensor memory
+        const int vb = (j & 1) ? S::OFF_V1 : S::OFF_V0;
+        for (int part = 0; part < 2; ++part)
           for (int ks = 0; ks < PN / 16; ++ks) {
-            const uint64_t ad = smem_desc_sw128(pa + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(smem + S::OFF_V + ks * 16 * 128, S::TILE, 1024);
-            tc_mma(tm_O, ad, bd, idesc, j > 0 || part > 0 || ks > 0);
+            const uint64_t bd = smem_desc_sw128(smem + vb + ks * 16 * 128, S::TILE, 1024);
+            tc_mma_ts(tm_O, tm_P + part * 64 + ks * 8, bd, idesc, j > 0 || part > 0 || ks > 0);
           }
-        }
+        tc_commit(&bars[BAR_VE0 + (j & 1)]);
         tc_commit(&bars[BAR_O]);
       }
       if (!ok) *abort_flag = 1;
-      // wait for every MMA this thread issued before TMEM may be released
+      // every MMA this thread issued must be complete before TMEM is released
       tc_commit(&bars[BAR_DRAIN]);
       if (!mbar_wait_bounded(&bars[BAR_DRAIN], 0)) *abort_flag = 1;
     }
   } else {
-    // ======================= softmax warps (row r = tid) =======================
-    const int r = tid;
-    const int lr = l0 + r / G;                       // prompt row of this TMEM lane
-    const int pos_r = p.pos0 + lr;                   // last visible token
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float mu = -INFINITY, ell = 0.f;
+    // ======================= softmax warpgroups =======================
+    const int wg = tid >> 7;                          // column half of S and O
+    const int r = tid & 127;                          // TMEM lane = query row of the tile
+    const int lr = l0 + r / G;                        // prompt row of this lane
+    const int pos_r = p.pos0 + lr;                    // last visible token
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int j = 0; j < n_tiles && ok; ++j) {
-      const int t0 = j * PN;
-      ok = mbar_wait_bounded(&bars[BAR_S], j & 1);
-      if (!ok) break;
-      tc_fence_after();
-      float s[PN];
+
+    // ---- prologue 1: P[g] -> three bf16 parts, MN-major 128B-swizzled tiles
+    {
+      const int i = tid >> 1, half = tid & 1;         // input dim i, outputs 64*half .. 64*half+63
+      const float* src = p.P + ((size_t)g * D + i) * D + half * 64;
+      const int rowoff = half * S::TILE + i * 128;
+#pragma unroll 4
+      for (int c = 0; c < 8; ++c) {
+        const float4 x0 = __ldg(reinterpret_cast<const float4*>(src + 8 * c));
+        const float4 x1 = __ldg(reinterpret_cast<const float4*>(src + 8 * c + 4));
+        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        uint32_t w1[4], w2[4], w3[4];
 #pragma unroll
-      for (int c = 0; c < PN; c += 32) tmem_ld32(tm_S + lane_base + c, *reinterpret_cast<float(*)[32]>(&s[c]));
-      tmem_wait_ld();
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < PN; ++c) {
-        if (t0 + c > pos_r) s[c] = -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 4; ++e) {
+          float r0 = x[2 * e], r1 = x[2 * e + 1];
+          const __nv_bfloat162 a = __floats2bfloat162_rn(r0, r1);
+          r0 -= __low2float(a);
+          r1 -= __high2float(a);
+          const __nv_bfloat162 bb = __floats2bfloat162_rn(r0, r1);
+          r0 -= __low2float(bb);
+          r1 -= __high2float(bb);
+          const __nv_bfloat162 cc = __floats2bfloat162_rn(r0, r1);
+          w1[e] = *reinterpret_cast<const uint32_t*>(&a);
+          w2[e] = *reinterpret_cast<const uint32_t*>(&bb);
+          w3[e] = *reinterpret_cast<const uint32_t*>(&cc);
+        }
+        const int off = rowoff + ((c ^ (i & 7)) << 4);
+        *reinterpret_cast<uint4*>(smem + S::OFF_V1 + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        *reinterpret_cast<uint4*>(smem + S::OFF_PP + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+        *reinterpret_cast<uint4*>(smem + S::OFF_QH + off) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
       }
-      // the previous PV must be complete before O is rescaled or P is rewritten
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[BAR_PS]);
+    }
+
+    // ---- prologue 2 (warpgroup 0): top-k of |q~| for this row, masked scaled q~ high/low parts
+    if (wg == 0) {
+      ok = wait_or_abort(&bars[BAR_QT], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        const int m = p.d_store;
+        uint32_t key[D];                              // |q~| bits + 1 for j < m (0 otherwise): order-preserving
+#pragma unroll
+        for (int c = 0; c < D; c += 32) tmem_ld32(tm_O + lane_base + c, *reinterpret_cast<float(*)[32]>(&key[c]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < D; ++j) key[j] = (j < m) ? ((key[j] & 0x7fffffffu) + 1u) : 0u;
+        // largest tau with #{key >= tau} >= k, bit by bit; stop early once exactly k keys are >= tau
+        uint32_t tau = 0;
+        int cnt_tau = D;
+#pragma unroll 1
+        for (int bit = 30; bit >= 0; --bit) {
+          const uint32_t cand = tau | (1u << bit);
+          int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+          for (int j = 0; j < D; ++j) cp[j & 7] += (key[j] >= cand);
+          const int c = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
+          if (c >= p.k) {
+            tau = cand;
+            cnt_tau = c;
+          }
+          if (__all_sync(0xffffffffu, cnt_tau == p.k)) break;
+        }
+        // selected: every key above tau, then keys equal to tau from the lowest index up
+        uint32_t selm[4], eqm[4];
+        int need = p.k;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          uint32_t gt = 0u, eq = 0u;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            gt |= (uint32_t)(key[32 * w + t] > tau) << t;
+            eq |= (uint32_t)(key[32 * w + t] == tau) << t;
+          }
+          selm[w] = gt;
+          eqm[w] = eq;
+          need -= __popc(gt);
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int ne = __popc(eqm[w]);
+          if (ne <= need) {
+            selm[w] |= eqm[w];
+            need -= ne;
+          } else if (need > 0) {
+            const uint32_t last = __fns(eqm[w], 0, need);   // position of the need-th tie in this word
+            selm[w] |= eqm[w] & (last >= 31 ? 0xffffffffu : ((2u << last) - 1u));
+            need = 0;
+          }
+        }
+        const bool live = lr < l_end;
+        if (p.sel_out != nullptr && live) {
+          int32_t* so = p.sel_out + (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * p.k;
+          int n = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            for (uint32_t word = selm[w]; word != 0u; word &= word - 1u) so[n++] = 32 * w + (__ffs(word) - 1);
+        }
+        // second pass over q~ (still in TMEM): masked, scaled, split, K-major swizzled rows
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(tm_O + lane_base + c0, v);
+          tmem_wait_ld();
+          const uint32_t word = selm[c0 >> 5];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {            // 8 dims = one 16-byte chunk
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int jj = 8 * cc + 2 * e;
+              const float x0 = ((word >> jj) & 1u) ? v[jj] * p.scale_log2 : 0.f;
+              const float x1 = ((word >> (jj + 1)) & 1u) ? v[jj + 1] * p.scale_log2 : 0.f;
+              // high part truncated, low part rounded: |x - hi - lo| <= 2^-16 |x|, unbiased
+              const uint32_t h0 = __float_as_uint(x0) & 0xffff0000u, h1 = __float_as_uint(x1) & 0xffff0000u;
+              hw[e] = pack_hi_halves(h0, h1);
+              lw[e] = pack_bf16(x0 - __uint_as_float(h0), x1 - __uint_as_float(h1));
+            }
+            const int chunk = (c0 >> 3) + cc;         // 0..15
+            const int off = (chunk >> 3) * S::TILE + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(smem + S::OFF_QH + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(smem + S::OFF_QL + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+      }
+      mbar_arrive(&bars[BAR_QM]);
+    }
+
+    // ---- main loop: this warpgroup's 64 columns of every S tile.  Every softmax
+    // thread runs all n_tiles iterations and reaches the named barrier in each,
+    // also after a failed wait (then it only raises the abort flag and skips the
+    // work), so a timeout never leaves a partner blocked at the barrier.
+    float mu = -INFINITY, ell = 0.f;
+    const int cbase = wg * 64;
+    if (!ok) *abort_flag = 1;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int t0 = j * PN;
+      float s[64];
+      float mx = -INFINITY;
+      if (ok) ok = wait_or_abort(&bars[BAR_S], j & 1, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tm_S + lane_base + cbase, *reinterpret_cast<float(*)[32]>(&s[0]));
+        tmem_ld32(tm_S + lane_base + cbase + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+        tmem_wait_ld();
+        const int tc0 = t0 + cbase;                   // token of s[0]
+        if (tc0 + 63 > pos_r) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (tc0 + c > pos_r) s[c] = -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+      }
+      // row maximum over both column halves
+      red[wg * 128 + r] = mx;
+      named_bar_sync(1, kSoftThreads);
+      mx = fmaxf(mx, red[(wg ^ 1) * 128 + r]);
+      if (!ok) {
+        *abort_flag = 1;
+        continue;
+      }
+      // S may now be overwritten by the next tile's QK (the partner has read this tile's maximum)
+      tc_fence_before();
+      mbar_arrive(&bars[BAR_SF]);
+      // running maximum: raised (and O, ell rescaled below) only when exceeded by 2^kLazy
+      const bool raise = mx > mu + kLazy;
+      const float mu_new = raise ? mx : mu;
+      // P = 2^(s - mu) as bf16 high + low parts, computed while the previous P V may still run;
+      // the row sum takes the values exactly as the tensor cores will see them
+      uint32_t hw[32], lw[32];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = ex2_ftz(s[c] - mu_new);
+        const float p1 = ex2_ftz(s[c + 1] - mu_new);
+        uint32_t h0, l0, h1, l1;
+        split_trunc(p0, h0, l0);
+        split_trunc(p1, h1, l1);
+        rs0 += __uint_as_float(h0) + __uint_as_float(l0);
+        rs1 += __uint_as_float(h1) + __uint_as_float(l1);
+        hw[c >> 1] = pack_hi_halves(h0, h1);
+        lw[c >> 1] = pack_hi_halves(l0, l1);
+      }
+      // the previous P V must be complete before O is rescaled or P is rewritten
       if (j > 0) {
-        ok = mbar_wait_bounded(&bars[BAR_O], (j - 1) & 1);
-        if (!ok) break;
+        ok = wait_or_abort(&bars[BAR_O], (j - 1) & 1, abort_flag);
+        if (!ok) {
+          *abort_flag = 1;
+          continue;
+        }
         tc_fence_after();
       }
-      if (mx > mu + kLazy) {
-        const float alpha = exp2f(mu - mx);          // 0 on the first visible tile
-        if (j > 0 && mu > -INFINITY) {
+      // P into tensor memory: this lane's row, tokens 64*wg .. 64*wg+63 as 32 packed columns
+      tmem_st32(tm_P + lane_base + 32 * wg, *reinterpret_cast<const float(*)[32]>(hw));
+      tmem_st32(tm_P + 64 + lane_base + 32 * wg, *reinterpret_cast<const float(*)[32]>(lw));
+      if (raise) {
+        const float alpha = ex2_ftz(mu - mu_new);     // 0 on the first tile
+        if (j > 0) {
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < 64; c += 32) {
             float o[32];
-            tmem_ld32(tm_O + lane_base + c, o);
+            tmem_ld32(tm_O + lane_base + cbase + c, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tm_O + lane_base + c, o);
+            tmem_st32(tm_O + lane_base + cbase + c, o);
           }
           tmem_wait_st();
         }
         ell *= alpha;
-        mu = mx;
+        mu = mu_new;
       }
-      // P = exp2(s - mu), high and low bf16 parts, K-major 128B-swizzled rows
-      unsigned char* ph = smem + S::OFF_PH;
-      unsigned char* pl = smem + S::OFF_PL;
-      float rs = 0.f;
-#pragma unroll
-      for (int c8 = 0; c8 < PN / 8; ++c8) {
-        uint32_t hw[4], lw[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = (mu == -INFINITY) ? 0.f : exp2f(s[8 * c8 + 2 * e] - mu);
-          const float p1 = (mu == -INFINITY) ? 0.f : exp2f(s[8 * c8 + 2 * e + 1] - mu);
-          rs += p0 + p1;
-          float h0, lo0, h1, lo1;
-          split_bf16(p0, h0, lo0);
-          split_bf16(p1, h1, lo1);
-          hw[e] = pack_bf16(h0, h1);
-          lw[e] = pack_bf16(lo0, lo1);
-        }
-        const int half = c8 >> 3, chunk = c8 & 7;
-        const int off = half * S::TILE + r * 128 + ((chunk ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(ph + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(pl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-      }
-      ell += rs;
+      ell += rs0 + rs1;
+      tmem_wait_st();
       // tokens past the chunk's keys are not in the cache yet: their V rows must be finite
       if (t0 + PN > kv_valid) {
-        ok = mbar_wait_bounded(&bars[BAR_V], j & 1);
-        if (!ok) break;
+        ok = wait_or_abort(&bars[BAR_VF0 + (j & 1)], (j >> 1) & 1, abort_flag);
+        if (!ok) {
+          *abort_flag = 1;
+          continue;
+        }
         if (t0 + r >= kv_valid) {
+          unsigned char* vrow = smem + ((j & 1) ? S::OFF_V1 : S::OFF_V0) + wg * S::TILE + r * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(smem + S::OFF_V + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(smem + S::OFF_V + S::TILE + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-          }
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[BAR_P]);
     }
-    // epilogue: O / l
-    if (ok) ok = mbar_wait_bounded(&bars[BAR_O], (n_tiles - 1) & 1);
+    // epilogue: O / (sum over both halves)
+    if (ok) ok = wait_or_abort(&bars[BAR_O], (n_tiles - 1) & 1, abort_flag);
+    red[wg * 128 + r] = ell;
+    named_bar_sync(1, kSoftThreads);                 // reached by every softmax thread
     if (ok) {
       tc_fence_after();
+      const float inv = 1.f / (ell + red[(wg ^ 1) * 128 + r]);
       const bool live = lr < l_end;
-      const int h = g * G + (r % G);
-      const size_t obase = (((size_t)b * p.L + lr) * p.Hq + h) * D;
-      const float inv = 1.f / ell;
+      const size_t obase = (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * D + cbase;
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float o[32];
-        tmem_ld32(tm_O + lane_base + c, o);
+        tmem_ld32(tm_O + lane_base + cbase + c, o);
         tmem_wait_ld();
         if (live) {
           if (p.out_bf16) {
@@ -492,56 +675,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && tid == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 template <int G>
-int launch_prefill_g(const aqua_cache* c, const PrefillParams& p, cudaStream_t st) {
+int launch_prefill_g(const aqua_cache* c, const PrefillParams& p, const void* q, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(prefill_select_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, D * D * 4) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(prefill_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::BYTES) !=
-            cudaSuccess)
+    if (cudaFuncSetAttribute(prefill_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::BYTES) !=
+        cudaSuccess)
       return check_launch("cudaFuncSetAttribute(prefill)");
     configured = true;
   }
-  const uint64_t rows_total = (uint64_t)p.B * p.Hkv * p.L * G;
   CUtensorMap tq, tk, tv;
-  int rc = encode_tmap_bf16_2d(&tq, p.qm, D, 2 * rows_total, D * 2, 64, PM, true);
+  // q [B*L][Hq][D]: box {64 dims, G heads, 128/G positions} = the CTA's 128 rows in (position, head) order
+  const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)p.Hq, (uint64_t)p.B * p.L};
+  const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)p.Hq * D * 2};
+  const uint32_t qbox[3] = {64u, (uint32_t)G, (uint32_t)(PM / G)};
+  int rc = encode_tmap_bf16_3d(&tq, q, qdims, qstr, qbox, true);
   if (rc == AQUA_OK)
     rc = encode_tmap_bf16_2d(&tk, c->k_proj, (uint64_t)c->Tcap, (uint64_t)c->B * c->Hkv * c->d_store,
                              (uint64_t)c->Tcap * 2, 64, (uint32_t)c->d_store, true);
   if (rc == AQUA_OK)
     rc = encode_tmap_bf16_2d(&tv, c->v, D, (uint64_t)c->B * c->Hkv * c->Tcap, D * 2, 64, PN, true);
   if (rc != AQUA_OK) return rc;
-  dim3 gsel((p.L * G + kSelRows - 1) / kSelRows, p.Hkv, p.B);
-  cudaError_t e = launch_pdl(prefill_select_kernel<G>, gsel, dim3(kSelWarps * 32), D * D * 4, st, p);
-  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "prefill_select_kernel: %s", cudaGetErrorString(e));
-  if ((rc = check_launch("prefill_select_kernel")) != AQUA_OK) return rc;
-  dim3 gattn((p.L + PM / G - 1) / (PM / G), p.Hkv, p.B);
-  e = launch_pdl(prefill_attn_kernel<G>, gattn, dim3(kAttnThreads), AttnSmem::BYTES, st, tq, tk, tv, p);
+  dim3 grid((p.L + PM / G - 1) / (PM / G), p.Hkv, p.B);
+  const cudaError_t e = launch_pdl(prefill_attn_kernel<G>, grid, dim3(kAttnThreads), AttnSmem::BYTES, st, tq, tk, tv, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "prefill_attn_kernel: %s", cudaGetErrorString(e));
   return check_launch("prefill_attn_kernel");
 }
 
 }  // namespace
 
-size_t prefill_workspace_bytes(const aqua_cache* c, int Hq, int L) {
-  return 2ull * (size_t)c->B * L * Hq * D * 2 + 256;   // q~m high and low parts
+size_t prefill_workspace_bytes(const aqua_cache*, int, int) {
+  return 256;   // reserved; the kernel keeps all its intermediates on chip
 }
 
 int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const float* P, int Hq, int k, float scale,
-                   void* out, int out_dtype, int32_t* sel_out, void* ws, cudaStream_t st) {
+                   void* out, int out_dtype, int32_t* sel_out, void*, cudaStream_t st) {
   if (c->d_store % 16 != 0)
     return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: d_store %d must be a multiple of 16", c->d_store);
   PrefillParams p;
-  p.q = q;
   p.P = P;
-  p.qm = static_cast<__nv_bfloat16*>(ws);
   p.out = out;
   p.sel_out = sel_out;
   p.ctrl = c->ctrl;
@@ -556,9 +734,9 @@ int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const fl
   p.out_bf16 = out_dtype == AQUA_BF16;
   p.scale_log2 = scale * kLog2e;
   switch (Hq / c->Hkv) {
-    case 1: return launch_prefill_g<1>(c, p, st);
-    case 2: return launch_prefill_g<2>(c, p, st);
-    case 4: return launch_prefill_g<4>(c, p, st);
+    case 1: return launch_prefill_g<1>(c, p, q, st);
+    case 2: return launch_prefill_g<2>(c, p, q, st);
+    case 4: return launch_prefill_g<4>(c, p, q, st);
     default: return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: Hq/Hkv = %d not in {1,2,4}", Hq / c->Hkv);
   }
 }

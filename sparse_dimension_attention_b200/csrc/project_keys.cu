@@ -12,7 +12,9 @@ namespace aqua {
 namespace {
 
 constexpr int D = kHeadDim;
-constexpr int kTokPerCta = 16;  // two tokens per warp
+constexpr int kWarps = 8;
+constexpr int kTokPerWarp = 4;
+constexpr int kTokPerCta = kWarps * kTokPerWarp;   // 32
 
 template <typename T>
 __device__ __forceinline__ void load4(const T* p, float (&f)[4]);
@@ -38,8 +40,11 @@ __device__ __forceinline__ void copy4(__nv_bfloat16* dst, const __nv_bfloat16* s
   *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
 }
 
-// grid (ceil(L/16), Hkv, B), block 256: P[g] is staged in shared memory by one
-// bulk copy; warp w projects tokens blockIdx.x*16 + 2w and +1 of (b, g).
+// grid (ceil(L/32), Hkv, B), block 256: P[g] is staged in shared memory by one
+// bulk copy; warp w projects tokens blockIdx.x*32 + 4w .. 4w+3 of (b, g) with
+// one pass over P, the projected keys are staged as a [dim][32 token] tile and
+// written out as runs of 32 consecutive slots per dimension row (the cache is
+// dimension-major), values are copied token-major.
 template <typename T>
 __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__ k_new,
                                                            const T* __restrict__ v_new,
@@ -48,8 +53,9 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
                                                            int32_t* len, int32_t* n_abs, int32_t* pos,
                                                            float* score, int32_t* ctrl, int B, int L,
                                                            int Hkv, int d_store, int Tcap) {
-  extern __shared__ __align__(128) float Ps[];   // [D][D]
-  __shared__ __align__(16) float xs[8][D];        // one key row per warp
+  extern __shared__ __align__(128) float Ps[];              // [D][D]
+  __shared__ __align__(16) float xs[kWarps][kTokPerWarp][D];  // the warp's key rows
+  __shared__ T kt[D][kTokPerCta];                           // projected keys, dimension-major
   __shared__ __align__(8) uint64_t pbar;
   __shared__ int is_last;
   const int g = blockIdx.y, b = blockIdx.z;
@@ -58,6 +64,10 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
   // advances them only after every CTA has taken one.
   const int base = __ldcg(len + b);
   const int abase = n_abs ? __ldcg(n_abs + b) : base;
+  const int l0 = blockIdx.x * kTokPerCta;
+  const int ntok = min(kTokPerCta, L - l0);
+  const size_t unit = (size_t)b * Hkv + g;
+  const bool in_range = base >= 0 && base + l0 + ntok <= Tcap;
   if (threadIdx.x == 0) {
     mbar_init(&pbar, 1);
     fence_barrier_init();
@@ -67,38 +77,42 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     mbar_arrive_expect_tx(&pbar, D * D * 4);
     bulk_g2s_plain(Ps, P + (size_t)g * D * D, D * D * 4, &pbar);
   }
+  // key rows of this warp's tokens (zeros past the chunk), values copied meanwhile
+#pragma unroll
+  for (int t = 0; t < kTokPerWarp; ++t) {
+    const int l = warp * kTokPerWarp + t;
+    float kv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (l < ntok) {
+      const size_t row = ((size_t)b * L + l0 + l) * Hkv + g;
+      load4<T>(k_new + row * D + 4 * lane, kv);
+      if (in_range) {
+        const int slot = base + l0 + l;
+        copy4<T>(vcache + (unit * Tcap + slot) * D + 4 * lane, v_new + row * D + 4 * lane);
+        if (pos != nullptr && lane == 0) {
+          pos[unit * Tcap + slot] = abase + l0 + l;
+          score[unit * Tcap + slot] = 0.f;
+        }
+      }
+    }
+    *reinterpret_cast<float4*>(&xs[warp][t][4 * lane]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+  }
+  __syncwarp();
   const bool ok = mbar_wait_bounded(&pbar, 0);
   const bool bad = __syncthreads_or(!ok);
   if (bad && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_TIMEOUT);
-#pragma unroll 1
-  for (int j = 0; j < kTokPerCta / 8 && !bad; ++j) {
-    const int l = blockIdx.x * kTokPerCta + warp * (kTokPerCta / 8) + j;
-    if (l >= L) break;
-    if (base < 0 || base + l >= Tcap) {
-      if (lane == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
-      break;
-    }
-    const size_t row = ((size_t)b * L + l) * Hkv + g;
-    float kv[4];
-    load4<T>(k_new + row * D + 4 * lane, kv);
-    *reinterpret_cast<float4*>(&xs[warp][4 * lane]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
-    __syncwarp();
-    float acc[4];
-    project_row_smem(Ps, xs[warp], lane, acc);
-    __syncwarp();
-    const int slot = base + l;
-    const size_t unit = (size_t)b * Hkv + g;
-    T* kp = kproj + unit * d_store * (size_t)Tcap + slot;
+  if (!in_range && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity
+  if (!bad && in_range) {
+    float y[kTokPerWarp][4];
+    project_rows_smem<kTokPerWarp>(Ps, &xs[warp][0][0], lane, y);
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int jd = 4 * lane + s;
-      if (jd < d_store) kp[(size_t)jd * Tcap] = Elem<T>::from_f32(acc[s]);
-    }
-    copy4<T>(vcache + (unit * Tcap + slot) * D + 4 * lane, v_new + row * D + 4 * lane);
-    if (pos != nullptr && lane == 0) {
-      pos[unit * Tcap + slot] = abase + l;
-      score[unit * Tcap + slot] = 0.f;
-    }
+    for (int t = 0; t < kTokPerWarp; ++t)
+#pragma unroll
+      for (int s = 0; s < 4; ++s) kt[4 * lane + s][warp * kTokPerWarp + t] = Elem<T>::from_f32(y[t][s]);
+    __syncthreads();
+    // dimension row jd, tokens 0..ntok-1 -> slots base+l0 .. : one warp per row, one lane per token
+    T* kp = kproj + unit * d_store * (size_t)Tcap + base + l0;
+    for (int jd = warp; jd < d_store; jd += kWarps)
+      if (lane < ntok) kp[(size_t)jd * Tcap + lane] = kt[jd][lane];
   }
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -74,8 +74,10 @@ def test_h2o_decision_is_bit_exact():
         assert int(cache.len[0].item()) == min(n, budget)
 
 
-def test_h2o_steps_match_oracle():
-    """Truncated cache (m = 96), k = 64 within it, budget 64 = 16 recent + 48 heavy, 40 steps."""
+@pytest.mark.parametrize("fused", [False, True])
+def test_h2o_steps_match_oracle(fused):
+    """Truncated cache (m = 96), k = 64 within it, budget 64 = 16 recent + 48 heavy, 40 steps;
+    the step's key/value appended by aqua_project_keys or by the decode call itself."""
     B, Hq, Hkv, T0, m, k, budget, recent, steps = 2, 8, 2, 64, 96, 64, 64, 16, 40
     P64, P32, cache = _h2o_setup(B, Hq, Hkv, T0, m, budget)
     inp = synth.decode_inputs(B, Hq, Hkv, T0, bf16=True, steps=steps)
@@ -91,10 +93,14 @@ def test_h2o_steps_match_oracle():
     ws = torch.empty(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
     for s in range(steps):
-        aq.aqua_project_keys(cache.desc, tdev(inp["k_new"][s][:, None], torch.bfloat16),
-                             tdev(inp["v_new"][s][:, None], torch.bfloat16), Pt, 1)
-        aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], torch.bfloat16), Pt, Hq, k, out, ws, scores_out=sc,
-                            lse_out=lse)
+        kn, vn = tdev(inp["k_new"][s], torch.bfloat16), tdev(inp["v_new"][s], torch.bfloat16)
+        if fused:
+            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], torch.bfloat16), Pt, Hq, k, out, ws, scores_out=sc,
+                                lse_out=lse, k_new=kn, v_new=vn)
+        else:
+            aq.aqua_project_keys(cache.desc, kn[:, None], vn[:, None], Pt, 1)
+            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], torch.bfloat16), Pt, Hq, k, out, ws, scores_out=sc,
+                                lse_out=lse)
         aq.aqua_h2o_update(cache.desc, sc, lse, Hq, budget, recent, ev)
         torch.cuda.synchronize()
         got_out = out.float().cpu().numpy().astype(np.float64)
