@@ -196,7 +196,7 @@ class DecodeBench:
         self.v_d = self.v_h.cuda()
         self.out = torch.empty((B, Hq, 128), dtype=self.dt, device="cuda")
         self.out_h = torch.empty((B, Hq, 128), dtype=self.dt).pin_memory()
-        self.ws = torch.empty(aq.aqua_decode_workspace_size(self.cache.desc, Hq), dtype=torch.uint8, device="cuda")
+        self.ws = torch.zeros(aq.aqua_decode_workspace_size(self.cache.desc, Hq), dtype=torch.uint8, device="cuda")
         self.sel = torch.empty((B, Hq, 128), dtype=torch.int32, device="cuda")
 
     def rewind(self):
@@ -463,7 +463,7 @@ class H2OBench:
         self.lse = torch.zeros((B, Hq), dtype=torch.float32, device="cuda")
         self.out = torch.empty((B, Hq, 128), dtype=bf, device="cuda")
         self.ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
-        self.ws = torch.empty(aq.aqua_decode_workspace_size(self.cache.desc, Hq), dtype=torch.uint8, device="cuda")
+        self.ws = torch.zeros(aq.aqua_decode_workspace_size(self.cache.desc, Hq), dtype=torch.uint8, device="cuda")
         self.n_steps = 0
         torch.cuda.synchronize()
 

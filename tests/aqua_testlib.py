@@ -54,7 +54,7 @@ def run_decode(cache: aq.AquaCache, q: np.ndarray, Pt: torch.Tensor, k: int, out
     qproj = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
     lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
     sc = torch.zeros((B, Hq, cache.Tcap), dtype=torch.float32, device="cuda") if scores else None
-    ws = torch.empty(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     aq.aqua_decode_attn(cache.desc, qt, Pt, Hq, k, out, ws, sel_out=sel, qproj_out=qproj, lse_out=lse,
                         scores_out=sc)
     torch.cuda.synchronize()

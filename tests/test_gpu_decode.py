@@ -228,7 +228,7 @@ def test_fused_append_equals_separate_append(kv):
         Pt = fill_cache(c, inp["k_hist"], inp["v_hist"], P32)
     outs = []
     for mode, c in enumerate(caches):
-        ws = torch.empty(aq.aqua_decode_workspace_size(c.desc, Hq), dtype=torch.uint8, device="cuda")
+        ws = torch.zeros(aq.aqua_decode_workspace_size(c.desc, Hq), dtype=torch.uint8, device="cuda")
         res = []
         for s in range(2):
             q = tdev(inp["q"][s], dt)

@@ -49,7 +49,7 @@ def test_h2o_decision_is_bit_exact():
     sc = torch.zeros((B, Hq, cache.Tcap), dtype=torch.float32, device="cuda")
     lse = torch.zeros((B, Hq), dtype=torch.float32, device="cuda")
     out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
     inf_lse = torch.full((B, Hq), float("inf"), device="cuda")
     for s in range(6):
@@ -90,7 +90,7 @@ def test_h2o_steps_match_oracle(fused):
     sc = torch.zeros((B, Hq, cache.Tcap), dtype=torch.float32, device="cuda")
     lse = torch.zeros((B, Hq), dtype=torch.float32, device="cuda")
     out = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
     for s in range(steps):
         kn, vn = tdev(inp["k_new"][s], torch.bfloat16), tdev(inp["v_new"][s], torch.bfloat16)

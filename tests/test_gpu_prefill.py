@@ -134,14 +134,16 @@ def test_prefill_row_matches_decode():
     sel = torch.empty((1, L, Hq, k), dtype=torch.int32, device="cuda")
     ws = torch.empty(aq.aqua_prefill_workspace_size(cache.desc, Hq, L), dtype=torch.uint8, device="cuda")
     aq.aqua_prefill_attn(cache.desc, q, 0, L, Pt, Hq, k, o, ws, sel_out=sel)
-    wsd = torch.empty(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
+    wsd = torch.zeros(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     for p in (0, 63, 127, 159):
         cache.len.fill_(p + 1)
         od = torch.empty((1, Hq, 128), dtype=torch.float32, device="cuda")
         sd = torch.empty((1, Hq, k), dtype=torch.int32, device="cuda")
         aq.aqua_decode_attn(cache.desc, q[:, p].contiguous(), Pt, Hq, k, od, wsd, sel_out=sd)
         torch.cuda.synchronize()
-        # same f32 projection routine on both paths: identical selections
-        np.testing.assert_array_equal(sd.cpu().numpy()[0], sel.cpu().numpy()[0, p])
+        # both paths project in f32 (in different summation orders): the sets
+        # agree except where the k-th and (k+1)-th magnitudes are a near tie
+        qt = np.stack([O.project(inp["q"][0, p, h], P64[h // (Hq // Hkv)]) for h in range(Hq)])
+        _check_sel(sd.cpu().numpy()[0], sel.cpu().numpy()[0, p], qt, k)
         err = rel_err_rows(od.cpu().numpy()[0].astype(np.float64), o.cpu().numpy()[0, p].astype(np.float64))
         assert np.max(err) <= 1e-4, (p, np.max(err))

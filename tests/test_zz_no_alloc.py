@@ -26,7 +26,7 @@ def test_static_scratch_matches_workspace_entry_point():
     static = aq.AquaCache(B, Hkv, T + 16)
     for c in (with_ws, static):
         Pt = fill_cache(c, inp["k_hist"], inp["v_hist"], P32)
-    ws = torch.empty(aq.aqua_decode_workspace_size(with_ws.desc, Hq), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(aq.aqua_decode_workspace_size(with_ws.desc, Hq), dtype=torch.uint8, device="cuda")
     for s in range(2):                                   # two calls in a row
         q = tdev(inp["q"][s], torch.bfloat16)
         kn, vn = tdev(inp["k_new"][s], torch.bfloat16), tdev(inp["v_new"][s], torch.bfloat16)
