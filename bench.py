@@ -81,25 +81,68 @@ def peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons during the timed region: an NVML thread
+    polling every 2 ms (read-only queries), else nvidia-smi at its shortest loop."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
+        import threading
         self.proc = None
+        self.sm, self.smax, self.reasons = [], [], set()
+        self.stop_evt = threading.Event()
+        self.thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(ident)
+            self.nv = pynvml
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "10"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
+    def _poll(self):
+        nv = self.nv
+        while not self.stop_evt.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                self.smax.append(float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS:
+                    if r & getattr(nv, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self.stop_evt.wait(0.002)
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=2)
+            return {"sm_mhz": statistics.median(self.sm) if self.sm else None,
+                    "sm_max_mhz": max(self.smax) if self.smax else None,
+                    "reasons": sorted(self.reasons), "samples": len(self.sm), "source": "nvml"}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvidia-smi unavailable"}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "no clock source"}
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -121,7 +164,7 @@ class ClockSampler:
                 if val.lower().startswith("active"):
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------- distributed
@@ -489,7 +532,9 @@ class H2OBench:
         qo = B * Hq * 128 * 2 * 2
         return attn + scores + h2o + move + append + qo
 
-    def report(self, W: int) -> dict:
+    def report(self, W: int, K: int = 200) -> dict:
+        """Steady state from T_abs = budget to T_end (runs shorter than 100 main
+        steps replay the 256-step graph only K // 4 + 1 times)."""
         torch, wl = self.torch, self.wl
         G = wl["Hq"] // wl["Hkv"]
         for _ in range(W):
@@ -510,6 +555,8 @@ class H2OBench:
         torch.cuda.synchronize()
         t_abs0 = wl["budget"] + self.n_steps                               # tokens seen so far
         reps = max(1, (wl["T_end"] - t_abs0) // self.GRAPH_STEPS)
+        if K < 100:
+            reps = min(reps, K // 4 + 1)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
@@ -610,7 +657,10 @@ def main():
     ap.add_argument("--impl", default="aqua", choices=["aqua", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--k", type=int, default=None)
-    ap.add_argument("--no-extras", action="store_true", help="skip the k sweep and the long-context line")
+    ap.add_argument("--no-extras", action="store_true", help="only the main decode line")
+    ap.add_argument("--extras", default="sweep,long,prefill,h2o",
+                    help="comma list of extra lines: sweep (k sweep), long (long context), prefill (chunked "
+                         "prefill), h2o (truncated cache + H2O steady state)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -668,7 +718,8 @@ def main():
         "gpu_launches": 2 * K,
         "clocks": clk,
     }
-    if not args.no_extras:
+    extras = set() if args.no_extras else {x.strip() for x in args.extras.split(",") if x.strip()}
+    if "sweep" in extras:
         sweep = []
         for kk in (128, 96, 64, 32):
             u = bench.union_sizes(kk, min(K, 8))
@@ -682,8 +733,10 @@ def main():
         for r in sweep:
             r["speedup_vs_dense"] = dense / r["decode_us"]
         line["k_sweep"] = sweep
-        del bench
-        torch.cuda.empty_cache()
+    P = bench.P
+    del bench
+    torch.cuda.empty_cache()
+    if "long" in extras:
         lwl = WORKLOADS["long-context-decode"]
         lb = DecodeBench(lwl, min(K, 50), W)
         lu = lb.union_sizes(lwl["k"], min(K, 50, lb.n_in))
@@ -696,15 +749,16 @@ def main():
                                 "queries_per_s": world * Kl / (t_ms / 1e3), "ms_per_step": t_ms / Kl,
                                 "decode_us": 1e3 * statistics.mean(d_ms), "decode_gbs": ach,
                                 "frac": ach / hbm_peak}
-        P = lb.P
         del lb
         torch.cuda.empty_cache()
+    if "prefill" in extras:
         pb = PrefillBench(PREFILL, P)
         line["prefill"] = pb.report(min(K, 20), W, bf16_peak, peak_kind)
         del pb
         torch.cuda.empty_cache()
+    if "h2o" in extras:
         hb = H2OBench(H2O_WL, P)
-        r = hb.report(W)
+        r = hb.report(W, K)
         r["frac"] = r["hbm_gbs"] / hbm_peak
         line["truncated_h2o"] = r
         del hb

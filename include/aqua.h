@@ -226,8 +226,9 @@ AQUA_API int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0,
  * last slot is moved into its place and len[b] becomes len[b] - 1.
  *   scores [B][Hq][Tcap], lse [B][Hq]  from aqua_decode_attn
  *   evicted_out nullable [B][Hkv] int32: evicted absolute position, or -1
- * Requires pos, score and n_abs in the cache.  cache->max_len is lowered to
- * min(max_len, budget) on the host.
+ * Requires pos, score and n_abs in the cache and Hq/Hkv in {1, 2, 4}
+ * (AQUA_ERR_UNSUPPORTED otherwise, nothing launched).  cache->max_len is
+ * lowered to min(max_len, budget) on the host.
  */
 AQUA_API int aqua_h2o_update(aqua_cache* cache, const float* scores, const float* lse, int Hq, int budget,
                     int recent, int32_t* evicted_out, aqua_stream_t stream);

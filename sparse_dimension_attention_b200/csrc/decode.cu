@@ -105,46 +105,62 @@ __device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, flo
 // ============================================================================
 // query projection + magnitude top-k + group union
 // ============================================================================
+// Selection kernel geometry: NWQ warps project each of the G query heads
+// (each over its own slice of the input dimensions), one more warp appends.
+template <int G>
+struct QprojCfg {
+  static constexpr int NWQ = (G == 4) ? 2 : 4;
+  static constexpr int WARPS = G * NWQ + 1;
+};
+constexpr int kPChunks = 4;   // P[g] staged as four 32-row chunks, each with its own barrier
+
 template <typename T, int G>
-__global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(DecodeParams p) {
+  constexpr int NWQ = QprojCfg<G>::NWQ;
+  constexpr int ROWS = D / NWQ;                 // input dims per projection warp
+  constexpr int CROWS = D / kPChunks;           // rows per P chunk
+  static_assert(ROWS % 4 == 0 && (ROWS % CROWS == 0 || CROWS % ROWS == 0), "projection slices vs P chunks");
   extern __shared__ __align__(128) float Ps[];   // P[g], [D][D]
   __shared__ __align__(16) float qs[G][D];
+  __shared__ __align__(16) float part[NWQ][G][D];
   __shared__ __align__(16) float knew_s[D];
   __shared__ uint32_t masks[G][4];
-  __shared__ __align__(8) uint64_t pbar;
+  __shared__ __align__(8) uint64_t pbars[kPChunks];
   __shared__ int is_last;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, g = u % p.Hkv;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = g * G + (w < G ? w : 0);
+  const int hw = w / NWQ, sl = w % NWQ;         // head and slice of a projection warp (w < G * NWQ)
+  const int h = g * G + (hw < G ? hw : 0);
   const int m = p.d_store;
   const bool append = p.k_new != nullptr;
 
   if (threadIdx.x == 0) {
-    mbar_init(&pbar, 1);
+    for (int c = 0; c < kPChunks; ++c) mbar_init(&pbars[c], 1);
     fence_barrier_init();
   }
   pdl_launch_dependents();   // the attention kernel may take free SMs for its prologue
   pdl_wait();                // inputs and the cache may come from the previous kernel
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(&pbar, D * D * 4);
-    bulk_g2s_plain(Ps, p.P + (size_t)g * D * D, D * D * 4, &pbar);
+    for (int c = 0; c < kPChunks; ++c) {
+      mbar_arrive_expect_tx(&pbars[c], CROWS * D * 4);
+      bulk_g2s_plain(Ps + c * CROWS * D, p.P + (size_t)g * D * D + c * CROWS * D, CROWS * D * 4, &pbars[c]);
+    }
   }
-  const T* qrow = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D;
-  float qv[4];
+  if (w < G * NWQ && sl == 0) {
+    const T* qrow = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D;
 #pragma unroll
-  for (int s = 0; s < 4; ++s) qv[s] = Elem<T>::load(qrow + 4 * lane + s);
-  const bool ok = mbar_wait_bounded(&pbar, 0);
-  if (__syncthreads_or(!ok)) {
-    if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
-    return;
+    for (int s = 0; s < 4; ++s) qs[hw][4 * lane + s] = Elem<T>::load(qrow + 4 * lane + s);
   }
+  __syncthreads();
+  bool ok = true;
 
   const int len_before = __ldcg(p.len + b);   // read before the append ticket below
-  if (w == G) {
-    // ---- fused append of the new token of unit (b, g)
+  if (w == G * NWQ) {
+    // ---- fused append of the new token of unit (b, g), in the key projection order
     if (append) {
+      for (int c = 0; c < kPChunks; ++c) ok = mbar_wait_bounded(&pbars[c], 0) && ok;
       const int slot = len_before;
       if (slot < 0 || slot >= p.Tcap) {
         if (lane == 0) record_status(p.ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
@@ -171,17 +187,40 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
         }
       }
     }
-  } else {
-    // q~_j for j = 4*lane + s; q is read back from shared memory as a broadcast,
-    // two accumulator chains (even / odd input dims)
-    qs[w][4 * lane + 0] = qv[0];
-    qs[w][4 * lane + 1] = qv[1];
-    qs[w][4 * lane + 2] = qv[2];
-    qs[w][4 * lane + 3] = qv[3];
-    __syncwarp();
+  } else if (w < G * NWQ) {
+    // partial q~ of head hw over input dims [sl*ROWS, (sl+1)*ROWS), outputs
+    // 4*lane .. 4*lane+3: two chains (even / odd rows), each chunk as it lands
+    float a[4] = {0.f, 0.f, 0.f, 0.f}, c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i0 = sl * ROWS; i0 < (sl + 1) * ROWS; i0 += 4) {
+      if (i0 % CROWS == 0) ok = mbar_wait_bounded(&pbars[i0 / CROWS], 0) && ok;
+      const float4 x4 = *reinterpret_cast<const float4*>(&qs[hw][i0]);
+      const float4 p0 = reinterpret_cast<const float4*>(Ps + (i0 + 0) * D)[lane];
+      const float4 p1 = reinterpret_cast<const float4*>(Ps + (i0 + 1) * D)[lane];
+      const float4 p2 = reinterpret_cast<const float4*>(Ps + (i0 + 2) * D)[lane];
+      const float4 p3 = reinterpret_cast<const float4*>(Ps + (i0 + 3) * D)[lane];
+      a[0] = fmaf(x4.x, p0.x, a[0]); a[1] = fmaf(x4.x, p0.y, a[1]); a[2] = fmaf(x4.x, p0.z, a[2]); a[3] = fmaf(x4.x, p0.w, a[3]);
+      c4[0] = fmaf(x4.y, p1.x, c4[0]); c4[1] = fmaf(x4.y, p1.y, c4[1]); c4[2] = fmaf(x4.y, p1.z, c4[2]); c4[3] = fmaf(x4.y, p1.w, c4[3]);
+      a[0] = fmaf(x4.z, p2.x, a[0]); a[1] = fmaf(x4.z, p2.y, a[1]); a[2] = fmaf(x4.z, p2.z, a[2]); a[3] = fmaf(x4.z, p2.w, a[3]);
+      c4[0] = fmaf(x4.w, p3.x, c4[0]); c4[1] = fmaf(x4.w, p3.y, c4[1]); c4[2] = fmaf(x4.w, p3.z, c4[2]); c4[3] = fmaf(x4.w, p3.w, c4[3]);
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) part[sl][hw][4 * lane + s2] = a[s2] + c4[s2];
+  }
+  if (__syncthreads_or(!ok)) {
+    if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+    return;
+  }
+  if (w < G * NWQ && sl == 0) {
+    // q~_j for j = 4*lane + s: the slices' partials added in slice order
     float qt[4];
-    project_row_smem(Ps, qs[w], lane, qt);
-    __syncwarp();
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) {
+      float y = part[0][hw][4 * lane + s2];
+#pragma unroll
+      for (int x = 1; x < NWQ; ++x) y += part[x][hw][4 * lane + s2];
+      qt[s2] = y;
+    }
 
     // Keys: magnitude bits + 1 for candidate dims (j < m), 0 otherwise, so that
     // unsigned order equals |q~| order and non-candidates rank below everything.
@@ -192,16 +231,21 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
       key[s2] = (j < m) ? (__float_as_uint(fabsf(qt[s2])) + 1u) : 0u;
     }
     // Radix select of the k-th largest key: the largest tau with
-    // #{key >= tau} >= k, one bit per round; counts by ballot + popc.
+    // #{key >= tau} >= k, one bit per round, counts by ballot + popc; done as
+    // soon as exactly k keys are >= tau (the set is then already decided).
     uint32_t tau = 0;
-#pragma unroll 4
-    for (int bit = 31; bit >= 0; --bit) {
+    int cnt = D;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0 && cnt != p.k; --bit) {
       const uint32_t cand = tau | (1u << bit);
       const int c = __popc(__ballot_sync(0xffffffffu, key[0] >= cand)) +
                     __popc(__ballot_sync(0xffffffffu, key[1] >= cand)) +
                     __popc(__ballot_sync(0xffffffffu, key[2] >= cand)) +
                     __popc(__ballot_sync(0xffffffffu, key[3] >= cand));
-      if (c >= p.k) tau = cand;
+      if (c >= p.k) {
+        tau = cand;
+        cnt = c;
+      }
     }
     int ngt = 0, neq = 0;
   #pragma unroll
@@ -244,7 +288,7 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
         ++opos;
       }
       if (p.qproj_out) p.qproj_out[bh * D + j] = qt[s];
-      qs[w][j] = sel[s] ? qt[s] * p.scale_log2 : 0.f;
+      qs[hw][j] = sel[s] ? qt[s] * p.scale_log2 : 0.f;
     }
     const uint32_t nib = (uint32_t)sel[0] | ((uint32_t)sel[1] << 1) | ((uint32_t)sel[2] << 2) |
                          ((uint32_t)sel[3] << 3);
@@ -252,12 +296,12 @@ __global__ void __launch_bounds__((G + 1) * 32) qproj_topk_kernel(DecodeParams p
   #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
       const uint32_t word = __reduce_or_sync(0xffffffffu, (lane >> 3) == wd ? shifted : 0u);
-      if (lane == 0) masks[w][wd] = word;
+      if (lane == 0) masks[hw][wd] = word;
     }
   }
 
   // sequences with no tokens: zero output, lse = -inf
-  if (w < G && !append && seq_len(p.len, b, p.Tcap) <= 0) {
+  if (w < G * NWQ && sl == 0 && !append && seq_len(p.len, b, p.Tcap) <= 0) {
     const size_t bh = (size_t)b * p.Hq + h;
     for (int j = lane; j < D; j += 32) store_val(p, bh * D + j, 0.f);
     if (p.lse_out && lane == 0) p.lse_out[bh] = -INFINITY;
@@ -1245,7 +1289,8 @@ int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
       return check_launch("cudaFuncSetAttribute(qproj_topk_kernel)");
     configured = true;
   }
-  const cudaError_t e = launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3((G + 1) * 32), D * D * 4, st, p);
+  const cudaError_t e =
+      launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), D * D * 4, st, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
   return check_launch("qproj_topk_kernel");
 }

@@ -30,7 +30,9 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
   return a.score < b.score || (a.score == b.score && a.pos < b.pos);
 }
 
-template <typename T>
+constexpr int kTokPerThread = 8;   // tokens whose loads one thread issues together
+
+template <typename T, int G>
 __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kproj, T* __restrict__ vcache,
                                                               int32_t* len, const int32_t* __restrict__ n_abs,
                                                               int32_t* __restrict__ pos, float* __restrict__ score,
@@ -42,24 +44,46 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   __shared__ int s_victim, s_vpos, is_last;
   const int u = blockIdx.x;
   const int b = u / Hkv, g = u % Hkv;
-  const int G = Hq / Hkv;
   const int n = min(max(__ldcg(len + b), 0), Tcap);   // read before the ticket below
   const int newest = __ldcg(n_abs + b) - 1;
   const size_t ub = (size_t)u * Tcap;
+  const size_t bh0 = (size_t)b * Hq + (size_t)g * G;   // first query head of the group
+  float lse_h[G];
+#pragma unroll
+  for (int x = 0; x < G; ++x) lse_h[x] = lse[bh0 + x];
 
+  // Per slot t: score[t] += sum over the group's heads (in head order) of
+  // exp(scores - lse); candidates are the slots outside the recent window.
+  // A thread issues the loads of kTokPerThread slots before using any of
+  // them: the kernel is bound by memory latency, not bandwidth.
   Cand best{INFINITY, 0, -1};
-  for (int t = threadIdx.x; t < n; t += kThreads) {
-    float acc = 0.f;
-    for (int h = g * G; h < (g + 1) * G; ++h) {
-      const size_t bh = (size_t)b * Hq + h;
-      acc += expf(scores[bh * Tcap + t] - lse[bh]);
+  for (int tb = threadIdx.x; tb < n; tb += kThreads * kTokPerThread) {
+    float sv[kTokPerThread][G], scv[kTokPerThread];
+    int psv[kTokPerThread];
+#pragma unroll
+    for (int r = 0; r < kTokPerThread; ++r) {
+      const int t = tb + r * kThreads;
+      if (t < n) {
+#pragma unroll
+        for (int x = 0; x < G; ++x) sv[r][x] = scores[(bh0 + x) * Tcap + t];
+        scv[r] = score[ub + t];
+        psv[r] = pos[ub + t];
+      }
     }
-    const float sc = score[ub + t] + acc;
-    score[ub + t] = sc;
-    const int ps = pos[ub + t];
-    if (ps <= newest - recent) {
-      const Cand cnd{sc, ps, t};
-      if (better(cnd, best)) best = cnd;
+#pragma unroll
+    for (int r = 0; r < kTokPerThread; ++r) {
+      const int t = tb + r * kThreads;
+      if (t < n) {
+        float acc = 0.f;
+#pragma unroll
+        for (int x = 0; x < G; ++x) acc += expf(sv[r][x] - lse_h[x]);
+        const float sc = scv[r] + acc;
+        score[ub + t] = sc;
+        if (psv[r] <= newest - recent) {
+          const Cand cnd{sc, psv[r], t};
+          if (better(cnd, best)) best = cnd;
+        }
+      }
     }
   }
   // block arg-min
@@ -117,19 +141,30 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   }
 }
 
+template <int G>
+void launch_h2o_g(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
+                  int32_t* evicted_out, int n_units, cudaStream_t st) {
+  if (c->dtype == AQUA_BF16) {
+    h2o_update_kernel<__nv_bfloat16, G><<<n_units, kThreads, 0, st>>>(
+        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos,
+        c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+  } else {
+    h2o_update_kernel<float, G><<<n_units, kThreads, 0, st>>>(
+        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl,
+        scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+  }
+}
+
 }  // namespace
 
 int launch_h2o_update(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
                       int32_t* evicted_out, cudaStream_t st) {
   const int n_units = c->B * c->Hkv;
-  if (c->dtype == AQUA_BF16) {
-    h2o_update_kernel<__nv_bfloat16><<<n_units, kThreads, 0, st>>>(
-        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos,
-        c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
-  } else {
-    h2o_update_kernel<float><<<n_units, kThreads, 0, st>>>(
-        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl,
-        scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+  switch (Hq / c->Hkv) {
+    case 1: launch_h2o_g<1>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    case 2: launch_h2o_g<2>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    case 4: launch_h2o_g<4>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    default: return set_error(AQUA_ERR_UNSUPPORTED, "aqua_h2o_update: Hq/Hkv = %d not in {1,2,4}", Hq / c->Hkv);
   }
   return check_launch("h2o_update_kernel");
 }

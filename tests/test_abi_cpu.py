@@ -119,6 +119,9 @@ def test_h2o_argument_checks(lib):
     c = _desc(pos=0x9000, score=0x9100)
     assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 8, 16, 17, None, None) == abi.AQUA_ERR_ARG
     assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 8, 0, 0, None, None) == abi.AQUA_ERR_ARG
+    # group sizes the decode step does not produce: rejected before any launch
+    assert lib.aqua_h2o_update(ctypes.byref(c), 0x5000, 0x6000, 3 * c.Hkv, 16, 4, None, None) == \
+        abi.AQUA_ERR_UNSUPPORTED
 
 
 def test_prefill_argument_checks(lib):
