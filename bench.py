@@ -189,13 +189,23 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Maximum of x over the ranks (the timing of a multi-GPU run is the slowest
+    rank's).  The reduction tensor lives where the process group's backend
+    works: on the GPU for nccl, on the host for gloo."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Units per second of the whole job: every rank processes its own replica of
+    the workload (weak scaling), timed by the slowest rank."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 # ----------------------------------------------------------------------------- AQUA arm
@@ -681,7 +691,7 @@ def main():
     total_ms, step_ms, clk = bench.timed(K, W, wl["k"], world, clocks=(rank == 0))
     total_ms = max_over_ranks(total_ms, world)
     ms_step = total_ms / K
-    value = world * wl["B"] * K / (total_ms / 1e3)
+    value = whole_job_rate(wl["B"], K, world, total_ms)
     T_steps = [wl["T"] + s for s in range(K)]
     dec_bytes = [bench.bytes_decode(usz[s % usz.shape[0]], T_steps[s]) for s in range(K)]
     achieved = (sum(dec_bytes) + K * bench.bytes_append()) / (sum(step_ms) / 1e3) / 1e9
@@ -713,7 +723,7 @@ def main():
         "launch": "K steps captured in one CUDA graph (kernels chained with programmatic dependent launch)",
         "eager_step_us": 1e3 * eager_ms / min(K, 100),
         "unfused_step_us": 1e3 * unfused_ms,
-        "e2e": {"value": world * wl["B"] * K / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(wl["B"], K, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
         "clocks": clk,
