@@ -233,6 +233,17 @@ AQUA_API int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0,
 AQUA_API int aqua_h2o_update(aqua_cache* cache, const float* scores, const float* lse, int Hq, int budget,
                     int recent, int32_t* evicted_out, aqua_stream_t stream);
 
+/*
+ * Diagnostic: launches one CTA that waits, with the bounded wait every kernel
+ * of the library uses, on a barrier that is never completed, for limit_ns
+ * nanoseconds (1 us .. 2 s); the wait runs out, the kernel records
+ * AQUA_ERR_TIMEOUT in the cache's status word (read it with aqua_status) and
+ * returns.  It lets a caller check the time-out path on its GPU: nothing
+ * faults or hangs and the context stays usable.  The paper has no counterpart.
+ * Errors: AQUA_ERR_ARG for a missing ctrl block or a limit outside the range.
+ */
+AQUA_API int aqua_selftest_wait_timeout(aqua_cache* cache, unsigned long long limit_ns, aqua_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

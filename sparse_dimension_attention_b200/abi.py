@@ -31,6 +31,7 @@ EXPORTED = (
     "aqua_decode_workspace_size", "aqua_decode_attn", "aqua_decode_attn_static",
     "aqua_prefill_workspace_size", "aqua_prefill_attn",
     "aqua_h2o_update",
+    "aqua_selftest_wait_timeout",
 )
 
 
@@ -75,6 +76,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "aqua_decode_workspace_size": (c_size_t, [C, c_int]),
         "aqua_decode_attn": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
         "aqua_decode_attn_static": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P]),
+        "aqua_selftest_wait_timeout": (c_int, [C, ctypes.c_ulonglong, P]),
         "aqua_prefill_workspace_size": (c_size_t, [C, c_int, c_int]),
         "aqua_prefill_attn": (c_int, [C, P, c_int, c_int, P, c_int, c_int, c_float, P, c_int, P, P, c_size_t, P]),
         "aqua_h2o_update": (c_int, [C, P, P, c_int, c_int, c_int, P, P]),
@@ -115,6 +117,12 @@ def aqua_version() -> int:
 
 def aqua_last_error() -> str:
     return load_library().aqua_last_error().decode()
+
+
+def aqua_selftest_wait_timeout(cache: aqua_cache, limit_ns: int, stream=None) -> None:
+    """One CTA waits on a barrier nothing completes for limit_ns; the device
+    records AQUA_ERR_TIMEOUT in the cache's status word (see aqua_status)."""
+    _check(load_library().aqua_selftest_wait_timeout(ctypes.byref(cache), limit_ns, _stream(stream)))
 
 
 def aqua_status(cache: aqua_cache, stream=None) -> int:

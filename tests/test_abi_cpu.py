@@ -124,6 +124,14 @@ def test_h2o_argument_checks(lib):
         abi.AQUA_ERR_UNSUPPORTED
 
 
+def test_selftest_argument_checks(lib):
+    c = _desc()
+    assert lib.aqua_selftest_wait_timeout(ctypes.byref(c), 10, None) == abi.AQUA_ERR_ARG        # under 1 us
+    assert lib.aqua_selftest_wait_timeout(ctypes.byref(c), 3 * 10 ** 9, None) == abi.AQUA_ERR_ARG  # over 2 s
+    nc = _desc(ctrl=None)
+    assert lib.aqua_selftest_wait_timeout(ctypes.byref(nc), 10 ** 6, None) == abi.AQUA_ERR_ARG
+
+
 def test_prefill_argument_checks(lib):
     c = _desc()
     ws = lib.aqua_prefill_workspace_size(ctypes.byref(c), 8, 32)
