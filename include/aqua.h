@@ -148,11 +148,12 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  * the len[b] cached tokens.
  *   q          [B][Hq][d]  cache dtype; query head h uses KV head h / (Hq/Hkv)
  *   k_new, v_new  nullable [B][Hkv][d] cache dtype: the step's new key and
- *              value.  When given they are appended first, exactly as
+ *              value.  When given they are appended, exactly as
  *              aqua_project_keys(cache, k_new, v_new, P, 1) would (slot len[b],
- *              len[b] += 1, cache->max_len += 1), inside the same launch that
- *              projects the queries, so the step sees its own token.  When NULL
- *              the caller appended the step's key beforehand.
+ *              len[b] += 1, cache->max_len += 1), and the step attends them
+ *              (len[b] + 1 tokens).  On the device len[b] and n_abs[b] advance
+ *              when the step's last kernel finishes.  When NULL the caller
+ *              appended the step's key beforehand.
  *   P          [Hkv][d][d] f32
  *   k          dimensions kept per query head, 1 <= k <= d_store
  *   scale      score scale; <= 0 selects 1/sqrt(d) (d = full head dim)

@@ -20,7 +20,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // control-word indices inside aqua_cache::ctrl
-enum CtrlWord { kCtrlStatus = 0, kCtrlAppendTicket = 1, kCtrlH2OTicket = 2 };
+enum CtrlWord { kCtrlStatus = 0, kCtrlAppendTicket = 1, kCtrlH2OTicket = 2, kCtrlStepTicket = 3 };
 
 // ---------------------------------------------------------------- host side errors
 int set_error(int code, const char* fmt, ...);

@@ -72,17 +72,39 @@ struct DecodeParams {
   // optional fused append of the step's new token (k_new == nullptr: none)
   const void* k_new;      // [B][Hkv][D] cache dtype
   const void* v_new;      // [B][Hkv][D]
-  int32_t* len_w;         // == len, written by the append ticket
+  int32_t* len_w;         // == len, advanced by the attention kernel's last CTA
   int32_t* n_abs;
   int32_t* pos;
   float* score;
   int B, Hq, Hkv, d_store, Tcap, k;
+  int len_add;            // 1 with a fused append: the step attends len[b] + 1 tokens
   int out_bf16;
   float scale_log2;
 };
 
 // cached tokens of sequence b, clamped to the cache capacity (lengths are caller-owned device data)
 __device__ __forceinline__ int seq_len(const int32_t* len, int b, int Tcap) { return min(max(len[b], 0), Tcap); }
+// tokens the attention kernels attend for sequence b: the cached ones plus the
+// token appended in this step.  len[b] itself is advanced only at the end of
+// the attention kernel (step_done), so it is stable while both kernels run.
+__device__ __forceinline__ int kv_len(const DecodeParams& p, int b) {
+  return min(max(p.len[b], 0) + p.len_add, p.Tcap);
+}
+
+// Called once per attention CTA (thread 0) after all of its work: the last CTA
+// of the grid advances the lengths of a step with a fused append.
+__device__ __forceinline__ void step_done(const DecodeParams& p) {
+  if (p.len_add == 0) return;
+  __threadfence();
+  if (atomicAdd(p.ctrl + kCtrlStepTicket, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
+    __threadfence();
+    for (int bb = 0; bb < p.B; ++bb) {
+      p.len_w[bb] += p.len_add;
+      if (p.n_abs) p.n_abs[bb] += p.len_add;
+    }
+    p.ctrl[kCtrlStepTicket] = 0;
+  }
+}
 
 __device__ __forceinline__ float warp_max(float x) {
 #pragma unroll
@@ -126,7 +148,6 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
   __shared__ __align__(16) float knew_s[D];
   __shared__ uint32_t masks[G][4];
   __shared__ __align__(8) uint64_t pbars[kPChunks];
-  __shared__ int is_last;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, g = u % p.Hkv;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -139,8 +160,11 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
     for (int c = 0; c < kPChunks; ++c) mbar_init(&pbars[c], 1);
     fence_barrier_init();
   }
-  pdl_launch_dependents();   // the attention kernel may take free SMs for its prologue
   pdl_wait();                // inputs and the cache may come from the previous kernel
+  // Released only after the previous kernel is complete: the attention kernel
+  // then reads lengths and history K~/V before its own wait, which this kernel
+  // does not change (it writes only slot len[b] and leaves len[b] alone).
+  pdl_launch_dependents();
   __syncthreads();
   if (threadIdx.x == 0) {
     for (int c = 0; c < kPChunks; ++c) {
@@ -156,7 +180,7 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
   __syncthreads();
   bool ok = true;
 
-  const int len_before = __ldcg(p.len + b);   // read before the append ticket below
+  const int len_before = __ldcg(p.len + b);   // the append slot
   if (w == G * NWQ) {
     // ---- fused append of the new token of unit (b, g), in the key projection order
     if (append) {
@@ -333,22 +357,6 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
     p.ucount[u] = __popc(um[0]) + __popc(um[1]) + __popc(um[2]) + __popc(um[3]);
     p.counters[u] = 0;
   }
-  if (!append) return;
-  // every CTA has read len[b]; the last one advances the lengths
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    is_last = (atomicAdd(p.ctrl + kCtrlAppendTicket, 1) == (int)gridDim.x - 1);
-  }
-  __syncthreads();
-  if (is_last) {
-    __threadfence();
-    for (int bb = threadIdx.x; bb < p.B; bb += blockDim.x) {
-      p.len_w[bb] += 1;
-      if (p.n_abs) p.n_abs[bb] += 1;
-    }
-    if (threadIdx.x == 0) p.ctrl[kCtrlAppendTicket] = 0;
-  }
 }
 
 // ============================================================================
@@ -420,7 +428,7 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   const int chunk = (n_units + NT - 1) / NT;
   const int u_lo = min(n_units, tid * chunk), u_hi = min(n_units, u_lo + chunk);
   long long my_tiles = 0;
-  for (int u = u_lo; u < u_hi; ++u) my_tiles += (seq_len(p.len, u / p.Hkv, p.Tcap) + TT - 1) / TT;
+  for (int u = u_lo; u < u_hi; ++u) my_tiles += (kv_len(p, u / p.Hkv) + TT - 1) / TT;
   long long N;
   const long long t_excl = block_excl_scan<NT>(my_tiles, scratch, &N);
   // Effective grid: never more CTAs than tiles, so every CTA owns at least one
@@ -433,7 +441,7 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   {
     long long ts = t_excl;
     for (int u = u_lo; u < u_hi; ++u) {
-      const long long nt = (seq_len(p.len, u / p.Hkv, p.Tcap) + TT - 1) / TT;
+      const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
       if (nt > 0) my_segs += cta_of_tile(ts + nt - 1, N, C) - cta_of_tile(ts, N, C) + 1;
       ts += nt;
     }
@@ -443,7 +451,7 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   {
     long long ts = t_excl, sb = s_excl;
     for (int u = u_lo; u < u_hi; ++u) {
-      const long long nt = (seq_len(p.len, u / p.Hkv, p.Tcap) + TT - 1) / TT;
+      const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
       if (nt > 0 && ts <= my_start && my_start < ts + nt) {
         sch[0] = u;
         sch[1] = ts;
@@ -474,7 +482,7 @@ struct UnitWalker {
     ts = S.ts0;
     sb = S.sb0;
     b = u / p.Hkv;
-    Tb = seq_len(p.len, b, p.Tcap);
+    Tb = kv_len(p, b);
     te = ts + (Tb + TT - 1) / TT;
     cf = cta_of_tile(ts, S.N, S.C);
     nseg = cta_of_tile(te - 1, S.N, S.C) - cf + 1;
@@ -488,7 +496,7 @@ struct UnitWalker {
       sb += nseg;
       ++u;
       b = u / p.Hkv;
-      Tb = seq_len(p.len, b, p.Tcap);
+      Tb = kv_len(p, b);
       ts = te;
       te = ts + (Tb + TT - 1) / TT;
       if (te > ts) {
@@ -656,13 +664,23 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     fence_barrier_init();
   }
   if (tid == NCT) prefetch_tmap(&tmap_v);
-  pdl_launch_dependents();
-  pdl_wait();   // the projection kernel (and any append) must be complete
+  // The schedule depends only on the lengths, which the projection kernel does
+  // not change (the lengths advance at the end of this kernel, and the
+  // projection kernel releases this one only once its own predecessors are
+  // complete): compute it while the projection kernel runs.  Loading tiles
+  // early as well was measured to slow the step down (the copies compete with
+  // the projection kernel's latency-bound loads).
   Sched Sd;
-  if (!make_schedule<TT, NTHREADS_BF16>(p, sch + 4, sch, Sd)) return;
+  const bool has_work = make_schedule<TT, NTHREADS_BF16>(p, sch + 4, sch, Sd);
   fence_proxy_async_smem();
   __syncthreads();
-  const int n_tiles = (int)(Sd.my_end - Sd.my_start);
+  const int n_tiles = has_work ? (int)(Sd.my_end - Sd.my_start) : 0;
+  pdl_launch_dependents();
+  pdl_wait();   // the projection kernel (and its append) must be complete
+  if (!has_work) {
+    if (tid == 0) step_done(p);
+    return;
+  }
 
   if (warp >= NCW) {
     // ======================= producer warps =======================
@@ -970,6 +988,8 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     finish_segment<G>(p, hh, tid, Mh, Lh, red, s_last);
     named_bar_sync(1, NCT);
   }
+  named_bar_sync(1, NCT);               // every consumer warp is done with this CTA's work
+  if (tid == 0) step_done(p);
 }
 
 // ============================================================================
@@ -1025,7 +1045,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
   pdl_launch_dependents();
   pdl_wait();
   Sched Sd;
-  if (!make_schedule<TT, NTHREADS>(p, sch + 4, sch, Sd)) return;
+  if (!make_schedule<TT, NTHREADS>(p, sch + 4, sch, Sd)) {
+    if (tid == 0) step_done(p);
+    return;
+  }
   const int n_tiles = (int)(Sd.my_end - Sd.my_start);
 
   if (warp == NCW) {
@@ -1275,6 +1298,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
     finish_segment<G>(p, hh, tid, m_run, l_run, red, s_last);
     named_bar_sync(1, NCT);
   }
+  named_bar_sync(1, NCT);               // every consumer warp is done with this CTA's work
+  if (tid == 0) step_done(p);
 }
 
 // ============================================================================
@@ -1389,6 +1414,7 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.k_new = k_new;
   p.v_new = v_new;
   p.len_w = c->len;
+  p.len_add = (k_new != nullptr) ? 1 : 0;
   p.n_abs = c->n_abs;
   p.pos = c->pos;
   p.score = c->score;
