@@ -374,9 +374,19 @@ struct StageHdr {
 };
 constexpr int kFirst = 1, kLast = 2;
 
-// CTA that owns flat tile t when N tiles are split over C CTAs as [floor(c N / C), floor((c+1) N / C))
-__device__ __forceinline__ int cta_of_tile(long long t, long long N, int C) {
-  long long c = ((t + 1) * C + N - 1) / N - 1;
+// The tiles of all (sequence, KV head) units form one flat sequence of
+// positions in which every non-empty unit first occupies kBoundaryTiles
+// positions without work, then one position per tile.  CTA c takes positions
+// [floor(c NV / C), floor((c+1) NV / C)): a CTA whose range crosses into a
+// new unit pays a second segment merge and a switch of the selection data
+// (measured at about four tiles' time at the Llama decode shape) and receives
+// that many fewer tiles.  Its tiles are the real positions of its range,
+// which are consecutive in the plain tile order.
+constexpr int kBoundaryTiles = 4;
+
+// CTA whose range holds position p (positions split as above over C CTAs)
+__device__ __forceinline__ int cta_of_pos(long long p, long long NV, int C) {
+  long long c = ((p + 1) * C + NV - 1) / NV - 1;
   return (int)(c < C - 1 ? c : C - 1);
 }
 
@@ -412,14 +422,15 @@ __device__ __forceinline__ long long block_excl_scan(long long v, long long* sh,
 }
 
 struct Sched {
-  long long N, my_start, my_end;
+  long long N, NV;             // tiles, positions
+  long long my_start, my_end;  // this CTA's tiles (plain tile order)
   int C;
-  int u0;
-  long long ts0, sb0;
+  int u0;                      // unit of tile my_start
+  long long ts0, sb0, vs0;     // its first tile, first partial slot and first position
 };
 
-// Flat tile range of this CTA and its first unit.  Returns false (for the
-// whole CTA) when the CTA has no tile.  `scratch` needs 32 long longs.
+// This CTA's tiles and first unit.  Returns false (for the whole CTA) when the
+// CTA has no tile.  `scratch` needs 32 long longs; sch[0..7] receive results.
 template <int TT, int NT>
 __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long long* sch, Sched& S) {
   const int tid = threadIdx.x;
@@ -427,65 +438,79 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   const int c = blockIdx.x;
   const int chunk = (n_units + NT - 1) / NT;
   const int u_lo = min(n_units, tid * chunk), u_hi = min(n_units, u_lo + chunk);
-  long long my_tiles = 0;
-  for (int u = u_lo; u < u_hi; ++u) my_tiles += (kv_len(p, u / p.Hkv) + TT - 1) / TT;
-  long long N;
+  long long my_tiles = 0, my_pos = 0;
+  for (int u = u_lo; u < u_hi; ++u) {
+    const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
+    my_tiles += nt;
+    my_pos += nt > 0 ? nt + kBoundaryTiles : 0;
+  }
+  long long N, NV;
   const long long t_excl = block_excl_scan<NT>(my_tiles, scratch, &N);
-  // Effective grid: never more CTAs than tiles, so every CTA owns at least one
-  // tile and the CTAs covering a unit are consecutive (the ticket count relies
-  // on it).  The host sizes the grid from an upper bound of the lengths.
-  const int C = (int)min((long long)gridDim.x, N);
+  const long long v_excl = block_excl_scan<NT>(my_pos, scratch, &NV);
+  const int C = (int)min((long long)gridDim.x, NV);
   if (c >= C) return false;
-  const long long my_start = (long long)c * N / C, my_end = (long long)(c + 1) * N / C;
+  const long long a = (long long)c * NV / C, e = (long long)(c + 1) * NV / C;   // this CTA's positions
   long long my_segs = 0;
   {
-    long long ts = t_excl;
+    long long vs = v_excl;
     for (int u = u_lo; u < u_hi; ++u) {
       const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
-      if (nt > 0) my_segs += cta_of_tile(ts + nt - 1, N, C) - cta_of_tile(ts, N, C) + 1;
-      ts += nt;
+      if (nt == 0) continue;
+      const long long first = vs + kBoundaryTiles;
+      my_segs += cta_of_pos(first + nt - 1, NV, C) - cta_of_pos(first, NV, C) + 1;
+      vs = first + nt;
     }
   }
   long long NS;
   const long long s_excl = block_excl_scan<NT>(my_segs, scratch, &NS);
+  if (tid == 0 && e == NV) sch[1] = N;    // the last CTA's tiles run to the end
   {
-    long long ts = t_excl, sb = s_excl;
+    long long ts = t_excl, vs = v_excl, sb = s_excl;
     for (int u = u_lo; u < u_hi; ++u) {
       const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
-      if (nt > 0 && ts <= my_start && my_start < ts + nt) {
-        sch[0] = u;
-        sch[1] = ts;
-        sch[2] = sb;
+      if (nt == 0) continue;
+      const long long first = vs + kBoundaryTiles, end = first + nt;   // unit's positions: [vs, end)
+      if (vs <= a && a < end) {          // the range starts in this unit: its first tile at or after a
+        sch[0] = ts + (a > first ? a - first : 0);
+        sch[2] = u;
+        sch[3] = ts;
+        sch[4] = sb;
+        sch[5] = vs;
       }
-      if (nt > 0) sb += cta_of_tile(ts + nt - 1, N, C) - cta_of_tile(ts, N, C) + 1;
+      if (vs <= e && e < end) sch[1] = ts + (e > first ? e - first : 0);
+      sb += cta_of_pos(end - 1, NV, C) - cta_of_pos(first, NV, C) + 1;
       ts += nt;
+      vs = end;
     }
   }
   __syncthreads();
   S.N = N;
+  S.NV = NV;
   S.C = C;
-  S.my_start = my_start;
-  S.my_end = my_end;
-  S.u0 = (int)sch[0];
-  S.ts0 = sch[1];
-  S.sb0 = sch[2];
-  return true;
+  S.my_start = sch[0];
+  S.my_end = sch[1];
+  S.u0 = (int)sch[2];
+  S.ts0 = sch[3];
+  S.sb0 = sch[4];
+  S.vs0 = sch[5];
+  return S.my_end > S.my_start;
 }
 
 // Walks the units of this CTA's tile range; one instance per producer warp.
 struct UnitWalker {
   int u, b, Tb, nU, nseg, cf;
-  long long ts, te, sb;
+  long long ts, te, sb, vs;    // unit u: tiles [ts, te), first partial slot, first position
   template <int TT>
   __device__ void start(const DecodeParams& p, const Sched& S) {
     u = S.u0;
     ts = S.ts0;
     sb = S.sb0;
+    vs = S.vs0;
     b = u / p.Hkv;
     Tb = kv_len(p, b);
     te = ts + (Tb + TT - 1) / TT;
-    cf = cta_of_tile(ts, S.N, S.C);
-    nseg = cta_of_tile(te - 1, S.N, S.C) - cf + 1;
+    cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
+    nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
     nU = p.ucount[u];
   }
   // advance to the unit holding flat tile t; true when the unit changed
@@ -494,14 +519,15 @@ struct UnitWalker {
     bool changed = false;
     while (t >= te) {
       sb += nseg;
+      if (te > ts) vs += kBoundaryTiles + (te - ts);
       ++u;
       b = u / p.Hkv;
       Tb = kv_len(p, b);
       ts = te;
       te = ts + (Tb + TT - 1) / TT;
       if (te > ts) {
-        cf = cta_of_tile(ts, S.N, S.C);
-        nseg = cta_of_tile(te - 1, S.N, S.C) - cf + 1;
+        cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
+        nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
         nU = p.ucount[u];
       } else {
         nseg = 0;
@@ -629,7 +655,7 @@ struct SmemBF16 {
   static constexpr int OFF_HDR = OFF_ML + (NCW * G * 3 + 2 * G) * 4;
   static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
   static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int OFF_MISC = OFF_SCH + 36 * 8;
+  static constexpr int OFF_MISC = OFF_SCH + 40 * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 };
@@ -671,7 +697,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   // early as well was measured to slow the step down (the copies compete with
   // the projection kernel's latency-bound loads).
   Sched Sd;
-  const bool has_work = make_schedule<TT, NTHREADS_BF16>(p, sch + 4, sch, Sd);
+  const bool has_work = make_schedule<TT, NTHREADS_BF16>(p, sch + 8, sch, Sd);
   fence_proxy_async_smem();
   __syncthreads();
   const int n_tiles = has_work ? (int)(Sd.my_end - Sd.my_start) : 0;
@@ -1009,7 +1035,7 @@ struct SmemF32 {
   static constexpr int OFF_HDR = OFF_WST + 2 * SLOTS * NCW * 4;
   static constexpr int OFF_BAR = OFF_HDR + NSTAGE * (int)sizeof(StageHdr);
   static constexpr int OFF_SCH = OFF_BAR + 2 * NSTAGE * 8;
-  static constexpr int OFF_MISC = OFF_SCH + 36 * 8;
+  static constexpr int OFF_MISC = OFF_SCH + 40 * 8;
   static constexpr int BYTES = OFF_MISC + 16;
 };
 
@@ -1045,7 +1071,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
   pdl_launch_dependents();
   pdl_wait();
   Sched Sd;
-  if (!make_schedule<TT, NTHREADS>(p, sch + 4, sch, Sd)) {
+  if (!make_schedule<TT, NTHREADS>(p, sch + 8, sch, Sd)) {
     if (tid == 0) step_done(p);
     return;
   }

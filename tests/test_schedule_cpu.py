@@ -1,49 +1,103 @@
-"""The decode kernel's split of the flat tile sequence over CTAs, restated on the
-CPU: every CTA owns at least one tile, the CTAs covering a unit are consecutive,
-the owner formula is right, and partial-slot ids are dense (the ticket-based
-combine relies on all three)."""
+"""The decode kernels' split of the tile sequence over CTAs, restated on the
+CPU.  Every non-empty unit (sequence, KV head) occupies W boundary positions
+followed by its tiles in a flat sequence of positions; CTAs split the positions
+evenly, so a CTA whose range crosses into a new unit (and pays a second
+selection switch and segment merge) gets fewer tiles.  Checked here: the real
+tiles of every CTA are contiguous and cover every tile exactly once, the CTAs
+covering a unit are consecutive, the owner formula is right, partial-slot ids
+are dense, and the slot count stays within the workspace bound (the
+ticket-based combine relies on all of it)."""
 import random
 
+W = 4          # boundary positions per unit (kBoundaryTiles in csrc/decode.cu)
 
-def cta_of_tile(t, N, C):
-    c = ((t + 1) * C + N - 1) // N - 1
+
+def cta_of_pos(p, NV, C):
+    c = ((p + 1) * C + NV - 1) // NV - 1
     return min(c, C - 1)
 
 
-def _check(tiles, grid):
+def split(tiles, grid, w=W):
+    """Real tile range [start, end) of every CTA, and the units' virtual starts."""
+    vstart, vs = [], 0
+    for nt in tiles:
+        vstart.append(vs)
+        vs += nt + w if nt else 0
+    NV = vs
+    C = min(grid, NV)
+    N = sum(tiles)
+
+    def real_index(pos):
+        # first real tile at virtual position >= pos (N past the end)
+        r = 0
+        for u, nt in enumerate(tiles):
+            if nt == 0:
+                continue
+            first = vstart[u] + w
+            if pos < first:
+                return r
+            if pos < first + nt:
+                return r + (pos - first)
+            r += nt
+        return N
+
+    ranges = [(real_index(c * NV // C), real_index((c + 1) * NV // C)) for c in range(C)]
+    return ranges, vstart, NV, C
+
+
+def _check(tiles, grid, w=W):
     N = sum(tiles)
     if N == 0:
         return
-    C = min(grid, N)                      # effective grid
-    ranges = [(c * N // C, (c + 1) * N // C) for c in range(C)]
-    assert all(e > s for s, e in ranges)
+    ranges, vstart, NV, C = split(tiles, grid, w)
+    # the CTAs' real ranges tile [0, N) in order
+    pos = 0
+    for s, e in ranges:
+        assert s == pos and e >= s
+        pos = e
+    assert pos == N
     ts = sb = 0
     slots = set()
-    for nt in tiles:
+    for u, nt in enumerate(tiles):
         if nt == 0:
             continue
-        cf, cl = cta_of_tile(ts, N, C), cta_of_tile(ts + nt - 1, N, C)
+        first, last = vstart[u] + w, vstart[u] + w + nt - 1
+        cf, cl = cta_of_pos(first, NV, C), cta_of_pos(last, NV, C)
         cover = [c for c, (s, e) in enumerate(ranges) if s < ts + nt and e > ts]
         assert cover == list(range(cf, cl + 1))
         slots.update(sb + c - cf for c in cover)
-        for t in range(ts, ts + nt):
-            s, e = ranges[cta_of_tile(t, N, C)]
-            assert s <= t < e
+        for j in range(nt):                                  # owner of every tile
+            s, e = ranges[cta_of_pos(first + j, NV, C)]
+            assert s <= ts + j < e
         sb += cl - cf + 1
         ts += nt
     assert slots == set(range(sb))
-    assert sb <= sum(1 for t in tiles if t) + C - 1      # workspace bound: units + CTAs
+    assert sb <= sum(1 for t in tiles if t) + C - 1          # workspace bound: units + CTAs
 
 
 def test_schedule_random():
     rng = random.Random(0)
-    for _ in range(5000):
+    for _ in range(4000):
         tiles = [rng.choice([0, 0, 1, 2, 3, 8, 65]) for _ in range(rng.randint(1, 12))]
-        _check(tiles, rng.randint(1, 160))
+        _check(tiles, rng.randint(1, 160), w=rng.choice([0, 1, 3]))
 
 
 def test_schedule_grid_larger_than_tiles():
-    _check([8, 8, 1, 1, 0, 0, 5, 5], 64)
-    _check([1], 148)
-    _check([64] * 64, 148)
-    _check([1024] * 8, 148)
+    for w in (0, W):
+        _check([8, 8, 1, 1, 0, 0, 5, 5], 64, w)
+        _check([1], 148, w)
+        _check([64] * 64, 148, w)
+        _check([1024] * 8, 148, w)
+
+
+def test_boundary_positions_balance_the_split():
+    """At the Llama decode shape (64 units of 65 tiles over 148 CTAs) the CTAs
+    that cross into a second unit get fewer tiles than those that do not."""
+    tiles = [65] * 64
+    ranges, vstart, NV, C = split(tiles, 148)
+    one, two = [], []
+    starts = {sum(tiles[:u]) for u in range(64)}
+    for s, e in ranges:
+        crosses = any(s < b < e for b in starts)
+        (two if crosses else one).append(e - s)
+    assert two and one and max(two) < max(one)
