@@ -154,7 +154,11 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  *              (len[b] + 1 tokens).  On the device len[b] and n_abs[b] advance
  *              when the step's last kernel finishes.  When NULL the caller
  *              appended the step's key beforehand.
- *   P          [Hkv][d][d] f32
+ *   P          [Hkv][d][d] f32.  Read before the step waits for the
+ *              preceding kernel on the stream, which is safe unless the
+ *              kernel that wrote P released its dependents early through
+ *              programmatic dependent launch (no kernel here that writes P
+ *              does).
  *   k          dimensions kept per query head, 1 <= k <= d_store
  *   scale      score scale; <= 0 selects 1/sqrt(d) (d = full head dim)
  *   out        [B][Hq][d]  out_dtype (AQUA_F32 or AQUA_BF16, RNE)

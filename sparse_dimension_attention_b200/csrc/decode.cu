@@ -127,211 +127,210 @@ __device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, flo
 // ============================================================================
 // query projection + magnitude top-k + group union
 // ============================================================================
-// Selection kernel geometry: NWQ warps project each of the G query heads
-// (each over its own slice of the input dimensions), one more warp appends.
+// Selection kernel geometry: NPW = 4 G warps first project row slices of all
+// G query heads (each warp RW input dims, so P is read from shared memory once
+// per CTA), then rank the dims, four warps per head (32 dims each); one more
+// warp appends the step's key and value.
 template <int G>
 struct QprojCfg {
-  static constexpr int NWQ = (G == 4) ? 2 : 4;
-  static constexpr int WARPS = G * NWQ + 1;
+  static constexpr int NWQ = 4;                 // selection warps per head
+  static constexpr int NPW = G * NWQ;           // projection and selection warps
+  static constexpr int WARPS = NPW + 1;
 };
 constexpr int kPChunks = 4;   // P[g] staged as four 32-row chunks, each with its own barrier
 
 template <typename T, int G>
 __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(DecodeParams p) {
-  constexpr int NWQ = QprojCfg<G>::NWQ;
-  constexpr int ROWS = D / NWQ;                 // input dims per projection warp
+  constexpr int NWQ = QprojCfg<G>::NWQ, NPW = QprojCfg<G>::NPW;
+  constexpr int NPT = NPW * 32;                 // threads of the projection/selection warps
+  constexpr int RW = D / NPW;                   // input dims per projection warp
   constexpr int CROWS = D / kPChunks;           // rows per P chunk
-  static_assert(ROWS % 4 == 0 && (ROWS % CROWS == 0 || CROWS % ROWS == 0), "projection slices vs P chunks");
+  static_assert(NWQ * 32 == D, "four warps of 32 dims rank one head");
+  static_assert(RW % 4 == 0 && CROWS % RW == 0, "projection slices vs P chunks");
   extern __shared__ __align__(128) float Ps[];   // P[g], [D][D]
-  __shared__ __align__(16) float qs[G][D];
-  __shared__ __align__(16) float part[NWQ][G][D];
+  __shared__ __align__(16) float qs[G][D];       // q rows, later the kept scaled q~
+  __shared__ __align__(16) float part[NPW][G][D];
+  __shared__ __align__(16) uint32_t keys[G][D];
   __shared__ __align__(16) float knew_s[D];
-  __shared__ uint32_t masks[G][4];
+  __shared__ uint32_t masks[G][NWQ];
+  __shared__ int nkeep[G][NWQ];
   __shared__ __align__(8) uint64_t pbars[kPChunks];
+  __shared__ int s_abort;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, g = u % p.Hkv;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hw = w / NWQ, sl = w % NWQ;         // head and slice of a projection warp (w < G * NWQ)
-  const int h = g * G + (hw < G ? hw : 0);
   const int m = p.d_store;
   const bool append = p.k_new != nullptr;
 
   if (threadIdx.x == 0) {
     for (int c = 0; c < kPChunks; ++c) mbar_init(&pbars[c], 1);
     fence_barrier_init();
-  }
-  pdl_wait();                // inputs and the cache may come from the previous kernel
-  // Released only after the previous kernel is complete: the attention kernel
-  // then reads lengths and history K~/V before its own wait, which this kernel
-  // does not change (it writes only slot len[b] and leaves len[b] alone).
-  pdl_launch_dependents();
-  __syncthreads();
-  if (threadIdx.x == 0) {
+    // P is staged before the wait on the previous kernel: the kernels that may
+    // still be running then (the attention kernels of a previous step or chunk,
+    // the only ones that release their dependents early) never write it.
     for (int c = 0; c < kPChunks; ++c) {
       mbar_arrive_expect_tx(&pbars[c], CROWS * D * 4);
       bulk_g2s_plain(Ps + c * CROWS * D, p.P + (size_t)g * D * D + c * CROWS * D, CROWS * D * 4, &pbars[c]);
     }
   }
-  if (w < G * NWQ && sl == 0) {
-    const T* qrow = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) qs[hw][4 * lane + s] = Elem<T>::load(qrow + 4 * lane + s);
-  }
+  pdl_wait();                // the other inputs and the cache may come from the previous kernel
+  // Released only after the previous kernel is complete: the attention kernel
+  // then reads lengths and history K~/V before its own wait, which this kernel
+  // does not change (it writes only slot len[b] and leaves len[b] alone).
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) s_abort = 0;
   __syncthreads();
-  bool ok = true;
 
-  const int len_before = __ldcg(p.len + b);   // the append slot
-  if (w == G * NWQ) {
-    // ---- fused append of the new token of unit (b, g), in the key projection order
-    if (append) {
-      for (int c = 0; c < kPChunks; ++c) ok = mbar_wait_bounded(&pbars[c], 0) && ok;
-      const int slot = len_before;
-      if (slot < 0 || slot >= p.Tcap) {
-        if (lane == 0) record_status(p.ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
-      } else {
-        const T* kr = static_cast<const T*>(p.k_new) + (size_t)u * D;
+  if (w == NPW) {
+    // ---- fused append of the new token of unit (b, g), in the key projection
+    // order.  This warp takes no part in the selection below (which does not
+    // depend on it), so the two run side by side.
+    if (!append) return;
+    const int slot = __ldcg(p.len + b);
+    const int nabs = p.pos != nullptr ? __ldcg(p.n_abs + b) : 0;
+    const T* kr = static_cast<const T*>(p.k_new) + (size_t)u * D;
+    const T* vr = static_cast<const T*>(p.v_new) + (size_t)u * D;
+    float kx[4];
+    T vx[4];
 #pragma unroll
-        for (int s2 = 0; s2 < 4; ++s2) knew_s[4 * lane + s2] = Elem<T>::load(kr + 4 * lane + s2);
-        __syncwarp();
-        float kt[4];
-        project_row_smem(Ps, knew_s, lane, kt);
-        T* kp = const_cast<T*>(static_cast<const T*>(p.kproj)) + (size_t)u * p.d_store * p.Tcap + slot;
-#pragma unroll
-        for (int s2 = 0; s2 < 4; ++s2) {
-          const int jd = 4 * lane + s2;
-          if (jd < p.d_store) kp[(size_t)jd * p.Tcap] = Elem<T>::from_f32(kt[s2]);
-        }
-        T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * D;
-        const T* vr = static_cast<const T*>(p.v_new) + (size_t)u * D;
-#pragma unroll
-        for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = vr[4 * lane + s2];
-        if (p.pos != nullptr && lane == 0) {
-          p.pos[(size_t)u * p.Tcap + slot] = __ldcg(p.n_abs + b);
-          p.score[(size_t)u * p.Tcap + slot] = 0.f;
-        }
-      }
+    for (int s2 = 0; s2 < 4; ++s2) {
+      kx[s2] = Elem<T>::load(kr + 4 * lane + s2);
+      vx[s2] = vr[4 * lane + s2];
     }
-  } else if (w < G * NWQ) {
-    // partial q~ of head hw over input dims [sl*ROWS, (sl+1)*ROWS), outputs
-    // 4*lane .. 4*lane+3: two chains (even / odd rows), each chunk as it lands
-    float a[4] = {0.f, 0.f, 0.f, 0.f}, c4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int i0 = sl * ROWS; i0 < (sl + 1) * ROWS; i0 += 4) {
-      if (i0 % CROWS == 0) ok = mbar_wait_bounded(&pbars[i0 / CROWS], 0) && ok;
-      const float4 x4 = *reinterpret_cast<const float4*>(&qs[hw][i0]);
+    bool ok = true;
+    for (int c = 0; c < kPChunks; ++c) ok = mbar_wait_bounded(&pbars[c], 0) && ok;
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+      return;
+    }
+    if (slot < 0 || slot >= p.Tcap) {
+      if (lane == 0) record_status(p.ctrl, AQUA_ERR_ARG);   // device length beyond capacity: write nothing
+      return;
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) knew_s[4 * lane + s2] = kx[s2];
+    __syncwarp();
+    float kt[4];
+    project_row_smem(Ps, knew_s, lane, kt);
+    T* kp = const_cast<T*>(static_cast<const T*>(p.kproj)) + (size_t)u * p.d_store * p.Tcap + slot;
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) {
+      const int jd = 4 * lane + s2;
+      if (jd < p.d_store) kp[(size_t)jd * p.Tcap] = Elem<T>::from_f32(kt[s2]);
+    }
+    T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * D;
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = vx[s2];
+    if (p.pos != nullptr && lane == 0) {
+      p.pos[(size_t)u * p.Tcap + slot] = nabs;
+      p.score[(size_t)u * p.Tcap + slot] = 0.f;
+    }
+    return;
+  }
+
+  // ---- projection/selection warps (named barrier 1 over their NPT threads)
+  if (w < G) {
+    const T* qrow = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + g * G + w) * D;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) qs[w][4 * lane + s] = Elem<T>::load(qrow + 4 * lane + s);
+  }
+  named_bar_sync(1, NPT);
+  {
+    // partial q~ of every head over input dims [w*RW, (w+1)*RW), outputs
+    // 4*lane .. 4*lane+3: two chains per head (even / odd rows)
+    const bool ok = mbar_wait_bounded(&pbars[w * RW / CROWS], 0);
+    float a[G][4], c4[G][4];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2) a[hh][s2] = c4[hh][s2] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RW; r += 4) {
+      const int i0 = w * RW + r;
       const float4 p0 = reinterpret_cast<const float4*>(Ps + (i0 + 0) * D)[lane];
       const float4 p1 = reinterpret_cast<const float4*>(Ps + (i0 + 1) * D)[lane];
       const float4 p2 = reinterpret_cast<const float4*>(Ps + (i0 + 2) * D)[lane];
       const float4 p3 = reinterpret_cast<const float4*>(Ps + (i0 + 3) * D)[lane];
-      a[0] = fmaf(x4.x, p0.x, a[0]); a[1] = fmaf(x4.x, p0.y, a[1]); a[2] = fmaf(x4.x, p0.z, a[2]); a[3] = fmaf(x4.x, p0.w, a[3]);
-      c4[0] = fmaf(x4.y, p1.x, c4[0]); c4[1] = fmaf(x4.y, p1.y, c4[1]); c4[2] = fmaf(x4.y, p1.z, c4[2]); c4[3] = fmaf(x4.y, p1.w, c4[3]);
-      a[0] = fmaf(x4.z, p2.x, a[0]); a[1] = fmaf(x4.z, p2.y, a[1]); a[2] = fmaf(x4.z, p2.z, a[2]); a[3] = fmaf(x4.z, p2.w, a[3]);
-      c4[0] = fmaf(x4.w, p3.x, c4[0]); c4[1] = fmaf(x4.w, p3.y, c4[1]); c4[2] = fmaf(x4.w, p3.z, c4[2]); c4[3] = fmaf(x4.w, p3.w, c4[3]);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float4 x4 = *reinterpret_cast<const float4*>(&qs[hh][i0]);
+        float* A = a[hh];
+        float* C = c4[hh];
+        A[0] = fmaf(x4.x, p0.x, A[0]); A[1] = fmaf(x4.x, p0.y, A[1]); A[2] = fmaf(x4.x, p0.z, A[2]); A[3] = fmaf(x4.x, p0.w, A[3]);
+        C[0] = fmaf(x4.y, p1.x, C[0]); C[1] = fmaf(x4.y, p1.y, C[1]); C[2] = fmaf(x4.y, p1.z, C[2]); C[3] = fmaf(x4.y, p1.w, C[3]);
+        A[0] = fmaf(x4.z, p2.x, A[0]); A[1] = fmaf(x4.z, p2.y, A[1]); A[2] = fmaf(x4.z, p2.z, A[2]); A[3] = fmaf(x4.z, p2.w, A[3]);
+        C[0] = fmaf(x4.w, p3.x, C[0]); C[1] = fmaf(x4.w, p3.y, C[1]); C[2] = fmaf(x4.w, p3.z, C[2]); C[3] = fmaf(x4.w, p3.w, C[3]);
+      }
     }
 #pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) part[sl][hw][4 * lane + s2] = a[s2] + c4[s2];
+    for (int hh = 0; hh < G; ++hh)
+      *reinterpret_cast<float4*>(&part[w][hh][4 * lane]) =
+          make_float4(a[hh][0] + c4[hh][0], a[hh][1] + c4[hh][1], a[hh][2] + c4[hh][2], a[hh][3] + c4[hh][3]);
+    if (!ok) s_abort = 1;
   }
-  if (__syncthreads_or(!ok)) {
+  named_bar_sync(1, NPT);
+  if (s_abort) {
     if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
     return;
   }
-  if (w < G * NWQ && sl == 0) {
-    // q~_j for j = 4*lane + s: the slices' partials added in slice order
-    float qt[4];
-#pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) {
-      float y = part[0][hw][4 * lane + s2];
-#pragma unroll
-      for (int x = 1; x < NWQ; ++x) y += part[x][hw][4 * lane + s2];
-      qt[s2] = y;
-    }
 
-    // Keys: magnitude bits + 1 for candidate dims (j < m), 0 otherwise, so that
-    // unsigned order equals |q~| order and non-candidates rank below everything.
-    uint32_t key[4];
+  // ---- selection: warp (hw, sl) ranks dims i = 32 sl + lane of head hw.
+  // Keys: magnitude bits + 1 for candidate dims (i < m), 0 otherwise, so that
+  // unsigned order equals |q~| order and non-candidates rank below every
+  // candidate (NaN payloads are clamped to one key above inf).  rank_i = #{j : key_j > key_i} + #{j < i : key_j == key_i}
+  // (ties to the lower index) and dim i is kept iff i < m and rank_i < k.
+  const int hw = w / NWQ, sl = w % NWQ;
+  const int h = g * G + hw;
+  const size_t bh = (size_t)b * p.Hq + h;
+  const int i = 32 * sl + lane;
+  float qt = part[0][hw][i];                    // q~_i: the slices' partials added in slice order
 #pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) {
-      const int j = 4 * lane + s2;
-      key[s2] = (j < m) ? (__float_as_uint(fabsf(qt[s2])) + 1u) : 0u;
-    }
-    // Radix select of the k-th largest key: the largest tau with
-    // #{key >= tau} >= k, one bit per round, counts by ballot + popc; done as
-    // soon as exactly k keys are >= tau (the set is then already decided).
-    uint32_t tau = 0;
-    int cnt = D;
-#pragma unroll 1
-    for (int bit = 31; bit >= 0 && cnt != p.k; --bit) {
-      const uint32_t cand = tau | (1u << bit);
-      const int c = __popc(__ballot_sync(0xffffffffu, key[0] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[1] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[2] >= cand)) +
-                    __popc(__ballot_sync(0xffffffffu, key[3] >= cand));
-      if (c >= p.k) {
-        tau = cand;
-        cnt = c;
-      }
-    }
-    int ngt = 0, neq = 0;
-  #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      ngt += __popc(__ballot_sync(0xffffffffu, key[s] > tau));
-      neq += (key[s] == tau);
-    }
-    const int need = p.k - ngt;  // ties to take, lowest index first
-    int incl = neq;
-  #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int rank = incl - neq;
-    bool sel[4];
-    int nsel = 0;
-  #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      sel[s] = key[s] > tau;
-      if (key[s] == tau) {
-        sel[s] = rank < need;
-        ++rank;
-      }
-      nsel += sel[s];
-    }
-    int pincl = nsel;
-  #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, pincl, o);
-      if (lane >= o) pincl += y;
-    }
-    int opos = pincl - nsel;
-    const size_t bh = (size_t)b * p.Hq + h;
-  #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const int j = 4 * lane + s;
-      if (sel[s]) {
-        if (p.sel_out) p.sel_out[bh * p.k + opos] = j;
-        ++opos;
-      }
-      if (p.qproj_out) p.qproj_out[bh * D + j] = qt[s];
-      qs[hw][j] = sel[s] ? qt[s] * p.scale_log2 : 0.f;
-    }
-    const uint32_t nib = (uint32_t)sel[0] | ((uint32_t)sel[1] << 1) | ((uint32_t)sel[2] << 2) |
-                         ((uint32_t)sel[3] << 3);
-    const uint32_t shifted = nib << (4 * (lane & 7));
-  #pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-      const uint32_t word = __reduce_or_sync(0xffffffffu, (lane >> 3) == wd ? shifted : 0u);
-      if (lane == 0) masks[hw][wd] = word;
-    }
+  for (int x = 1; x < NPW; ++x) qt += part[x][hw][i];
+  const uint32_t ki = i < m ? min(__float_as_uint(fabsf(qt)), 0x7F800001u) + 1u : 0u;   // NaN above inf
+  keys[hw][i] = ki;
+  named_bar_sync(1, NPT);
+  // Keys are below 2^31, so key_j > key_i exactly when key_i - key_j wraps
+  // around, i.e. has its top bit set: one subtraction and one shifted add each.
+  uint32_t gt = 0;
+  const uint4* kv = reinterpret_cast<const uint4*>(keys[hw]);
+#pragma unroll 8
+  for (int j4 = 0; j4 < D / 4; ++j4) {
+    const uint4 kj = kv[j4];
+    gt += ((ki - kj.x) >> 31) + ((ki - kj.y) >> 31) + ((ki - kj.z) >> 31) + ((ki - kj.w) >> 31);
   }
+  // Equal keys share gt, so exactly k candidates have gt < k unless a group of
+  // equal keys straddles the cut; only then is the index order needed.
+  bool keep = i < m && (int)gt < p.k;
+  uint32_t bal = __ballot_sync(0xffffffffu, keep);
+  if (lane == 0) nkeep[hw][sl] = __popc(bal);
+  named_bar_sync(1, NPT);
+  int tot = 0;
+#pragma unroll
+  for (int x = 0; x < NWQ; ++x) tot += nkeep[hw][x];
+  if (tot > p.k) {                              // uniform over the head's warps
+    if (keep) {
+      int eq_lo = 0;
+      for (int j = 0; j < i; ++j) eq_lo += keys[hw][j] == ki;
+      keep = (int)gt + eq_lo < p.k;
+    }
+    bal = __ballot_sync(0xffffffffu, keep);
+  }
+  if (lane == 0) masks[hw][sl] = bal;
+  if (p.qproj_out) p.qproj_out[bh * D + i] = qt;
+  qs[hw][i] = keep ? qt * p.scale_log2 : 0.f;
 
   // sequences with no tokens: zero output, lse = -inf
-  if (w < G * NWQ && sl == 0 && !append && seq_len(p.len, b, p.Tcap) <= 0) {
-    const size_t bh = (size_t)b * p.Hq + h;
+  if (sl == 0 && !append && seq_len(p.len, b, p.Tcap) <= 0) {
     for (int j = lane; j < D; j += 32) store_val(p, bh * D + j, 0.f);
     if (p.lse_out && lane == 0) p.lse_out[bh] = -INFINITY;
   }
-  __syncthreads();
+  named_bar_sync(1, NPT);
 
+  if (p.sel_out && keep) {                      // kept dims of the head in ascending order
+    int pos = __popc(bal & ((1u << lane) - 1u));
+    for (int x = 0; x < sl; ++x) pos += __popc(masks[hw][x]);
+    p.sel_out[bh * p.k + pos] = i;
+  }
   uint32_t um[4];
 #pragma unroll
   for (int wd = 0; wd < 4; ++wd) {
@@ -340,7 +339,7 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
     for (int hh = 0; hh < G; ++hh) x |= masks[hh][wd];
     um[wd] = x;
   }
-  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+  for (int j = threadIdx.x; j < D; j += NPT) {
     const int wd = j >> 5, bit = j & 31;
     // register selects instead of a run-time index into um[]
     const uint32_t word = wd == 0 ? um[0] : (wd == 1 ? um[1] : (wd == 2 ? um[2] : um[3]));
@@ -390,35 +389,51 @@ __device__ __forceinline__ int cta_of_pos(long long p, long long NV, int C) {
   return (int)(c < C - 1 ? c : C - 1);
 }
 
-// exclusive scan over all NT threads of the block; *total receives the sum
+// exclusive scans of two values over all NT threads of the block at once;
+// tot[0], tot[1] receive the sums
 template <int NT>
-__device__ __forceinline__ long long block_excl_scan(long long v, long long* sh, long long* total) {
+__device__ __forceinline__ void block_excl_scan2(long long v0, long long v1, long long* sh, long long (&excl)[2],
+                                                 long long (&tot)[2]) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int NW = NT / 32;
   static_assert(NW <= 32, "scan uses one warp for the warp totals");
-  long long x = v;
+  long long x0 = v0, x1 = v1;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const long long y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
+    const long long y0 = __shfl_up_sync(0xffffffffu, x0, o);
+    const long long y1 = __shfl_up_sync(0xffffffffu, x1, o);
+    if (lane >= o) {
+      x0 += y0;
+      x1 += y1;
+    }
   }
-  if (lane == 31) sh[warp] = x;
+  if (lane == 31) {
+    sh[warp] = x0;
+    sh[NW + warp] = x1;
+  }
   __syncthreads();
   if (warp == 0) {
-    long long y = lane < NW ? sh[lane] : 0;
+    long long y0 = lane < NW ? sh[lane] : 0, y1 = lane < NW ? sh[NW + lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long z = __shfl_up_sync(0xffffffffu, y, o);
-      if (lane >= o) y += z;
+      const long long z0 = __shfl_up_sync(0xffffffffu, y0, o);
+      const long long z1 = __shfl_up_sync(0xffffffffu, y1, o);
+      if (lane >= o) {
+        y0 += z0;
+        y1 += z1;
+      }
     }
-    if (lane < NW) sh[lane] = y;
+    if (lane < NW) {
+      sh[lane] = y0;
+      sh[NW + lane] = y1;
+    }
   }
   __syncthreads();
-  const long long base = warp > 0 ? sh[warp - 1] : 0;
-  *total = sh[NW - 1];
-  const long long excl = base + x - v;
+  excl[0] = (warp > 0 ? sh[warp - 1] : 0) + x0 - v0;
+  excl[1] = (warp > 0 ? sh[NW + warp - 1] : 0) + x1 - v1;
+  tot[0] = sh[NW - 1];
+  tot[1] = sh[2 * NW - 1];
   __syncthreads();
-  return excl;
 }
 
 struct Sched {
@@ -429,8 +444,21 @@ struct Sched {
   long long ts0, sb0, vs0;     // its first tile, first partial slot and first position
 };
 
+template <int TT>
+__device__ __forceinline__ long long unit_tiles(const DecodeParams& p, int u) {
+  return (kv_len(p, u / p.Hkv) + TT - 1) / TT;
+}
+
+// Partial slots: the segment of unit u on CTA c uses slot u + c.  The CTAs
+// covering a unit are consecutive and a later unit never starts on an earlier
+// CTA, so slots are distinct, consecutive within a unit, and below
+// n_units + C - 1 (no scan over the segment counts is needed).
+//
 // This CTA's tiles and first unit.  Returns false (for the whole CTA) when the
-// CTA has no tile.  `scratch` needs 32 long longs; sch[0..7] receive results.
+// CTA has no tile.  `scratch` needs 2 * NT / 32 long longs; sch[0..7] receive
+// results.  All NT threads take part: one paired scan of the units' tile and
+// position counts, then the thread whose units hold this CTA's first and last
+// positions writes them to sch.
 template <int TT, int NT>
 __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long long* sch, Sched& S) {
   const int tid = threadIdx.x;
@@ -438,47 +466,34 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   const int c = blockIdx.x;
   const int chunk = (n_units + NT - 1) / NT;
   const int u_lo = min(n_units, tid * chunk), u_hi = min(n_units, u_lo + chunk);
+  const long long nt_lo = u_lo < u_hi ? unit_tiles<TT>(p, u_lo) : 0;   // the usual case: one unit per thread
   long long my_tiles = 0, my_pos = 0;
   for (int u = u_lo; u < u_hi; ++u) {
-    const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
+    const long long nt = u == u_lo ? nt_lo : unit_tiles<TT>(p, u);
     my_tiles += nt;
     my_pos += nt > 0 ? nt + kBoundaryTiles : 0;
   }
-  long long N, NV;
-  const long long t_excl = block_excl_scan<NT>(my_tiles, scratch, &N);
-  const long long v_excl = block_excl_scan<NT>(my_pos, scratch, &NV);
+  long long excl[2], tot[2];
+  block_excl_scan2<NT>(my_tiles, my_pos, scratch, excl, tot);
+  const long long N = tot[0], NV = tot[1];
   const int C = (int)min((long long)gridDim.x, NV);
   if (c >= C) return false;
   const long long a = (long long)c * NV / C, e = (long long)(c + 1) * NV / C;   // this CTA's positions
-  long long my_segs = 0;
-  {
-    long long vs = v_excl;
-    for (int u = u_lo; u < u_hi; ++u) {
-      const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
-      if (nt == 0) continue;
-      const long long first = vs + kBoundaryTiles;
-      my_segs += cta_of_pos(first + nt - 1, NV, C) - cta_of_pos(first, NV, C) + 1;
-      vs = first + nt;
-    }
-  }
-  long long NS;
-  const long long s_excl = block_excl_scan<NT>(my_segs, scratch, &NS);
   if (tid == 0 && e == NV) sch[1] = N;    // the last CTA's tiles run to the end
   {
-    long long ts = t_excl, vs = v_excl, sb = s_excl;
+    long long ts = excl[0], vs = excl[1];
     for (int u = u_lo; u < u_hi; ++u) {
-      const long long nt = (kv_len(p, u / p.Hkv) + TT - 1) / TT;
+      const long long nt = u == u_lo ? nt_lo : unit_tiles<TT>(p, u);
       if (nt == 0) continue;
       const long long first = vs + kBoundaryTiles, end = first + nt;   // unit's positions: [vs, end)
       if (vs <= a && a < end) {          // the range starts in this unit: its first tile at or after a
         sch[0] = ts + (a > first ? a - first : 0);
         sch[2] = u;
         sch[3] = ts;
-        sch[4] = sb;
+        sch[4] = u + cta_of_pos(first, NV, C);
         sch[5] = vs;
       }
       if (vs <= e && e < end) sch[1] = ts + (e > first ? e - first : 0);
-      sb += cta_of_pos(end - 1, NV, C) - cta_of_pos(first, NV, C) + 1;
       ts += nt;
       vs = end;
     }
@@ -498,10 +513,10 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
 
 // Walks the units of this CTA's tile range; one instance per producer warp.
 struct UnitWalker {
-  int u, b, Tb, nU, nseg, cf;
-  long long ts, te, sb, vs;    // unit u: tiles [ts, te), first partial slot, first position
+  int u = 0, b = 0, Tb = 0, nU = 0, nseg = 0, cf = 0;
+  long long ts = 0, te = 0, sb = 0, vs = 0;   // unit u: tiles [ts, te), first partial slot, first position
   template <int TT>
-  __device__ void start(const DecodeParams& p, const Sched& S) {
+  __device__ void start(const DecodeParams& p, const Sched& S, bool with_nU = true) {
     u = S.u0;
     ts = S.ts0;
     sb = S.sb0;
@@ -511,14 +526,13 @@ struct UnitWalker {
     te = ts + (Tb + TT - 1) / TT;
     cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
     nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
-    nU = p.ucount[u];
+    nU = with_nU ? p.ucount[u] : 0;
   }
   // advance to the unit holding flat tile t; true when the unit changed
   template <int TT>
-  __device__ bool seek(const DecodeParams& p, const Sched& S, long long t) {
+  __device__ bool seek(const DecodeParams& p, const Sched& S, long long t, bool with_nU = true) {
     bool changed = false;
     while (t >= te) {
-      sb += nseg;
       if (te > ts) vs += kBoundaryTiles + (te - ts);
       ++u;
       b = u / p.Hkv;
@@ -528,7 +542,8 @@ struct UnitWalker {
       if (te > ts) {
         cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
         nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
-        nU = p.ucount[u];
+        sb = u + cf;
+        nU = with_nU ? p.ucount[u] : 0;
       } else {
         nseg = 0;
       }
@@ -678,9 +693,13 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_last[1] = 0;
 
-  // shared memory starts zeroed: padding rows and never-copied tokens must be finite
-  for (int i = tid; i < NSTAGE * S::STAGE / 16; i += NTHREADS_BF16)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
+  // the K~ rows of every stage start zeroed: union padding rows and never-copied
+  // tokens must be finite (the V halves are rewritten whole by every tile copy)
+  constexpr int KQ = S::KBYTES / 16;
+  for (int i = tid; i < NSTAGE * KQ; i += NTHREADS_BF16) {
+    const int s = i / KQ;
+    reinterpret_cast<uint4*>(smem + (size_t)s * S::STAGE + 2 * S::VHALF)[i - s * KQ] = make_uint4(0, 0, 0, 0);
+  }
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       // arrivals: one cp.async arrival per producer thread + the V tensor-copy arrival
@@ -701,6 +720,28 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   fence_proxy_async_smem();
   __syncthreads();
   const int n_tiles = has_work ? (int)(Sd.my_end - Sd.my_start) : 0;
+  // V tiles of the first stages are issued before the wait when they cannot
+  // hold this step's appended token (a unit's last tile holds it): nothing
+  // else the projection kernel writes is in them, and everything before it
+  // on the stream is complete once it has released this kernel.
+  uint32_t v_early = 0;
+  if (has_work && tid == NCT) {
+    const uint64_t pol = policy_evict_first();
+    UnitWalker W0;
+    W0.start<TT>(p, Sd, false);
+    for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
+      const long long t = Sd.my_start + it;
+      W0.seek<TT>(p, Sd, t, false);
+      const int t0 = (int)(t - W0.ts) * TT;
+      if (t0 + TT >= W0.Tb) break;
+      unsigned char* st = smem + (size_t)it * S::STAGE;
+      mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
+      const int row = W0.u * p.Tcap + t0;
+      tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
+      tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
+      v_early |= 1u << it;
+    }
+  }
   pdl_launch_dependents();
   pdl_wait();   // the projection kernel (and its append) must be complete
   if (!has_work) {
@@ -718,12 +759,13 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     UnitWalker W;
     W.start<TT>(p, Sd);
     if (pt == 0) {
-      // V tiles of the first stages do not depend on the union list: issue
-      // them before the union rows are fetched
+      // the other V tiles of the first stages do not depend on the union
+      // list either: issue them before the union rows are fetched
       UnitWalker W0 = W;
       for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
         const long long t = Sd.my_start + it;
         W0.seek<TT>(p, Sd, t);
+        if ((v_early >> it) & 1u) continue;
         const StageHdr h0 = W0.header(Sd, t, TT);
         unsigned char* st = smem + (size_t)it * S::STAGE;
         mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
@@ -1333,15 +1375,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 // ============================================================================
 template <typename T, int G>
 int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
+  // With no more units than SMs, the dynamic shared memory request is raised
+  // above half an SM's so that every CTA gets an SM of its own: the kernel is
+  // latency-bound, and CTAs sharing an SM were measured to take twice as long.
+  constexpr int kOwnSm = 116 * 1024;
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(qproj_topk_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, D * D * 4) !=
+    if (cudaFuncSetAttribute(qproj_topk_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOwnSm) !=
         cudaSuccess)
       return check_launch("cudaFuncSetAttribute(qproj_topk_kernel)");
     configured = true;
   }
+  const int smem = n_units <= device_sm_count() ? kOwnSm : D * D * 4;
   const cudaError_t e =
-      launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), D * D * 4, st, p);
+      launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), smem, st, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
   return check_launch("qproj_topk_kernel");
 }

@@ -4,9 +4,10 @@ followed by its tiles in a flat sequence of positions; CTAs split the positions
 evenly, so a CTA whose range crosses into a new unit (and pays a second
 selection switch and segment merge) gets fewer tiles.  Checked here: the real
 tiles of every CTA are contiguous and cover every tile exactly once, the CTAs
-covering a unit are consecutive, the owner formula is right, partial-slot ids
-are dense, and the slot count stays within the workspace bound (the
-ticket-based combine relies on all of it)."""
+covering a unit are consecutive, the owner formula is right, and the partial
+slots (unit u on CTA c takes slot u + c) are distinct, consecutive within a
+unit and below the workspace bound (the ticket-based combine relies on all of
+it)."""
 import random
 
 W = 4          # boundary positions per unit (kBoundaryTiles in csrc/decode.cu)
@@ -56,8 +57,8 @@ def _check(tiles, grid, w=W):
         assert s == pos and e >= s
         pos = e
     assert pos == N
-    ts = sb = 0
-    slots = set()
+    ts = 0
+    slots = []
     for u, nt in enumerate(tiles):
         if nt == 0:
             continue
@@ -65,14 +66,13 @@ def _check(tiles, grid, w=W):
         cf, cl = cta_of_pos(first, NV, C), cta_of_pos(last, NV, C)
         cover = [c for c, (s, e) in enumerate(ranges) if s < ts + nt and e > ts]
         assert cover == list(range(cf, cl + 1))
-        slots.update(sb + c - cf for c in cover)
+        slots += [u + c for c in cover]                      # consecutive within the unit
         for j in range(nt):                                  # owner of every tile
             s, e = ranges[cta_of_pos(first + j, NV, C)]
             assert s <= ts + j < e
-        sb += cl - cf + 1
         ts += nt
-    assert slots == set(range(sb))
-    assert sb <= sum(1 for t in tiles if t) + C - 1          # workspace bound: units + CTAs
+    assert len(set(slots)) == len(slots)                     # distinct across units
+    assert max(slots) < len(tiles) + C - 1                   # workspace bound: units + CTAs
 
 
 def test_schedule_random():
