@@ -208,6 +208,16 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t 
                : "memory");
 }
 
+// 4-, 8- or 16-byte asynchronous copy global -> shared (both addresses aligned to the size)
+template <int N>
+__device__ __forceinline__ void cp_async_small(void* dst, const void* src) {
+  static_assert(N == 4 || N == 8 || N == 16, "cp.async copies 4, 8 or 16 bytes");
+  if constexpr (N == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_u32(dst)), "l"(src), "n"(N) : "memory");
+}
+
 // arrive on `bar` once every cp.async this thread issued so far has landed
 // (the arrival is one of the barrier's expected arrivals)
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
@@ -222,6 +232,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// GPU-scope fetch-and-add with acquire-release semantics (returns the old value)
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

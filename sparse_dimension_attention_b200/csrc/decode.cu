@@ -58,7 +58,8 @@ struct DecodeParams {
   const void* kproj;
   const void* v;
   void* out;
-  float* qm;          // [n_units][D][G]
+  float* qm;          // [n_units][D][G] masked scaled q~ of the union rows, union order
+  float* qmn;         // [n_units][D][G] the same in dimension order (0 for dims no head kept)
   int32_t* ulist;     // [n_units][D]
   int32_t* ucount;    // [n_units]
   int32_t* counters;  // [n_units]
@@ -95,9 +96,7 @@ __device__ __forceinline__ int kv_len(const DecodeParams& p, int b) {
 // of the grid advances the lengths of a step with a fused append.
 __device__ __forceinline__ void step_done(const DecodeParams& p) {
   if (p.len_add == 0) return;
-  __threadfence();
-  if (atomicAdd(p.ctrl + kCtrlStepTicket, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
-    __threadfence();
+  if (atom_add_acq_rel_gpu(p.ctrl + kCtrlStepTicket, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
     for (int bb = 0; bb < p.B; ++bb) {
       p.len_w[bb] += p.len_add;
       if (p.n_abs) p.n_abs[bb] += p.len_add;
@@ -340,6 +339,9 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
     um[wd] = x;
   }
   for (int j = threadIdx.x; j < D; j += NPT) {
+    float* dn = p.qmn + ((size_t)u * D + j) * G;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) dn[hh] = qs[hh][j];
     const int wd = j >> 5, bit = j & 31;
     // register selects instead of a run-time index into um[]
     const uint32_t word = wd == 0 ? um[0] : (wd == 1 ? um[1] : (wd == 2 ? um[2] : um[3]));
@@ -374,14 +376,15 @@ struct StageHdr {
 constexpr int kFirst = 1, kLast = 2;
 
 // The tiles of all (sequence, KV head) units form one flat sequence of
-// positions in which every non-empty unit first occupies kBoundaryTiles
-// positions without work, then one position per tile.  CTA c takes positions
-// [floor(c NV / C), floor((c+1) NV / C)): a CTA whose range crosses into a
-// new unit pays a second segment merge and a switch of the selection data
-// (measured at about four tiles' time at the Llama decode shape) and receives
-// that many fewer tiles.  Its tiles are the real positions of its range,
-// which are consecutive in the plain tile order.
-constexpr int kBoundaryTiles = 4;
+// positions in which every non-empty unit first occupies kBoundaryPos
+// positions without work, then kTilePos positions per tile.  CTA c takes
+// positions [floor(c NV / C), floor((c+1) NV / C)) and the tiles whose first
+// position lies in that range (consecutive in the plain tile order).  A CTA
+// whose range crosses into a new unit pays a second segment merge and a
+// switch of the selection data, about 3.5 tiles' time at the Llama decode
+// shape (fitted to per-CTA timings), and receives that many fewer tiles.
+constexpr int kTilePos = 4;
+constexpr int kBoundaryPos = 14;
 
 // CTA whose range holds position p (positions split as above over C CTAs)
 __device__ __forceinline__ int cta_of_pos(long long p, long long NV, int C) {
@@ -471,12 +474,14 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   for (int u = u_lo; u < u_hi; ++u) {
     const long long nt = u == u_lo ? nt_lo : unit_tiles<TT>(p, u);
     my_tiles += nt;
-    my_pos += nt > 0 ? nt + kBoundaryTiles : 0;
+    my_pos += nt > 0 ? nt * kTilePos + kBoundaryPos : 0;
   }
   long long excl[2], tot[2];
   block_excl_scan2<NT>(my_tiles, my_pos, scratch, excl, tot);
   const long long N = tot[0], NV = tot[1];
-  const int C = (int)min((long long)gridDim.x, NV);
+  // at least kTilePos positions per CTA, so that every CTA between the first
+  // and last owner of a unit's tiles owns one of them (the merge counts them)
+  const int C = (int)min((long long)gridDim.x, max(1LL, NV / kTilePos));
   if (c >= C) return false;
   const long long a = (long long)c * NV / C, e = (long long)(c + 1) * NV / C;   // this CTA's positions
   if (tid == 0 && e == NV) sch[1] = N;    // the last CTA's tiles run to the end
@@ -485,15 +490,15 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
     for (int u = u_lo; u < u_hi; ++u) {
       const long long nt = u == u_lo ? nt_lo : unit_tiles<TT>(p, u);
       if (nt == 0) continue;
-      const long long first = vs + kBoundaryTiles, end = first + nt;   // unit's positions: [vs, end)
-      if (vs <= a && a < end) {          // the range starts in this unit: its first tile at or after a
-        sch[0] = ts + (a > first ? a - first : 0);
+      const long long first = vs + kBoundaryPos, end = first + nt * kTilePos;   // unit's positions: [vs, end)
+      if (vs <= a && a < end) {          // the range starts in this unit: its first tile starts at or after a
+        sch[0] = ts + (a > first ? (a - first + kTilePos - 1) / kTilePos : 0);
         sch[2] = u;
         sch[3] = ts;
         sch[4] = u + cta_of_pos(first, NV, C);
         sch[5] = vs;
       }
-      if (vs <= e && e < end) sch[1] = ts + (e > first ? e - first : 0);
+      if (vs <= e && e < end) sch[1] = ts + (e > first ? (e - first + kTilePos - 1) / kTilePos : 0);
       ts += nt;
       vs = end;
     }
@@ -514,7 +519,14 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
 // Walks the units of this CTA's tile range; one instance per producer warp.
 struct UnitWalker {
   int u = 0, b = 0, Tb = 0, nU = 0, nseg = 0, cf = 0;
+  int nTb = 0, nnU = 0;                       // unit u + 1's length and union size, loaded on entering u
   long long ts = 0, te = 0, sb = 0, vs = 0;   // unit u: tiles [ts, te), first partial slot, first position
+  __device__ void preload(const DecodeParams& p, bool with_nU) {
+    if (u + 1 < p.B * p.Hkv) {
+      nTb = kv_len(p, (u + 1) / p.Hkv);
+      nnU = with_nU ? p.ucount[u + 1] : 0;
+    }
+  }
   template <int TT>
   __device__ void start(const DecodeParams& p, const Sched& S, bool with_nU = true) {
     u = S.u0;
@@ -524,26 +536,29 @@ struct UnitWalker {
     b = u / p.Hkv;
     Tb = kv_len(p, b);
     te = ts + (Tb + TT - 1) / TT;
-    cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
-    nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
+    cf = cta_of_pos(vs + kBoundaryPos, S.NV, S.C);
+    nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, S.NV, S.C) - cf + 1;
     nU = with_nU ? p.ucount[u] : 0;
+    preload(p, with_nU);
   }
   // advance to the unit holding flat tile t; true when the unit changed
   template <int TT>
   __device__ bool seek(const DecodeParams& p, const Sched& S, long long t, bool with_nU = true) {
     bool changed = false;
     while (t >= te) {
-      if (te > ts) vs += kBoundaryTiles + (te - ts);
+      if (te > ts) vs += kBoundaryPos + (te - ts) * kTilePos;
       ++u;
       b = u / p.Hkv;
-      Tb = kv_len(p, b);
+      Tb = nTb;                 // preloaded when the previous unit was entered
+      const int nU1 = nnU;
       ts = te;
       te = ts + (Tb + TT - 1) / TT;
+      preload(p, with_nU);
       if (te > ts) {
-        cf = cta_of_pos(vs + kBoundaryTiles, S.NV, S.C);
-        nseg = cta_of_pos(vs + kBoundaryTiles + (te - ts) - 1, S.NV, S.C) - cf + 1;
+        cf = cta_of_pos(vs + kBoundaryPos, S.NV, S.C);
+        nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, S.NV, S.C) - cf + 1;
         sb = u + cf;
-        nU = with_nU ? p.ucount[u] : 0;
+        nU = nU1;
       } else {
         nseg = 0;
       }
@@ -605,31 +620,22 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
   // publish this partial and take a ticket; the unit's last arrival merges.
   // The barrier orders every thread's partial stores before thread 0's
   // GPU-scope fence (fences are cumulative), which precedes the ticket.
+  // (the pattern of a barrier, then one thread's release, orders every
+  // thread's partial stores before the ticket; the last arrival's acquire,
+  // then a barrier, orders the other partials before every thread's loads)
   named_bar_sync(1, NCT);
-  if (tid == 0) {
-    __threadfence();
-    *s_last = (atomicAdd(p.counters + hh.u, 1) == hh.nseg - 1);
-  }
+  if (tid == 0) *s_last = (atom_add_acq_rel_gpu(p.counters + hh.u, 1) == hh.nseg - 1);
   named_bar_sync(1, NCT);
   if (!*s_last) return;
-  __threadfence();
   constexpr int MB = 8;   // partials fetched per round, loads in flight together
 #pragma unroll 1
   for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
     const int idx = tid + NCT * i;
     if (idx >= G * D) break;
     const int h = idx / D, dim = idx % D;
-    float M = -INFINITY;
-#pragma unroll 1
-    for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
-      float mv[MB];
-#pragma unroll
-      for (int j = 0; j < MB; ++j)
-        mv[j] = (s0 + j < hh.nseg) ? __ldcg(p.part_ml + ((size_t)(hh.seg0 + s0 + j) * G + h) * 2) : -INFINITY;
-#pragma unroll
-      for (int j = 0; j < MB; ++j) M = fmaxf(M, mv[j]);
-    }
-    float Lsum = 0.f, O = 0.f;
+    // one pass: each round of MB partials raises the running max and rescales
+    // what was summed before (nothing when it is the first round)
+    float M = -INFINITY, Lsum = 0.f, O = 0.f;
 #pragma unroll 1
     for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
       float mv[MB], lv[MB], ov[MB];
@@ -641,6 +647,15 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
         lv[j] = in ? __ldcg(p.part_ml + slot * 2 + 1) : 0.f;
         ov[j] = in ? __ldcg(p.part_o + slot * D + dim) : 0.f;
       }
+      float Mn = M;
+#pragma unroll
+      for (int j = 0; j < MB; ++j) Mn = fmaxf(Mn, mv[j]);
+      if (s0 > 0) {
+        const float c = exp2f(M - Mn);
+        Lsum *= c;
+        O *= c;
+      }
+      M = Mn;
 #pragma unroll
       for (int j = 0; j < MB; ++j) {
         const float f = exp2f(mv[j] - M);
@@ -673,6 +688,7 @@ struct SmemBF16 {
   static constexpr int OFF_MISC = OFF_SCH + 40 * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+  static_assert(KROW_BF16 >= 2 * TT + G * 4, "a K~ row's padding holds the row's G masked queries");
 };
 
 template <int G>
@@ -720,26 +736,45 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   fence_proxy_async_smem();
   __syncthreads();
   const int n_tiles = has_work ? (int)(Sd.my_end - Sd.my_start) : 0;
-  // V tiles of the first stages are issued before the wait when they cannot
-  // hold this step's appended token (a unit's last tile holds it): nothing
-  // else the projection kernel writes is in them, and everything before it
-  // on the stream is complete once it has released this kernel.
-  uint32_t v_early = 0;
-  if (has_work && tid == NCT) {
-    const uint64_t pol = policy_evict_first();
+  // The first n_nat tiles (at most NSTAGE, all in the CTA's first unit, none
+  // its last tile, which holds this step's appended token) are loaded before
+  // the wait: V, and every kept K~ row in dimension order (the union list that
+  // picks rows is not known yet).  Nothing the projection kernel writes is in
+  // them, and everything before it on the stream is complete once it has
+  // released this kernel.  Their scores contract over all d_store dims with
+  // the masked queries in dimension order (zero for dims no head kept), which
+  // is the same sum as over the union rows.
+  int n_nat = 0;
+  {
     UnitWalker W0;
     W0.start<TT>(p, Sd, false);
-    for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
+    const int u_first = W0.u;
+    for (int it = 0; has_work && it < NSTAGE && it < n_tiles; ++it) {
       const long long t = Sd.my_start + it;
       W0.seek<TT>(p, Sd, t, false);
       const int t0 = (int)(t - W0.ts) * TT;
-      if (t0 + TT >= W0.Tb) break;
+      if (W0.u != u_first || t0 + TT >= W0.Tb) break;
+      ++n_nat;
+      if (warp < NCW) continue;
+      const int pt = tid - NCT;
+      const uint64_t pol = policy_evict_first();
       unsigned char* st = smem + (size_t)it * S::STAGE;
-      mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
-      const int row = W0.u * p.Tcap + t0;
-      tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
-      tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
-      v_early |= 1u << it;
+      if (pt == 0) {
+        mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
+        const int row = W0.u * p.Tcap + t0;
+        tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
+        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
+      }
+      const int chunk = pt & 15, r0 = pt >> 4;
+      const __nv_bfloat16* kbase =
+          static_cast<const __nv_bfloat16*>(p.kproj) + (size_t)W0.u * p.d_store * p.Tcap + t0 + chunk * 8;
+      unsigned char* ks = st + 2 * S::VHALF + chunk * 16;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int r = r0 + 8 * j;
+        if (r < p.d_store) cp_async16(ks + r * KROW_BF16, kbase + (size_t)r * p.Tcap, pol);
+      }
+      cp_async_arrive_noinc(&full[it]);
     }
   }
   pdl_launch_dependents();
@@ -765,7 +800,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
         const long long t = Sd.my_start + it;
         W0.seek<TT>(p, Sd, t);
-        if ((v_early >> it) & 1u) continue;
+        if (it < n_nat) continue;
         const StageHdr h0 = W0.header(Sd, t, TT);
         unsigned char* st = smem + (size_t)it * S::STAGE;
         mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
@@ -774,21 +809,27 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
       }
     }
-    int urow[16];
+    // union rows of the current unit and, loaded ahead, of the next one
+    const int n_units = p.B * p.Hkv;
+    int urow[16], unext[16];
+    int unext_u = W.u + 1;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int r = r0 + 8 * j;
       urow[j] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
+      unext[j] = unext_u < n_units ? p.ulist[(size_t)unext_u * D + r] : 0;
     }
     for (int it = 0; it < n_tiles; ++it) {
       const long long t = Sd.my_start + it;
       if (W.seek<TT>(p, Sd, t)) {
+        const bool ahead = W.u == unext_u;      // else empty units were skipped
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int r = r0 + 8 * j;
-          urow[j] = r < W.nU ? p.ulist[(size_t)W.u * D + r] : 0;
-        }
+        for (int j = 0; j < 16; ++j) urow[j] = ahead ? unext[j] : p.ulist[(size_t)W.u * D + r0 + 8 * j];
+        unext_u = W.u + 1;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) unext[j] = unext_u < n_units ? p.ulist[(size_t)unext_u * D + r0 + 8 * j] : 0;
       }
+      if (it < n_nat) continue;                 // loaded before the wait
       const int s = it % NSTAGE;
       if (it >= NSTAGE) {
         bool ok = true;
@@ -817,6 +858,14 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
           const int r = r0 + 8 * j;
           if (r < hh.nU) cp_async16(ks + r * KROW_BF16, kbase + (size_t)urow[j] * p.Tcap, pol);
         }
+      }
+      if ((hh.flags & kFirst) || (it == n_nat && n_nat > 0)) {
+        // the masked queries of union row r (G floats) ride in the padding
+        // after the row's TT keys; the consumers read them on a unit's first
+        // tile (and on the first tile after the dimension-order ones)
+        const int r = r0 + 8 * chunk;
+        if (r < hh.nU)
+          cp_async_small<G * 4>(st + 2 * S::VHALF + r * KROW_BF16 + 2 * TT, p.qm + ((size_t)hh.u * D + r) * G);
       }
       cp_async_arrive_noinc(&full[s]);
     }
@@ -863,11 +912,20 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     unsigned char* st = smem + (size_t)s * S::STAGE;
     const unsigned char* ks_base = st + 2 * S::VHALF;
 
-    if (!dead && (hh.flags & kFirst)) {
-      if (hh.u != cur_u) {
+    // A operand: the masked queries of the unit in the order of the tile's K~
+    // rows, dimension order on the tiles loaded before the wait, union order
+    // (from the rows' padding) from the first tile after them on
+    const bool nat0 = it == 0 && n_nat > 0;
+    const bool comp0 = it == n_nat && n_nat > 0;
+    if (!dead && ((hh.flags & kFirst) || comp0)) {
+      if (hh.u != cur_u || nat0 || comp0) {
         cur_u = hh.u;
-        nks = (hh.nU + 15) / 16;
-        const float* qmu = p.qm + (size_t)hh.u * D * G;
+        const int nrow = nat0 ? p.d_store : hh.nU;
+        nks = (nrow + 15) / 16;
+        // source of row col's query for head grp: dimension-order array or the row padding
+        const float* qsrc = nat0 ? p.qmn + (size_t)hh.u * D * G + grp
+                                 : reinterpret_cast<const float*>(ks_base + 2 * TT + grp * 4);
+        const int qstride = nat0 ? G : KROW_BF16 / 4;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
@@ -876,7 +934,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int col = kk * 16 + half * 8 + 2 * q4 + e;
-              const float x = (head_row && col < hh.nU) ? __ldg(qmu + (size_t)col * G + grp) : 0.f;
+              const float x = (head_row && col < nrow) ? qsrc[col * qstride] : 0.f;
               split_bf16(x, hi2[e], lo2[e]);
             }
             afr[kk][half * 2] = pack_bf16(hi2[0], hi2[1]);       // row grp
@@ -884,6 +942,8 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
           }
         }
       }
+    }
+    if (!dead && (hh.flags & kFirst)) {
       mu = -INFINITY;
       ell = 0.f;
 #pragma unroll
@@ -1445,6 +1505,7 @@ size_t decode_workspace_bytes(int n_units, int G) {
   auto take = [&](size_t bytes) { off += (bytes + 255) & ~size_t(255); };
   const size_t nseg = (size_t)n_units + kMaxCtas;
   take((size_t)n_units * D * G * 4);  // qm
+  take((size_t)n_units * D * G * 4);  // qmn
   take((size_t)n_units * D * 4);      // ulist
   take((size_t)n_units * 4);          // ucount
   take((size_t)n_units * 4);          // counters
@@ -1468,6 +1529,7 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   };
   const size_t nseg = (size_t)n_units + kMaxCtas;
   p.qm = static_cast<float*>(take((size_t)n_units * D * G * 4));
+  p.qmn = static_cast<float*>(take((size_t)n_units * D * G * 4));
   p.ulist = static_cast<int32_t*>(take((size_t)n_units * D * 4));
   p.ucount = static_cast<int32_t*>(take((size_t)n_units * 4));
   p.counters = static_cast<int32_t*>(take((size_t)n_units * 4));

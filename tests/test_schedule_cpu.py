@@ -1,7 +1,8 @@
 """The decode kernels' split of the tile sequence over CTAs, restated on the
 CPU.  Every non-empty unit (sequence, KV head) occupies W boundary positions
-followed by its tiles in a flat sequence of positions; CTAs split the positions
-evenly, so a CTA whose range crosses into a new unit (and pays a second
+followed by P positions per tile in a flat sequence of positions; CTAs split
+the positions evenly and own the tiles whose first position falls in their
+range, so a CTA whose range crosses into a new unit (and pays a second
 selection switch and segment merge) gets fewer tiles.  Checked here: the real
 tiles of every CTA are contiguous and cover every tile exactly once, the CTAs
 covering a unit are consecutive, the owner formula is right, and the partial
@@ -10,7 +11,8 @@ unit and below the workspace bound (the ticket-based combine relies on all of
 it)."""
 import random
 
-W = 4          # boundary positions per unit (kBoundaryTiles in csrc/decode.cu)
+P = 4          # positions per tile (kTilePos in csrc/decode.cu)
+W = 14         # boundary positions per unit (kBoundaryPos)
 
 
 def cta_of_pos(p, NV, C):
@@ -18,27 +20,28 @@ def cta_of_pos(p, NV, C):
     return min(c, C - 1)
 
 
-def split(tiles, grid, w=W):
-    """Real tile range [start, end) of every CTA, and the units' virtual starts."""
+def split(tiles, grid, w=W, pt=P):
+    """Real tile range [start, end) of every CTA, and the units' virtual starts.
+    Tile j of a unit starting at position vs occupies positions from
+    vs + w + j pt; a CTA owns the tiles whose first position is in its range."""
     vstart, vs = [], 0
     for nt in tiles:
         vstart.append(vs)
-        vs += nt + w if nt else 0
+        vs += nt * pt + w if nt else 0
     NV = vs
-    C = min(grid, NV)
+    C = max(1, min(grid, NV // pt))     # every CTA's range spans at least one tile's positions
     N = sum(tiles)
 
     def real_index(pos):
-        # first real tile at virtual position >= pos (N past the end)
+        # first real tile whose first position is >= pos (N past the end)
         r = 0
         for u, nt in enumerate(tiles):
             if nt == 0:
                 continue
             first = vstart[u] + w
-            if pos < first:
-                return r
-            if pos < first + nt:
-                return r + (pos - first)
+            for j in range(nt):
+                if first + j * pt >= pos:
+                    return r + j
             r += nt
         return N
 
@@ -46,11 +49,11 @@ def split(tiles, grid, w=W):
     return ranges, vstart, NV, C
 
 
-def _check(tiles, grid, w=W):
+def _check(tiles, grid, w=W, pt=P):
     N = sum(tiles)
     if N == 0:
         return
-    ranges, vstart, NV, C = split(tiles, grid, w)
+    ranges, vstart, NV, C = split(tiles, grid, w, pt)
     # the CTAs' real ranges tile [0, N) in order
     pos = 0
     for s, e in ranges:
@@ -62,13 +65,13 @@ def _check(tiles, grid, w=W):
     for u, nt in enumerate(tiles):
         if nt == 0:
             continue
-        first, last = vstart[u] + w, vstart[u] + w + nt - 1
+        first, last = vstart[u] + w, vstart[u] + w + (nt - 1) * pt
         cf, cl = cta_of_pos(first, NV, C), cta_of_pos(last, NV, C)
-        cover = [c for c, (s, e) in enumerate(ranges) if s < ts + nt and e > ts]
+        cover = [c for c, (s, e) in enumerate(ranges) if s < e and s < ts + nt and e > ts]   # CTAs owning tiles
         assert cover == list(range(cf, cl + 1))
         slots += [u + c for c in cover]                      # consecutive within the unit
         for j in range(nt):                                  # owner of every tile
-            s, e = ranges[cta_of_pos(first + j, NV, C)]
+            s, e = ranges[cta_of_pos(first + j * pt, NV, C)]
             assert s <= ts + j < e
         ts += nt
     assert len(set(slots)) == len(slots)                     # distinct across units
@@ -79,15 +82,15 @@ def test_schedule_random():
     rng = random.Random(0)
     for _ in range(4000):
         tiles = [rng.choice([0, 0, 1, 2, 3, 8, 65]) for _ in range(rng.randint(1, 12))]
-        _check(tiles, rng.randint(1, 160), w=rng.choice([0, 1, 3]))
+        _check(tiles, rng.randint(1, 160), w=rng.choice([0, 1, 3, 14]), pt=rng.choice([1, 2, 4]))
 
 
 def test_schedule_grid_larger_than_tiles():
-    for w in (0, W):
-        _check([8, 8, 1, 1, 0, 0, 5, 5], 64, w)
-        _check([1], 148, w)
-        _check([64] * 64, 148, w)
-        _check([1024] * 8, 148, w)
+    for w, pt in ((0, 1), (3, 1), (W, P)):
+        _check([8, 8, 1, 1, 0, 0, 5, 5], 64, w, pt)
+        _check([1], 148, w, pt)
+        _check([64] * 64, 148, w, pt)
+        _check([1024] * 8, 148, w, pt)
 
 
 def test_boundary_positions_balance_the_split():
