@@ -196,7 +196,7 @@ enum {
   BAR_Q = 0,     // raw query rows landed (TMA)
   BAR_PS,        // P parts written (256 softmax threads)
   BAR_QT,        // q~ = q P complete in TMEM (commit)
-  BAR_QM,        // masked q~ high/low parts written (128 threads of warpgroup 0)
+  BAR_QM,        // masked q~ high/low parts written (both softmax warpgroups, 256 threads)
   BAR_KF0,       // K~ buffer 0 / 1 full (TMA)
   BAR_KF1,
   BAR_KE0,       // K~ buffer 0 / 1 free (commit after the QK MMAs reading it)
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < BAR_COUNT; ++i) {
-      const int cnt = (i == BAR_PS || i == BAR_SF || i == BAR_P) ? kSoftThreads : (i == BAR_QM ? 128 : 1);
+      const int cnt = (i == BAR_PS || i == BAR_SF || i == BAR_P || i == BAR_QM) ? kSoftThreads : 1;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -440,74 +440,98 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&bars[BAR_PS]);
     }
 
-    // ---- prologue 2 (warpgroup 0): top-k of |q~| for this row, masked scaled q~ high/low parts
-    if (wg == 0) {
+    // ---- prologue 2: top-k of |q~| for row r, masked scaled q~ high/low parts.
+    // Warpgroup wg holds dims 64 wg .. 64 wg + 63 of the row; the row's two
+    // threads (warps w and w + 4 share TMEM lanes) exchange counts through
+    // shared memory (the P part-2 area, free once q~ is complete) at a barrier
+    // of their two warps.  Both take every round and exchange whatever their
+    // waits returned, so neither is ever left alone at the barrier.
+    {
       ok = wait_or_abort(&bars[BAR_QT], 0, abort_flag);
+      int* xcnt = reinterpret_cast<int*>(smem + S::OFF_PP);   // [2 rounds][2 halves][128 rows]
+      const int pair_bar = 2 + (warp & 3);
+      const int m = p.d_store;
+      const int d0 = 64 * wg;
+      uint32_t key[64];                             // |q~| bits + 1 for dims < m (0 otherwise): order-preserving
       if (ok) {
         tc_fence_after();
-        const int m = p.d_store;
-        uint32_t key[D];                              // |q~| bits + 1 for j < m (0 otherwise): order-preserving
-#pragma unroll
-        for (int c = 0; c < D; c += 32) tmem_ld32(tm_O + lane_base + c, *reinterpret_cast<float(*)[32]>(&key[c]));
+        tmem_ld32(tm_O + lane_base + d0, *reinterpret_cast<float(*)[32]>(&key[0]));
+        tmem_ld32(tm_O + lane_base + d0 + 32, *reinterpret_cast<float(*)[32]>(&key[32]));
         tmem_wait_ld();
+      }
 #pragma unroll
-        for (int j = 0; j < D; ++j) key[j] = (j < m) ? ((key[j] & 0x7fffffffu) + 1u) : 0u;
-        // largest tau with #{key >= tau} >= k, bit by bit; stop early once exactly k keys are >= tau
-        uint32_t tau = 0;
-        int cnt_tau = D;
+      for (int j = 0; j < 64; ++j) key[j] = (ok && d0 + j < m) ? ((key[j] & 0x7fffffffu) + 1u) : 0u;
+      // largest tau with #{key >= tau} >= k, bit by bit; stop early once exactly k keys are >= tau
+      uint32_t tau = 0;
+      int cnt_tau = D;
+      int round = 0;
 #pragma unroll 1
-        for (int bit = 30; bit >= 0; --bit) {
-          const uint32_t cand = tau | (1u << bit);
-          int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int bit = 30; bit >= 0; --bit, ++round) {
+        const uint32_t cand = tau | (1u << bit);
+        int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-          for (int j = 0; j < D; ++j) cp[j & 7] += (key[j] >= cand);
-          const int c = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
-          if (c >= p.k) {
-            tau = cand;
-            cnt_tau = c;
-          }
-          if (__all_sync(0xffffffffu, cnt_tau == p.k)) break;
+        for (int j = 0; j < 64; ++j) cp[j & 7] += (key[j] >= cand);
+        const int ch = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
+        int* xr = xcnt + (round & 1) * 256;
+        xr[wg * 128 + r] = ch;
+        named_bar_sync(pair_bar, 64);
+        const int c = ch + xr[(wg ^ 1) * 128 + r];
+        if (c >= p.k) {
+          tau = cand;
+          cnt_tau = c;
         }
-        // selected: every key above tau, then keys equal to tau from the lowest index up
-        uint32_t selm[4], eqm[4];
-        int need = p.k;
+        if (__all_sync(0xffffffffu, cnt_tau == p.k)) break;   // same decision in the partner warp
+      }
+      // selected: every key above tau, then keys equal to tau from the lowest index up
+      uint32_t selm[2], eqm[2];
+      int ngt = 0, neq = 0;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          uint32_t gt = 0u, eq = 0u;
+      for (int w = 0; w < 2; ++w) {
+        uint32_t gt = 0u, eq = 0u;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            gt |= (uint32_t)(key[32 * w + t] > tau) << t;
-            eq |= (uint32_t)(key[32 * w + t] == tau) << t;
-          }
-          selm[w] = gt;
-          eqm[w] = eq;
-          need -= __popc(gt);
+        for (int t = 0; t < 32; ++t) {
+          gt |= (uint32_t)(key[32 * w + t] > tau) << t;
+          eq |= (uint32_t)(key[32 * w + t] == tau) << t;
         }
+        selm[w] = gt;
+        eqm[w] = eq;
+        ngt += __popc(gt);
+        neq += __popc(eq);
+      }
+      int* xg = xcnt + 512;                         // [2 halves][128 rows]: above-tau count | equal count << 16
+      xg[wg * 128 + r] = ngt | (neq << 16);
+      named_bar_sync(pair_bar, 64);
+      const int other = xg[(wg ^ 1) * 128 + r];
+      const int ngt_lo = wg == 0 ? ngt : (other & 0xffff), neq_lo = wg == 0 ? neq : (other >> 16);
+      int need = p.k - ngt - (other & 0xffff);      // ties to keep, taken from the lower half first
+      const int ties_lo = min(need, neq_lo);
+      if (wg == 1) need -= ties_lo;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int ne = __popc(eqm[w]);
-          if (ne <= need) {
-            selm[w] |= eqm[w];
-            need -= ne;
-          } else if (need > 0) {
-            const uint32_t last = __fns(eqm[w], 0, need);   // position of the need-th tie in this word
-            selm[w] |= eqm[w] & (last >= 31 ? 0xffffffffu : ((2u << last) - 1u));
-            need = 0;
-          }
+      for (int w = 0; w < 2; ++w) {
+        const int ne = __popc(eqm[w]);
+        if (ne <= need) {
+          selm[w] |= eqm[w];
+          need -= ne;
+        } else if (need > 0) {
+          const uint32_t last = __fns(eqm[w], 0, need);   // position of the need-th tie in this word
+          selm[w] |= eqm[w] & (last >= 31 ? 0xffffffffu : ((2u << last) - 1u));
+          need = 0;
         }
-        const bool live = lr < l_end;
-        if (p.sel_out != nullptr && live) {
-          int32_t* so = p.sel_out + (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * p.k;
-          int n = 0;
+      }
+      const bool live = lr < l_end;
+      if (ok && p.sel_out != nullptr && live) {
+        int32_t* so = p.sel_out + (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * p.k;
+        int n = wg == 0 ? 0 : ngt_lo + ties_lo;      // the lower half's kept dims come first
 #pragma unroll
-          for (int w = 0; w < 4; ++w)
-            for (uint32_t word = selm[w]; word != 0u; word &= word - 1u) so[n++] = 32 * w + (__ffs(word) - 1);
-        }
-        // second pass over q~ (still in TMEM): masked, scaled, split, K-major swizzled rows
+        for (int w = 0; w < 2; ++w)
+          for (uint32_t word = selm[w]; word != 0u; word &= word - 1u) so[n++] = d0 + 32 * w + (__ffs(word) - 1);
+      }
+      if (ok) {
+        // second pass over this half of q~ (still in TMEM): masked, scaled, split, K-major swizzled rows
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
           float v[32];
-          tmem_ld32(tm_O + lane_base + c0, v);
+          tmem_ld32(tm_O + lane_base + d0 + c0, v);
           tmem_wait_ld();
           const uint32_t word = selm[c0 >> 5];
 #pragma unroll
@@ -523,7 +547,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               hw[e] = pack_hi_halves(h0, h1);
               lw[e] = pack_bf16(x0 - __uint_as_float(h0), x1 - __uint_as_float(h1));
             }
-            const int chunk = (c0 >> 3) + cc;         // 0..15
+            const int chunk = ((d0 + c0) >> 3) + cc;  // 0..15
             const int off = (chunk >> 3) * S::TILE + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
             *reinterpret_cast<uint4*>(smem + S::OFF_QH + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4*>(smem + S::OFF_QL + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
