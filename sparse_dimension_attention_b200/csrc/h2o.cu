@@ -30,7 +30,7 @@ __device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
   return a.score < b.score || (a.score == b.score && a.pos < b.pos);
 }
 
-constexpr int kTokPerThread = 8;   // tokens whose loads one thread issues together
+constexpr int kTokPerThread = 9;   // tokens whose loads one thread issues together (2304 per pass)
 
 template <typename T, int G>
 __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kproj, T* __restrict__ vcache,
@@ -44,6 +44,8 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   __shared__ int s_victim, s_vpos, is_last;
   const int u = blockIdx.x;
   const int b = u / Hkv, g = u % Hkv;
+  // launched as a dependent of the decode step: every input below is its output
+  pdl_wait();
   const int n = min(max(__ldcg(len + b), 0), Tcap);   // read before the ticket below
   const int newest = __ldcg(n_abs + b) - 1;
   const size_t ub = (size_t)u * Tcap;
@@ -56,6 +58,16 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   // exp(scores - lse); candidates are the slots outside the recent window.
   // A thread issues the loads of kTokPerThread slots before using any of
   // them: the kernel is bound by memory latency, not bandwidth.
+  // the last slot's key column and value row, read ahead of the arg-min:
+  // they move into the victim's slot if one is evicted
+  const int last = n - 1;
+  T* kp = kproj + (size_t)u * d_store * Tcap;
+  T* vp = vcache + ub * D;
+  T klast = T(0.f), vlast = T(0.f);
+  if (n > budget) {
+    if (threadIdx.x < d_store) klast = kp[(size_t)threadIdx.x * Tcap + last];
+    if (threadIdx.x < D) vlast = vp[(size_t)last * D + threadIdx.x];
+  }
   Cand best{INFINITY, 0, -1};
   for (int tb = threadIdx.x; tb < n; tb += kThreads * kTokPerThread) {
     float sv[kTokPerThread][G], scv[kTokPerThread];
@@ -108,13 +120,11 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   }
   __syncthreads();
   const int v = s_victim;
-  if (v >= 0 && v != n - 1) {
+  if (v >= 0 && v != last) {
     // move the last slot into the evicted one
-    const int last = n - 1;
-    T* kp = kproj + (size_t)u * d_store * Tcap;
-    for (int j = threadIdx.x; j < d_store; j += kThreads) kp[(size_t)j * Tcap + v] = kp[(size_t)j * Tcap + last];
-    T* vp = vcache + ub * D;
-    for (int j = threadIdx.x; j < D; j += kThreads) vp[(size_t)v * D + j] = vp[(size_t)last * D + j];
+    static_assert(kThreads >= D, "one thread per key dimension and value element");
+    if (threadIdx.x < d_store) kp[(size_t)threadIdx.x * Tcap + v] = klast;
+    if (threadIdx.x < D) vp[(size_t)v * D + threadIdx.x] = vlast;
     if (threadIdx.x == 0) {
       pos[ub + v] = pos[ub + last];
       score[ub + v] = score[ub + last];
@@ -142,17 +152,24 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
 }
 
 template <int G>
-void launch_h2o_g(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
+int launch_h2o_g(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
                   int32_t* evicted_out, int n_units, cudaStream_t st) {
+  // programmatic dependent launch: the grid is resident as the decode step's
+  // CTAs retire and starts the moment the step completes (it waits first)
+  cudaError_t e;
   if (c->dtype == AQUA_BF16) {
-    h2o_update_kernel<__nv_bfloat16, G><<<n_units, kThreads, 0, st>>>(
-        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos,
-        c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+    e = launch_pdl(h2o_update_kernel<__nv_bfloat16, G>, dim3(n_units), dim3(kThreads), 0, st,
+                   static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len,
+                   (const int32_t*)c->n_abs, c->pos, c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq,
+                   c->Hkv, c->d_store, c->Tcap, budget, recent);
   } else {
-    h2o_update_kernel<float, G><<<n_units, kThreads, 0, st>>>(
-        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl,
-        scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap, budget, recent);
+    e = launch_pdl(h2o_update_kernel<float, G>, dim3(n_units), dim3(kThreads), 0, st,
+                   static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, (const int32_t*)c->n_abs,
+                   c->pos, c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap,
+                   budget, recent);
   }
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "h2o_update_kernel: %s", cudaGetErrorString(e));
+  return AQUA_OK;
 }
 
 }  // namespace
@@ -160,12 +177,14 @@ void launch_h2o_g(aqua_cache* c, const float* scores, const float* lse, int Hq, 
 int launch_h2o_update(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
                       int32_t* evicted_out, cudaStream_t st) {
   const int n_units = c->B * c->Hkv;
+  int rc;
   switch (Hq / c->Hkv) {
-    case 1: launch_h2o_g<1>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
-    case 2: launch_h2o_g<2>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
-    case 4: launch_h2o_g<4>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    case 1: rc = launch_h2o_g<1>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    case 2: rc = launch_h2o_g<2>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
+    case 4: rc = launch_h2o_g<4>(c, scores, lse, Hq, budget, recent, evicted_out, n_units, st); break;
     default: return set_error(AQUA_ERR_UNSUPPORTED, "aqua_h2o_update: Hq/Hkv = %d not in {1,2,4}", Hq / c->Hkv);
   }
+  if (rc != AQUA_OK) return rc;
   return check_launch("h2o_update_kernel");
 }
 
