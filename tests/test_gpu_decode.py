@@ -252,3 +252,30 @@ def test_fused_append_equals_separate_append(kv):
     ref = O.decode(inp["q"][1], P64, oracle_cache(k_all, P64, kv), v_all.transpose(0, 2, 1, 3), [T + 2] * B, k)
     err = rel_err_rows(outs[1][1].numpy().astype(np.float64), ref["out"])
     assert np.max(err) <= (TOL_F32_OUT if kv == "f32" else TOL_F32_OUT_BF16_CACHE)
+
+
+@pytest.mark.parametrize("G,d_store,seed", [(4, None, 0), (2, 96, 1), (1, None, 2), (4, 64, 3)])
+def test_decode_bf16_mixed_lengths(G, d_store, seed):
+    """Per-sequence lengths from one token to several tiles (one exactly one
+    tile long): units of 1..6 tiles put CTA ranges, unit boundaries and the
+    tiles loaded before the dependency wait in every relative position; group
+    sizes 1/2/4 carry 4/8/16 bytes of masked queries per K~ row."""
+    rng = np.random.default_rng(seed)
+    B, Hkv = 8, 2
+    lens = [int(x) for x in rng.integers(1, 700, size=B)]
+    lens[int(rng.integers(0, B))] = 128
+    k = 48 if d_store == 64 else 80
+    cache, res, ref, _ = _decode_case(B, G * Hkv, Hkv, max(lens) - 1, k, lens=lens, d_store=d_store)
+    _check_outputs(res, ref, "bf16", lens)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], k, d_store)
+
+
+def test_decode_bf16_many_small_units():
+    """128 (sequence, KV head) units of 1..300 tokens: fewer positions than
+    four per CTA for some splits, so the active CTA count is capped; every CTA
+    between a unit's first and last tile owners must own one of its tiles."""
+    rng = np.random.default_rng(7)
+    B, Hkv = 64, 2
+    lens = [int(x) for x in rng.integers(1, 300, size=B)]
+    cache, res, ref, _ = _decode_case(B, 4 * Hkv, Hkv, max(lens) - 1, 64, lens=lens)
+    _check_outputs(res, ref, "bf16", lens)
