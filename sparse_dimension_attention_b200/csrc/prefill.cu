@@ -460,7 +460,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
       }
 #pragma unroll
-      for (int j = 0; j < 64; ++j) key[j] = (ok && d0 + j < m) ? ((key[j] & 0x7fffffffu) + 1u) : 0u;
+      for (int j = 0; j < 64; ++j)   // NaN payloads clamp to one key above inf, so every key is below 2^31
+        key[j] = (ok && d0 + j < m) ? (min(key[j] & 0x7fffffffu, 0x7F800001u) + 1u) : 0u;
       // largest tau with #{key >= tau} >= k, bit by bit; stop early once exactly k keys are >= tau
       uint32_t tau = 0;
       int cnt_tau = D;
@@ -468,10 +469,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
       for (int bit = 30; bit >= 0; --bit, ++round) {
         const uint32_t cand = tau | (1u << bit);
-        int cp[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        // keys below cand: key - cand wraps past 2^31 (both are below 2^31)
+        uint32_t cp[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int j = 0; j < 64; ++j) cp[j & 7] += (key[j] >= cand);
-        const int ch = ((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7]));
+        for (int j = 0; j < 64; ++j) cp[j & 7] += (key[j] - cand) >> 31;
+        const int ch = 64 - (int)(((cp[0] + cp[1]) + (cp[2] + cp[3])) + ((cp[4] + cp[5]) + (cp[6] + cp[7])));
         int* xr = xcnt + (round & 1) * 256;
         xr[wg * 128 + r] = ch;
         named_bar_sync(pair_bar, 64);
