@@ -147,3 +147,49 @@ def test_prefill_row_matches_decode():
         _check_sel(sd.cpu().numpy()[0], sel.cpu().numpy()[0, p], qt, k)
         err = rel_err_rows(od.cpu().numpy()[0].astype(np.float64), o.cpu().numpy()[0, p].astype(np.float64))
         assert np.max(err) <= 1e-4, (p, np.max(err))
+
+
+def test_prefill_adversarial_ties():
+    """Identity projection (q~ = q exactly) and rows whose magnitudes tie
+    across both 64-dim halves of the row: the k kept dims are every larger one
+    and the lowest-index tied ones, as in the oracle."""
+    Hq, Hkv, L, k = 4, 1, 16, 40
+    P32 = np.eye(128, dtype=np.float32)[None]
+    rng = np.random.default_rng(11)
+    q = np.zeros((1, L, Hq, 128), dtype=np.float32)
+    for i in range(L):
+        for h in range(Hq):
+            r = (i * Hq + h) % 4
+            if r == 0:
+                q[0, i, h] = rng.integers(-2, 3, 128)            # five magnitude levels, ties everywhere
+            elif r == 1:
+                q[0, i, h] = 1.0                                 # all tied: the lowest k dims
+            elif r == 2:
+                q[0, i, h, :30] = 5.0                            # 30 larger, then 11 ties at dims 60..70
+                q[0, i, h, 60:71] = -2.0                         # straddling dim 64: dims 60..69 kept
+            else:
+                q[0, i, h, 100:] = -2.0                          # larger dims in the upper half only
+                q[0, i, h, :100] = 1.0
+    q = synth.cast_bf16(q)
+    k_tok = synth.cast_bf16(rng.standard_normal((1, L, Hkv, 128)).astype(np.float32))
+    v_tok = synth.cast_bf16(rng.standard_normal((1, L, Hkv, 128)).astype(np.float32))
+    cache = aq.AquaCache(1, Hkv, 128)
+    Pt = fill_cache(cache, k_tok, v_tok, P32)
+    o = torch.empty((1, L, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((1, L, Hq, k), -1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(aq.aqua_prefill_workspace_size(cache.desc, Hq, L), dtype=torch.uint8, device="cuda")
+    aq.aqua_prefill_attn(cache.desc, tdev(q, torch.bfloat16), 0, L, Pt, Hq, k, o, ws, sel_out=sel)
+    torch.cuda.synchronize()
+    assert aq.aqua_status(cache.desc) == aq.AQUA_OK
+    sel = sel.cpu().numpy()
+    for i in range(L):
+        for h in range(Hq):
+            np.testing.assert_array_equal(sel[0, i, h], O.select_dims(q[0, i, h].astype(np.float64), k),
+                                          err_msg=f"row {i} head {h}")
+    assert list(sel[0, 0, 1]) == list(range(k))
+    assert list(sel[0, 0, 2]) == list(range(30)) + list(range(60, 70))
+    assert list(sel[0, 0, 3]) == list(range(12)) + list(range(100, 128))
+    P64 = P32.astype(np.float64)
+    Kt = O.build_key_cache(k_tok[0], P64, "bf16").transpose(1, 0, 2)
+    o_ref, _ = O.prefill(q[0], 0, P64, Kt, v_tok[0].transpose(1, 0, 2), k, out_dtype="bf16")
+    assert np.max(rel_err_rows(o.float().cpu().numpy()[0].astype(np.float64), o_ref)) <= TOL_BF16_OUT
