@@ -79,6 +79,7 @@ struct DecodeParams {
   float* score;
   int B, Hq, Hkv, d_store, Tcap, k;
   int len_add;            // 1 with a fused append: the step attends len[b] + 1 tokens
+  int n_late;             // attention CTAs (the last ones) expected to start after the projection kernel
   int out_bf16;
   float scale_log2;
 };
@@ -386,10 +387,53 @@ constexpr int kFirst = 1, kLast = 2;
 constexpr int kTilePos = 4;
 constexpr int kBoundaryPos = 14;
 
-// CTA whose range holds position p (positions split as above over C CTAs)
-__device__ __forceinline__ int cta_of_pos(long long p, long long NV, int C) {
-  long long c = ((p + 1) * C + NV - 1) / NV - 1;
+// The split is in two parts.  The last n_late CTAs (by index) start only when
+// the projection kernel's CTAs leave their SMs (measured ≈ 2.2 µs after the
+// others at the Llama decode shape; a sweep of 0..14 positions was fastest at
+// 10), so the first c0 = C - n_late CTAs share the first E positions,
+// E = c0 (NV + n_late kLatePos) / C, and the late ones share the rest; within
+// each part CTA c takes [floor(c N / C), floor((c+1) N / C)).
+constexpr int kLatePos = 10;
+
+struct Split {
+  long long NV, E;   // positions in all, positions of the early part
+  int C, c0;         // CTAs in all, early CTAs
+};
+
+__device__ __forceinline__ int cta_of_pos_even(long long p, long long N, int C) {
+  const long long c = ((p + 1) * C + N - 1) / N - 1;
   return (int)(c < C - 1 ? c : C - 1);
+}
+
+// CTA whose range holds position p
+__device__ __forceinline__ int cta_of_pos(long long p, const Split& sp) {
+  return p < sp.E ? cta_of_pos_even(p, sp.E, sp.c0) : sp.c0 + cta_of_pos_even(p - sp.E, sp.NV - sp.E, sp.C - sp.c0);
+}
+
+// first position of CTA c's range (c = C gives NV)
+__device__ __forceinline__ long long split_start(int c, const Split& sp) {
+  return c <= sp.c0 ? (long long)c * sp.E / sp.c0
+                    : sp.E + (long long)(c - sp.c0) * (sp.NV - sp.E) / (sp.C - sp.c0);
+}
+
+// Both parts keep at least kTilePos positions per CTA (every CTA between the
+// first and last owner of a unit's tiles then owns one of them: the merge
+// counts them); otherwise the split is even.
+__device__ __forceinline__ Split make_split(long long NV, int grid, int n_late) {
+  Split sp;
+  sp.NV = NV;
+  sp.C = (int)min((long long)grid, max(1LL, NV / kTilePos));
+  sp.c0 = sp.C;
+  sp.E = NV;
+  if (n_late > 0 && n_late < sp.C) {
+    const int c0 = sp.C - n_late;
+    const long long E = (long long)c0 * (NV + (long long)n_late * kLatePos) / sp.C;
+    if (E <= NV && E / c0 >= kTilePos && (NV - E) / n_late >= kTilePos) {
+      sp.c0 = c0;
+      sp.E = E;
+    }
+  }
+  return sp;
 }
 
 // exclusive scans of two values over all NT threads of the block at once;
@@ -442,6 +486,7 @@ __device__ __forceinline__ void block_excl_scan2(long long v0, long long v1, lon
 struct Sched {
   long long N, NV;             // tiles, positions
   long long my_start, my_end;  // this CTA's tiles (plain tile order)
+  const Split* sp;             // positions over CTAs (in shared memory; read at unit switches)
   int C;
   int u0;                      // unit of tile my_start
   long long ts0, sb0, vs0;     // its first tile, first partial slot and first position
@@ -458,7 +503,8 @@ __device__ __forceinline__ long long unit_tiles(const DecodeParams& p, int u) {
 // n_units + C - 1 (no scan over the segment counts is needed).
 //
 // This CTA's tiles and first unit.  Returns false (for the whole CTA) when the
-// CTA has no tile.  `scratch` needs 2 * NT / 32 long longs; sch[0..7] receive
+// CTA has no tile.  `scratch` needs 2 * NT / 32 long longs (sch + 8 .. sch + 31);
+// sch[0..7] and the split (sch + 32) receive
 // results.  All NT threads take part: one paired scan of the units' tile and
 // position counts, then the thread whose units hold this CTA's first and last
 // positions writes them to sch.
@@ -479,11 +525,12 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   long long excl[2], tot[2];
   block_excl_scan2<NT>(my_tiles, my_pos, scratch, excl, tot);
   const long long N = tot[0], NV = tot[1];
-  // at least kTilePos positions per CTA, so that every CTA between the first
-  // and last owner of a unit's tiles owns one of them (the merge counts them)
-  const int C = (int)min((long long)gridDim.x, max(1LL, NV / kTilePos));
+  const Split sp = make_split(NV, gridDim.x, p.n_late);
+  Split* sp_s = reinterpret_cast<Split*>(sch + 32);
+  if (tid == 0) *sp_s = sp;
+  const int C = sp.C;
   if (c >= C) return false;
-  const long long a = (long long)c * NV / C, e = (long long)(c + 1) * NV / C;   // this CTA's positions
+  const long long a = split_start(c, sp), e = split_start(c + 1, sp);   // this CTA's positions
   if (tid == 0 && e == NV) sch[1] = N;    // the last CTA's tiles run to the end
   {
     long long ts = excl[0], vs = excl[1];
@@ -495,7 +542,7 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
         sch[0] = ts + (a > first ? (a - first + kTilePos - 1) / kTilePos : 0);
         sch[2] = u;
         sch[3] = ts;
-        sch[4] = u + cta_of_pos(first, NV, C);
+        sch[4] = u + cta_of_pos(first, sp);
         sch[5] = vs;
       }
       if (vs <= e && e < end) sch[1] = ts + (e > first ? (e - first + kTilePos - 1) / kTilePos : 0);
@@ -506,6 +553,7 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   __syncthreads();
   S.N = N;
   S.NV = NV;
+  S.sp = sp_s;
   S.C = C;
   S.my_start = sch[0];
   S.my_end = sch[1];
@@ -536,8 +584,8 @@ struct UnitWalker {
     b = u / p.Hkv;
     Tb = kv_len(p, b);
     te = ts + (Tb + TT - 1) / TT;
-    cf = cta_of_pos(vs + kBoundaryPos, S.NV, S.C);
-    nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, S.NV, S.C) - cf + 1;
+    cf = cta_of_pos(vs + kBoundaryPos, *S.sp);
+    nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, *S.sp) - cf + 1;
     nU = with_nU ? p.ucount[u] : 0;
     preload(p, with_nU);
   }
@@ -555,8 +603,8 @@ struct UnitWalker {
       te = ts + (Tb + TT - 1) / TT;
       preload(p, with_nU);
       if (te > ts) {
-        cf = cta_of_pos(vs + kBoundaryPos, S.NV, S.C);
-        nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, S.NV, S.C) - cf + 1;
+        cf = cta_of_pos(vs + kBoundaryPos, *S.sp);
+        nseg = cta_of_pos(vs + kBoundaryPos + (te - ts - 1) * kTilePos, *S.sp) - cf + 1;
         sb = u + cf;
         nU = nU1;
       } else {
@@ -1550,6 +1598,9 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.v_new = v_new;
   p.len_w = c->len;
   p.len_add = (k_new != nullptr) ? 1 : 0;
+  // the projection kernel gives each of its CTAs an SM of its own when there
+  // are no more units than SMs; that many attention CTAs then start late
+  p.n_late = n_units <= device_sm_count() ? n_units : 0;
   p.n_abs = c->n_abs;
   p.pos = c->pos;
   p.score = c->score;

@@ -20,7 +20,35 @@ def cta_of_pos(p, NV, C):
     return min(c, C - 1)
 
 
-def split(tiles, grid, w=W, pt=P):
+LATE = 10      # kLatePos: positions fewer for each of the last n_late CTAs
+
+
+def make_split(NV, grid, pt, n_late, late):
+    """(C, c0, E): C CTAs, the first c0 share positions [0, E), the rest [E, NV)."""
+    C = max(1, min(grid, NV // pt))     # every CTA's range spans at least one tile's positions
+    c0, E = C, NV
+    if 0 < n_late < C:
+        c = C - n_late
+        e = c * (NV + n_late * late) // C
+        if e <= NV and e // c >= pt and (NV - e) // n_late >= pt:
+            c0, E = c, e
+    return C, c0, E
+
+
+def split_start(c, NV, C, c0, E):
+    return c * E // c0 if c <= c0 else E + (c - c0) * (NV - E) // (C - c0)
+
+
+def cta_of_pos_even(p, N, C):
+    c = ((p + 1) * C + N - 1) // N - 1
+    return min(c, C - 1)
+
+
+def cta_of_pos2(p, NV, C, c0, E):
+    return cta_of_pos_even(p, E, c0) if p < E else c0 + cta_of_pos_even(p - E, NV - E, C - c0)
+
+
+def split(tiles, grid, w=W, pt=P, n_late=0, late=LATE, full=False):
     """Real tile range [start, end) of every CTA, and the units' virtual starts.
     Tile j of a unit starting at position vs occupies positions from
     vs + w + j pt; a CTA owns the tiles whose first position is in its range."""
@@ -29,7 +57,7 @@ def split(tiles, grid, w=W, pt=P):
         vstart.append(vs)
         vs += nt * pt + w if nt else 0
     NV = vs
-    C = max(1, min(grid, NV // pt))     # every CTA's range spans at least one tile's positions
+    C, c0, E = make_split(NV, grid, pt, n_late, late)
     N = sum(tiles)
 
     def real_index(pos):
@@ -45,15 +73,22 @@ def split(tiles, grid, w=W, pt=P):
             r += nt
         return N
 
-    ranges = [(real_index(c * NV // C), real_index((c + 1) * NV // C)) for c in range(C)]
+    ranges = [(real_index(split_start(c, NV, C, c0, E)), real_index(split_start(c + 1, NV, C, c0, E)))
+              for c in range(C)]
+    if full:
+        return ranges, vstart, NV, C, c0, E
     return ranges, vstart, NV, C
 
 
-def _check(tiles, grid, w=W, pt=P):
+def _check(tiles, grid, w=W, pt=P, n_late=0, late=LATE):
     N = sum(tiles)
     if N == 0:
         return
-    ranges, vstart, NV, C = split(tiles, grid, w, pt)
+    ranges, vstart, NV, C, c0, E = split(tiles, grid, w, pt, n_late, late, full=True)
+
+    def cta_of_pos(p, NV_, C_):
+        return cta_of_pos2(p, NV_, C_, c0, E)
+
     # the CTAs' real ranges tile [0, N) in order
     pos = 0
     for s, e in ranges:
@@ -82,15 +117,31 @@ def test_schedule_random():
     rng = random.Random(0)
     for _ in range(4000):
         tiles = [rng.choice([0, 0, 1, 2, 3, 8, 65]) for _ in range(rng.randint(1, 12))]
-        _check(tiles, rng.randint(1, 160), w=rng.choice([0, 1, 3, 14]), pt=rng.choice([1, 2, 4]))
+        _check(tiles, rng.randint(1, 160), w=rng.choice([0, 1, 3, 14]), pt=rng.choice([1, 2, 4]),
+               n_late=rng.choice([0, 0, 1, 5, 64, 200]), late=rng.choice([0, 3, 7, 20]))
 
 
 def test_schedule_grid_larger_than_tiles():
     for w, pt in ((0, 1), (3, 1), (W, P)):
-        _check([8, 8, 1, 1, 0, 0, 5, 5], 64, w, pt)
-        _check([1], 148, w, pt)
-        _check([64] * 64, 148, w, pt)
-        _check([1024] * 8, 148, w, pt)
+        for n_late in (0, 8, 64):
+            _check([8, 8, 1, 1, 0, 0, 5, 5], 64, w, pt, n_late)
+            _check([1], 148, w, pt, n_late)
+            _check([64] * 64, 148, w, pt, n_late)
+            _check([1024] * 8, 148, w, pt, n_late)
+
+
+def test_late_ctas_get_fewer_positions():
+    """At the Llama decode shape the 64 CTAs that start behind the projection
+    kernel's CTAs get about kLatePos fewer positions than the other 84."""
+    tiles = [65] * 64
+    NV = 64 * (65 * P + W)
+    C, c0, E = make_split(NV, 148, P, 64, LATE)
+    assert (C, c0) == (148, 84)
+    early = [split_start(c + 1, NV, C, c0, E) - split_start(c, NV, C, c0, E) for c in range(c0)]
+    late = [split_start(c + 1, NV, C, c0, E) - split_start(c, NV, C, c0, E) for c in range(c0, C)]
+    assert abs(sum(early) / len(early) - sum(late) / len(late) - LATE) < 1.0
+    ranges, _, _, _ = split(tiles, 148, n_late=64)
+    assert sum(e - s for s, e in ranges) == sum(tiles)
 
 
 def test_boundary_positions_balance_the_split():
