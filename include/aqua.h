@@ -138,6 +138,10 @@ AQUA_API int aqua_calibrate(const float* X, int n, int d, float* P_out, float* s
  * cache->max_len += L on the host.
  *   k_new, v_new  [B][L][Hkv][d]  cache dtype
  *   P             [Hkv][d][d]     f32, q~ = q P (row vector times P)
+ * k_new, v_new and P are read before the call waits for the preceding kernel
+ * on the stream (the lengths and the cache only after it), which is safe
+ * unless the kernel that wrote them released its dependents early through
+ * programmatic dependent launch (no kernel here that writes them does).
  * Errors: AQUA_ERR_ARG if cache->max_len + L > Tcap or L < 1.
  */
 AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void* v_new, const float* P,

@@ -29,22 +29,23 @@ __device__ __forceinline__ void load4(const __nv_bfloat16* p, float (&f)[4]) {
   f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
 }
 
-template <typename T>
-__device__ __forceinline__ void copy4(T* dst, const T* src);
-template <>
-__device__ __forceinline__ void copy4(float* dst, const float* src) {
-  *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(src);
-}
-template <>
-__device__ __forceinline__ void copy4(__nv_bfloat16* dst, const __nv_bfloat16* src) {
-  *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
-}
+// four consecutive elements as one vector (16 bytes of f32, 8 of bf16)
+template <typename T> struct Vec4;
+template <> struct Vec4<float> { using type = float4; };
+template <> struct Vec4<__nv_bfloat16> { using type = uint2; };
 
 // grid (ceil(L/32), Hkv, B), block 256: P[g] is staged in shared memory by one
 // bulk copy; warp w projects tokens blockIdx.x*32 + 4w .. 4w+3 of (b, g) with
 // one pass over P, the projected keys are staged as a [dim][32 token] tile and
 // written out as runs of 32 consecutive slots per dimension row (the cache is
 // dimension-major), values are copied token-major.
+//
+// Launched as a programmatic dependent of the previous kernel: everything up to
+// the projection reads only P and the new keys and values, so it runs while the
+// previous kernel (an attention kernel of the previous chunk or step, which
+// never writes them) finishes; the lengths are read, and the cache written,
+// after the wait.  The slots written lie at or past the lengths, which no
+// earlier kernel of the stream still reads.
 template <typename T>
 __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__ k_new,
                                                            const T* __restrict__ v_new,
@@ -53,6 +54,7 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
                                                            int32_t* len, int32_t* n_abs, int32_t* pos,
                                                            float* score, int32_t* ctrl, int B, int L,
                                                            int Hkv, int d_store, int Tcap) {
+  using V4 = typename Vec4<T>::type;
   extern __shared__ __align__(128) float Ps[];              // [D][D]
   __shared__ __align__(16) float xs[kWarps][kTokPerWarp][D];  // the warp's key rows
   __shared__ T kt[D][kTokPerCta];                           // projected keys, dimension-major
@@ -60,14 +62,9 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
   __shared__ int is_last;
   const int g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Lengths are read before this CTA takes its ticket below; the last CTA
-  // advances them only after every CTA has taken one.
-  const int base = __ldcg(len + b);
-  const int abase = n_abs ? __ldcg(n_abs + b) : base;
   const int l0 = blockIdx.x * kTokPerCta;
   const int ntok = min(kTokPerCta, L - l0);
   const size_t unit = (size_t)b * Hkv + g;
-  const bool in_range = base >= 0 && base + l0 + ntok <= Tcap;
   if (threadIdx.x == 0) {
     mbar_init(&pbar, 1);
     fence_barrier_init();
@@ -77,7 +74,8 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     mbar_arrive_expect_tx(&pbar, D * D * 4);
     bulk_g2s_plain(Ps, P + (size_t)g * D * D, D * D * 4, &pbar);
   }
-  // key rows of this warp's tokens (zeros past the chunk), values copied meanwhile
+  // key rows of this warp's tokens (zeros past the chunk); value rows held in registers
+  V4 vrow[kTokPerWarp];
 #pragma unroll
   for (int t = 0; t < kTokPerWarp; ++t) {
     const int l = warp * kTokPerWarp + t;
@@ -85,14 +83,7 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     if (l < ntok) {
       const size_t row = ((size_t)b * L + l0 + l) * Hkv + g;
       load4<T>(k_new + row * D + 4 * lane, kv);
-      if (in_range) {
-        const int slot = base + l0 + l;
-        copy4<T>(vcache + (unit * Tcap + slot) * D + 4 * lane, v_new + row * D + 4 * lane);
-        if (pos != nullptr && lane == 0) {
-          pos[unit * Tcap + slot] = abase + l0 + l;
-          score[unit * Tcap + slot] = 0.f;
-        }
-      }
+      vrow[t] = *reinterpret_cast<const V4*>(v_new + row * D + 4 * lane);
     }
     *reinterpret_cast<float4*>(&xs[warp][t][4 * lane]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
   }
@@ -100,15 +91,35 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
   const bool ok = mbar_wait_bounded(&pbar, 0);
   const bool bad = __syncthreads_or(!ok);
   if (bad && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_TIMEOUT);
-  if (!in_range && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity
-  if (!bad && in_range) {
+  if (!bad) {
     float y[kTokPerWarp][4];
     project_rows_smem<kTokPerWarp>(Ps, &xs[warp][0][0], lane, y);
 #pragma unroll
     for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
       for (int s = 0; s < 4; ++s) kt[4 * lane + s][warp * kTokPerWarp + t] = Elem<T>::from_f32(y[t][s]);
-    __syncthreads();
+  }
+  pdl_wait();
+  // Lengths are read before this CTA takes its ticket below; the last CTA
+  // advances them only after every CTA has taken one.
+  const int base = __ldcg(len + b);
+  const int abase = n_abs ? __ldcg(n_abs + b) : base;
+  const bool in_range = base >= 0 && base + l0 + ntok <= Tcap;
+  if (!in_range && threadIdx.x == 0) record_status(ctrl, AQUA_ERR_ARG);   // device length beyond capacity
+  __syncthreads();                                          // kt complete
+  if (!bad && in_range) {
+#pragma unroll
+    for (int t = 0; t < kTokPerWarp; ++t) {
+      const int l = warp * kTokPerWarp + t;
+      if (l < ntok) {
+        const int slot = base + l0 + l;
+        *reinterpret_cast<V4*>(vcache + (unit * Tcap + slot) * D + 4 * lane) = vrow[t];
+        if (pos != nullptr && lane == 0) {
+          pos[unit * Tcap + slot] = abase + l0 + l;
+          score[unit * Tcap + slot] = 0.f;
+        }
+      }
+    }
     // dimension row jd, tokens 0..ntok-1 -> slots base+l0 .. : one warp per row, one lane per token
     T* kp = kproj + unit * d_store * (size_t)Tcap + base + l0;
     for (int jd = warp; jd < d_store; jd += kWarps)
@@ -145,10 +156,12 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
         return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
       configured = true;
     }
-    project_keys_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), P,
-        static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs,
-        c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+    const cudaError_t e = launch_pdl(
+        project_keys_kernel<__nv_bfloat16>, grid, dim3(256), smem, st, static_cast<const __nv_bfloat16*>(k_new),
+        static_cast<const __nv_bfloat16*>(v_new), P, static_cast<__nv_bfloat16*>(c->k_proj),
+        static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store,
+        c->Tcap);
+    if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "project_keys_kernel: %s", cudaGetErrorString(e));
   } else {
     static bool configured = false;
     if (!configured) {
@@ -157,10 +170,11 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
         return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
       configured = true;
     }
-    project_keys_kernel<float><<<grid, 256, smem, st>>>(
-        static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
-        static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs, c->pos, c->score,
-        c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+    const cudaError_t e = launch_pdl(project_keys_kernel<float>, grid, dim3(256), smem, st,
+                                     static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
+                                     static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs,
+                                     c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+    if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "project_keys_kernel: %s", cudaGetErrorString(e));
   }
   return check_launch("project_keys_kernel");
 }
