@@ -1,10 +1,11 @@
 // AQUA decode step on sm_100a.
 //
-// qproj_topk_kernel -- one CTA per (sequence b, KV head g), one warp per query
-// head of the group (P[g] staged in shared memory by one bulk copy), plus one
+// qproj_topk_kernel -- one CTA per (sequence b, KV head g): four warps per
+// query head of the group project row slices of every head and then rank the
+// head's dimensions (P[g] staged in shared memory by bulk copies), plus one
 // warp that appends the step's new key and value when the call carries them
-// (k~ = k P rounded to the cache type, written at slot len[b]; the last CTA
-// advances the lengths):
+// (k~ = k P rounded to the cache type, written at slot len[b]; the attention
+// kernel's last CTA advances the lengths):
 //   q~ = q P                                  (abstract: "project query and key vectors")
 //   S_h = k largest |q~_j|, ties to lower j  (edgentiq, Online Inference: the dimensions
 //                                             with the highest "magnitude" in the projected query)
@@ -13,7 +14,7 @@
 //
 // decode_attn_*_kernel -- persistent, one CTA per SM.  The cached tokens of all
 // (b, g) units are cut into tiles of TT tokens and the flat tile sequence is
-// split evenly over the CTAs.  Per tile a producer warp gathers the |U_g|
+// split over the CTAs by a position model (see kTilePos).  Per tile the producer warps gather the |U_g|
 // selected rows of the dimension-major K~ cache (one union read per GQA group)
 // and the V tile into shared memory with asynchronous bulk / tensor copies,
 // three stages deep.  Consumer warps compute the scores on the selected
