@@ -279,3 +279,14 @@ def test_decode_bf16_many_small_units():
     lens = [int(x) for x in rng.integers(1, 300, size=B)]
     cache, res, ref, _ = _decode_case(B, 4 * Hkv, Hkv, max(lens) - 1, 64, lens=lens)
     _check_outputs(res, ref, "bf16", lens)
+
+
+def test_decode_bf16_more_units_than_sms():
+    """160 (sequence, KV head) units, more than the GPU's SMs: the selection
+    kernel shares SMs and the attention split is even (no late part)."""
+    rng = np.random.default_rng(9)
+    B, Hkv = 80, 2
+    lens = [int(x) for x in rng.integers(1, 260, size=B)]
+    cache, res, ref, _ = _decode_case(B, 2 * Hkv, Hkv, max(lens) - 1, 48, lens=lens)
+    _check_outputs(res, ref, "bf16", lens)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 48)
