@@ -210,7 +210,9 @@ def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: flo
 
 # ----------------------------------------------------------------------------- AQUA arm
 class DecodeBench:
-    def __init__(self, wl: dict, steps: int, warmup: int, seed_steps: int | None = None):
+    def __init__(self, wl: dict, steps: int, warmup: int, seed_steps: int | None = None, P=None):
+        """P: optional projection [Hkv, d, d] (f32, on the device); by default the
+        offline step computes it from the calibration matrix on the GPU."""
         import torch
         import sparse_dimension_attention_b200 as aq
         from sparse_dimension_attention_b200 import build
@@ -222,13 +224,16 @@ class DecodeBench:
         self.esize = 2 if kv == "bf16" else 4
         n_steps = max(steps, warmup, 1) + 1
         self.n_in = n_steps
-        # offline step: P from the calibration matrix, on the GPU
-        X = torch.from_numpy(synth.calibration_matrix()).cuda()
-        P1 = torch.empty((128, 128), dtype=torch.float32, device="cuda")
-        sig = torch.empty((128,), dtype=torch.float32, device="cuda")
-        ws = torch.empty(aq.aqua_calibrate_workspace_size(X.shape[0], 128), dtype=torch.uint8, device="cuda")
-        aq.aqua_calibrate(X, P1, sig, ws)
-        self.P = P1.unsqueeze(0).expand(Hkv, 128, 128).contiguous()
+        if P is not None:
+            self.P = P[:Hkv].contiguous()
+        else:
+            # offline step: P from the calibration matrix, on the GPU
+            X = torch.from_numpy(synth.calibration_matrix()).cuda()
+            P1 = torch.empty((128, 128), dtype=torch.float32, device="cuda")
+            sig = torch.empty((128,), dtype=torch.float32, device="cuda")
+            ws = torch.empty(aq.aqua_calibrate_workspace_size(X.shape[0], 128), dtype=torch.uint8, device="cuda")
+            aq.aqua_calibrate(X, P1, sig, ws)
+            self.P = P1.unsqueeze(0).expand(Hkv, 128, 128).contiguous()
         # history of T-1 tokens so the first step attends T
         inp = synth.decode_inputs(B, Hq, Hkv, T - 1, bf16=(kv == "bf16"), steps=n_steps)
         self.T0 = T - 1
