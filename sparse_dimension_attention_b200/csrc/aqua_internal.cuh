@@ -290,6 +290,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// named barrier that also counts the participating threads whose predicate is true
+__device__ __forceinline__ int named_bar_popc(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.popc.u32 %0, %2, %3, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return (int)r;
+}
+
 // named barrier that also ORs a predicate over the participating threads
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
   uint32_t r;

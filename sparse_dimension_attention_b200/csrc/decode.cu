@@ -151,10 +151,9 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
   extern __shared__ __align__(128) float Ps[];   // P[g], [D][D]
   __shared__ __align__(16) float qs[G][D];       // q rows, later the kept scaled q~
   __shared__ __align__(16) float part[NPW][G][D];
-  __shared__ __align__(16) uint32_t keys[G][D];
   __shared__ __align__(16) float knew_s[D];
   __shared__ uint32_t masks[G][NWQ];
-  __shared__ int nkeep[G][NWQ];
+  __shared__ int neq[G][NWQ];
   __shared__ __align__(8) uint64_t pbars[kPChunks];
   __shared__ int s_abort;
   const int u = blockIdx.x;
@@ -288,34 +287,35 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(Dec
 #pragma unroll
   for (int x = 1; x < NPW; ++x) qt += part[x][hw][i];
   const uint32_t ki = i < m ? min(__float_as_uint(fabsf(qt)), 0x7F800001u) + 1u : 0u;   // NaN above inf
-  keys[hw][i] = ki;
-  named_bar_sync(1, NPT);
-  // Keys are below 2^31, so key_j > key_i exactly when key_i - key_j wraps
-  // around, i.e. has its top bit set: one subtraction and one shifted add each.
-  uint32_t gt = 0;
-  const uint4* kv = reinterpret_cast<const uint4*>(keys[hw]);
-#pragma unroll 8
-  for (int j4 = 0; j4 < D / 4; ++j4) {
-    const uint4 kj = kv[j4];
-    gt += ((ki - kj.x) >> 31) + ((ki - kj.y) >> 31) + ((ki - kj.z) >> 31) + ((ki - kj.w) >> 31);
-  }
-  // Equal keys share gt, so exactly k candidates have gt < k unless a group of
-  // equal keys straddles the cut; only then is the index order needed.
-  bool keep = i < m && (int)gt < p.k;
-  uint32_t bal = __ballot_sync(0xffffffffu, keep);
-  if (lane == 0) nkeep[hw][sl] = __popc(bal);
-  named_bar_sync(1, NPT);
-  int tot = 0;
-#pragma unroll
-  for (int x = 0; x < NWQ; ++x) tot += nkeep[hw][x];
-  if (tot > p.k) {                              // uniform over the head's warps
-    if (keep) {
-      int eq_lo = 0;
-      for (int j = 0; j < i; ++j) eq_lo += keys[hw][j] == ki;
-      keep = (int)gt + eq_lo < p.k;
+  // tau = the largest value with #{key >= tau} >= k over the head's 128 keys
+  // (its four warps, one key per thread), one bit per round from the top (keys
+  // are below 2^31), each count one barrier reduction over the four warps; the
+  // search stops once exactly k keys are >= tau.
+  const int hbar = 2 + hw;                      // named barrier of the head's warps
+  uint32_t tau = 0;
+  int cnt = D;
+#pragma unroll 1
+  for (int bit = 30; bit >= 0 && cnt != p.k; --bit) {   // cnt is uniform over the head's warps
+    const uint32_t cand = tau | (1u << bit);
+    const int c = named_bar_popc(hbar, NWQ * 32, ki >= cand);
+    if (c >= p.k) {
+      tau = cand;
+      cnt = c;
     }
-    bal = __ballot_sync(0xffffffffu, keep);
   }
+  bool keep = i < m && ki >= tau;
+  if (cnt > p.k) {
+    // equal keys straddle the cut: every key above tau, then keys equal to tau
+    // from the lowest index up
+    const int ngt = named_bar_popc(hbar, NWQ * 32, ki > tau);
+    const uint32_t eqb = __ballot_sync(0xffffffffu, ki == tau);
+    if (lane == 0) neq[hw][sl] = __popc(eqb);
+    named_bar_sync(hbar, NWQ * 32);
+    int before = __popc(eqb & ((1u << lane) - 1u));
+    for (int x = 0; x < sl; ++x) before += neq[hw][x];
+    keep = i < m && (ki > tau || (ki == tau && before < p.k - ngt));
+  }
+  const uint32_t bal = __ballot_sync(0xffffffffu, keep);
   if (lane == 0) masks[hw][sl] = bal;
   if (p.qproj_out) p.qproj_out[bh * D + i] = qt;
   qs[hw][i] = keep ? qt * p.scale_log2 : 0.f;
