@@ -210,7 +210,7 @@ def whole_job_rate(units_per_rank_step: int, steps: int, world: int, max_ms: flo
 
 # ----------------------------------------------------------------------------- AQUA arm
 class DecodeBench:
-    def __init__(self, wl: dict, steps: int, warmup: int, seed_steps: int | None = None, P=None):
+    def __init__(self, wl: dict, steps: int, warmup: int, P=None):
         """P: optional projection [Hkv, d, d] (f32, on the device); by default the
         offline step computes it from the calibration matrix on the GPU."""
         import torch
