@@ -140,8 +140,10 @@ struct QprojCfg {
 };
 constexpr int kPChunks = 4;   // P[g] staged as four 32-row chunks, each with its own barrier
 
-template <typename T, int G>
-__global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32) qproj_topk_kernel(DecodeParams p) {
+// MINB = 2 caps the registers so that two CTAs share an SM (used when the
+// units outnumber the SMs, which would otherwise run in two waves).
+template <typename T, int G, int MINB>
+__global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kernel(DecodeParams p) {
   constexpr int NWQ = QprojCfg<G>::NWQ, NPW = QprojCfg<G>::NPW;
   constexpr int NPT = NPW * 32;                 // threads of the projection/selection warps
   constexpr int RW = D / NPW;                   // input dims per projection warp
@@ -1482,22 +1484,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 // ============================================================================
 // host launch
 // ============================================================================
+template <typename T, int G, int MINB>
+cudaError_t launch_qproj_variant(const DecodeParams& p, int n_units, int smem, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(qproj_topk_kernel<T, G, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  return launch_pdl(qproj_topk_kernel<T, G, MINB>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), smem, st, p);
+}
+
 template <typename T, int G>
 int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
   // With no more units than SMs, the dynamic shared memory request is raised
   // above half an SM's so that every CTA gets an SM of its own: the kernel is
   // latency-bound, and CTAs sharing an SM were measured to take twice as long.
+  // With more units, two CTAs share each SM (registers capped to fit), rather
+  // than a second wave.
   constexpr int kOwnSm = 116 * 1024;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(qproj_topk_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOwnSm) !=
-        cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(qproj_topk_kernel)");
-    configured = true;
-  }
-  const int smem = n_units <= device_sm_count() ? kOwnSm : D * D * 4;
-  const cudaError_t e =
-      launch_pdl(qproj_topk_kernel<T, G>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), smem, st, p);
+  const cudaError_t e = n_units <= device_sm_count()
+                            ? launch_qproj_variant<T, G, 1>(p, n_units, kOwnSm, st)
+                            : launch_qproj_variant<T, G, 2>(p, n_units, D * D * 4, st);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
   return check_launch("qproj_topk_kernel");
 }
