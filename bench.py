@@ -47,6 +47,11 @@ PREFILL = dict(B=1, Hq=32, Hkv=8, L_total=4096, chunk=512, k=96)
 # truncated cache (first m projected dims stored), k within them, H2O budget of
 # `recent` newest + heavy hitters; absolute length runs from `budget` to T_end
 H2O_WL = dict(B=32, Hq=32, Hkv=8, m=96, k=64, budget=2048, recent=256, T_end=32768)
+# break-even sweep over the context length and k at the Llama decode shape (one
+# cache built at the largest T; shorter contexts rewind the lengths)
+T_SWEEP = dict(B=8, Hq=32, Hkv=8, kv="bf16", d_store=128, Ts=(512, 1024, 2048, 4096, 8192, 16384, 32768),
+               ks=(128, 96, 64, 32))
+L2_BYTES = 126e6
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -644,6 +649,41 @@ class H2OBench:
                 "l2": "no flush: each step streams %.0f MB, above the 126 MB L2" % (by / 1e6)}
 
 
+def t_sweep(P, K: int, W: int, world: int) -> dict:
+    """Decode step time over context lengths T and selection sizes k at the
+    Llama decode shape, against k = d at the same T (the same kernels: at k = d
+    the selection keeps every dimension, so the comparison isolates what the
+    smaller union saves against the fixed per-step costs).  Also the pages'
+    flop break-even T* = d^2 (1 + 1/G) / (d - k) of AQUA against dense attention
+    per query head, for reference."""
+    tw = dict(T_SWEEP)
+    Ts, ks = tw.pop("Ts"), tw.pop("ks")
+    wl = dict(tw, T=max(Ts), k=ks[0])
+    tb = DecodeBench(wl, K, W, P=P)
+    unions = {kk: tb.union_sizes(kk, min(K, 8)) for kk in ks}
+    G, d = wl["Hq"] // wl["Hkv"], 128
+    rows = []
+    for T in Ts:
+        tb.T0 = T - 1
+        dense_us = None
+        for kk in ks:
+            t_ms, d_ms, _ = tb.timed(K, W, kk, world, clocks=False)
+            t_ms = max_over_ranks(t_ms, world)
+            u = unions[kk]
+            by = [tb.bytes_decode(u[s % u.shape[0]], T + s) + tb.bytes_append() for s in range(K)]
+            us = 1e3 * t_ms / K
+            dense_us = us if kk == d else dense_us
+            rows.append({"T": T, "k": kk, "decode_us": us, "mean_union": float(u.mean()),
+                         "decode_gbs": sum(by) / (t_ms / 1e3) / 1e9,
+                         "speedup_vs_k_d": (dense_us / us) if dense_us else None,
+                         "l2_resident": by[0] < L2_BYTES})
+    del tb
+    return {"workload": "llama3.1-8b-decode T x k sweep", "B": wl["B"], "Hq": wl["Hq"], "Hkv": wl["Hkv"],
+            "rows": rows, "launch": "K steps in one CUDA graph per (T, k)",
+            "flop_breakeven_T": {str(kk): d * d * (1 + 1 / G) / (d - kk) for kk in ks if kk < d},
+            "note": "l2_resident: a step's algorithmic bytes fit in the 126 MB L2 (no flush between steps)"}
+
+
 def cpu_baseline(wl: dict, budget_s: float = 12.0) -> dict:
     """The oracle, as it stands, on the host cores: decode steps of one sequence
     (all its query heads) repeated until about budget_s seconds have run."""
@@ -726,7 +766,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="only the main decode line")
     ap.add_argument("--extras", default="sweep,long,prefill,h2o",
                     help="comma list of extra lines: sweep (k sweep), long (long context), prefill (chunked "
-                         "prefill), h2o (truncated cache + H2O steady state)")
+                         "prefill), h2o (truncated cache + H2O steady state); tsweep (break-even sweep over "
+                         "T and k, not in the default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -804,6 +845,9 @@ def main():
     P = bench.P
     del bench
     torch.cuda.empty_cache()
+    if "tsweep" in extras:
+        line["t_sweep"] = t_sweep(P, min(K, 50), W, world)
+        torch.cuda.empty_cache()
     if "long" in extras:
         lwl = WORKLOADS["long-context-decode"]
         lb = DecodeBench(lwl, min(K, 50), W)
