@@ -141,6 +141,23 @@ def test_dense_k_equals_standard_attention():
         np.testing.assert_allclose(res["out"][0, h], ref, rtol=1e-11, atol=1e-12)
 
 
+def test_dense_k_lse_equals_standard_logsumexp():
+    """k = d with an orthogonal P: the step's log-sum-exp of the scaled scores is
+    the textbook one over the raw q.k (closed form), computed here by scipy."""
+    from scipy.special import logsumexp
+    d, T, Hq = 128, 300, 4
+    P = _rand_orthogonal(d, 7)[None]
+    q = synth.qk_tensor((1, Hq, d), 2)
+    k = synth.qk_tensor((1, T, 1, d), 3)
+    v = synth.v_tensor((1, T, 1, d), 4)
+    Kt = O.build_key_cache(k, P, "f64").transpose(0, 2, 1, 3)
+    res = O.decode(q, P, Kt, v.transpose(0, 2, 1, 3), [T], k=d)
+    for h in range(Hq):
+        s = (k[0, :, 0].astype(np.float64) @ q[0, h].astype(np.float64)) / math.sqrt(d)
+        assert abs(res["lse"][0, h] - logsumexp(s)) <= 1e-12 * max(1.0, abs(logsumexp(s)))
+        np.testing.assert_allclose(np.sum(res["probs"][0][h]), 1.0, rtol=1e-13)
+
+
 def test_dense_k_equals_standard_attention_fp32_cache():
     d, T = 128, 257
     P = _rand_orthogonal(d, 6)[None]
@@ -224,6 +241,28 @@ def test_truncated_cache_matches_zero_tail_query():
     np.testing.assert_array_equal(o_md, o_full)
 
 
+def test_truncated_cache_build_and_decode_keep_the_leading_dims():
+    """The stored cache with m < d feeds a decode step that equals the full-cache
+    step for queries whose projection vanishes beyond m (the leading m projected
+    dimensions are the ones kept), and m = d is the untruncated cache."""
+    d, m, k, T, Hq = 128, 96, 64, 90, 2
+    P = _rand_orthogonal(d, 13)
+    rng = np.random.default_rng(6)
+    qt = rng.standard_normal((1, Hq, d))
+    qt[..., m:] = 0.0
+    q = qt @ P.T                                   # so that q P = qt
+    kk = rng.standard_normal((1, T, 1, d))
+    V = rng.standard_normal((1, 1, T, d))
+    full = O.build_key_cache(kk, P[None], "f64").transpose(0, 2, 1, 3)
+    trunc = O.build_key_cache(kk, P[None], "f64", m).transpose(0, 2, 1, 3)
+    assert trunc.shape[-1] == m
+    r_full = O.decode(q, P[None], full, V, [T], k)
+    r_tr = O.decode(q, P[None], trunc, V, [T], k, m=m)
+    np.testing.assert_array_equal(r_full["sel"], r_tr["sel"])
+    np.testing.assert_allclose(r_tr["out"], r_full["out"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(O.build_key_cache(kk, P[None], "f64", d), O.build_key_cache(kk, P[None], "f64"))
+
+
 # --------------------------------------------------------------------------- prefill vs decode
 
 def test_prefill_row_equals_decode_and_chunk_invariance():
@@ -273,6 +312,25 @@ def test_h2o_large_budget_is_plain_decode():
     for s in range(steps):
         res = O.decode(inp["q"][s], P, Kt, v_all.transpose(0, 2, 1, 3), [T0 + s + 1], 64)
         np.testing.assert_allclose(outs[s], res["out"][0], rtol=1e-12, atol=1e-13)
+
+
+def test_h2o_cumulative_score_is_sum_of_group_probabilities():
+    """With no eviction, a token's cumulative score after the last step is the
+    sum, over every step since it entered and over the group's query heads, of
+    its softmax probability in a plain decode step over the same tokens."""
+    T0, steps, G = 30, 4, 2
+    P, inp, seqs, outs, evs = _h2o_run(budget=1000, recent=8, steps=steps, T0=T0)
+    k_all = np.concatenate([inp["k_hist"], inp["k_new"].transpose(1, 0, 2, 3)], axis=1)
+    v_all = np.concatenate([inp["v_hist"], inp["v_new"].transpose(1, 0, 2, 3)], axis=1)
+    Kt = O.build_key_cache(k_all, P, "bf16").transpose(0, 2, 1, 3)
+    acc = np.zeros((2, T0 + steps))
+    for s in range(steps):
+        res = O.decode(inp["q"][s], P, Kt, v_all.transpose(0, 2, 1, 3), [T0 + s + 1], 64)
+        for h in range(4):
+            acc[h // G, :T0 + s + 1] += res["probs"][0][h]
+    for g in range(2):
+        assert seqs[g].pos == list(range(T0 + steps))
+        np.testing.assert_allclose(seqs[g].score, acc[g], rtol=1e-12, atol=1e-15)
 
 
 def test_h2o_recent_equals_budget_is_sliding_window():
