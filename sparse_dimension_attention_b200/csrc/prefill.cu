@@ -234,14 +234,20 @@ __device__ __forceinline__ void issue_qk(unsigned char* smem, uint32_t tm_S, int
                                          uint32_t idesc) {
   using S = AttnSmem;
   const int kb = (j & 1) ? S::OFF_K1 : S::OFF_K0;
-  int n = 0;
+  const int nks = DS / 16;
+  // Descriptors of the first k-step, built once; a later k-step adds its byte
+  // offset / 16 to the start-address field (every offset is a multiple of 16 and
+  // every address stays below 2^18, so the field never carries).  The issuing
+  // thread then spends one add per MMA.
+  const uint64_t bd0 = smem_desc_sw128(smem + kb, DS * 128, 1024);
+#pragma unroll
   for (int part = 0; part < 2; ++part) {
-    const int qa = part == 0 ? S::OFF_QH : S::OFF_QL;
-    for (int ks = 0; ks < DS / 16; ++ks, ++n) {
-      const uint64_t ad = smem_desc_sw128(smem + qa + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
-      const uint64_t bd = smem_desc_sw128(smem + kb + ks * 16 * 128, DS * 128, 1024);
-      tc_mma(tm_S, ad, bd, idesc, n > 0);
-    }
+    const uint64_t ad0 = smem_desc_sw128(smem + (part == 0 ? S::OFF_QH : S::OFF_QL), 16, 1024);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks)
+      if (ks < nks)
+        tc_mma(tm_S, ad0 + (uint64_t)(((ks >> 2) * S::TILE + (ks & 3) * 32) >> 4),
+               bd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc, part > 0 || ks > 0);
   }
   tc_commit(&bars[BAR_KE0 + (j & 1)]);
   tc_commit(&bars[BAR_S]);
@@ -353,13 +359,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok) {
         tc_fence_after();
         // q~ = q (P1 + P2 + P3): A = raw q rows (K-major), B = P parts (MN-major: input dim x output dim)
+        const uint64_t aq0 = smem_desc_sw128(smem + S::OFF_QL, 16, 1024);
+#pragma unroll
         for (int part = 0; part < 3; ++part) {
           const int part_off = part == 0 ? S::OFF_V1 : (part == 1 ? S::OFF_PP : S::OFF_QH);
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = smem_desc_sw128(smem + S::OFF_QL + (ks >> 2) * S::TILE + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(smem + part_off + ks * 16 * 128, S::TILE, 1024);
-            tc_mma(tm_O, ad, bd, idesc, part > 0 || ks > 0);
-          }
+          const uint64_t bp0 = smem_desc_sw128(smem + part_off, S::TILE, 1024);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            tc_mma(tm_O, aq0 + (uint64_t)(((ks >> 2) * S::TILE + (ks & 3) * 32) >> 4),
+                   bp0 + (uint64_t)((ks * 16 * 128) >> 4), idesc, part > 0 || ks > 0);
         }
         tc_commit(&bars[BAR_QT]);
         ok = wait_or_abort(&bars[BAR_QM], 0, abort_flag);
@@ -384,11 +392,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         // O += Ph V + Pl V, P (128 rows x 128 tokens, two tokens per column) from tensor memory
         const int vb = (j & 1) ? S::OFF_V1 : S::OFF_V0;
+        const uint64_t bv0 = smem_desc_sw128(smem + vb, S::TILE, 1024);   // k-step ks adds ks * 2048 B / 16
+#pragma unroll
         for (int part = 0; part < 2; ++part)
-          for (int ks = 0; ks < PN / 16; ++ks) {
-            const uint64_t bd = smem_desc_sw128(smem + vb + ks * 16 * 128, S::TILE, 1024);
-            tc_mma_ts(tm_O, tm_P + part * 64 + ks * 8, bd, idesc, j > 0 || part > 0 || ks > 0);
-          }
+#pragma unroll
+          for (int ks = 0; ks < PN / 16; ++ks)
+            tc_mma_ts(tm_O, tm_P + part * 64 + ks * 8, bv0 + (uint64_t)((ks * 16 * 128) >> 4), idesc,
+                      j > 0 || part > 0 || ks > 0);
         tc_commit(&bars[BAR_VE0 + (j & 1)]);
         tc_commit(&bars[BAR_O]);
       }
