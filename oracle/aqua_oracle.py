@@ -23,8 +23,9 @@ fp32), and a bf16 output tensor holds the RNE rounding of the exact output.
 The oracle implements both roundings itself (``round_bf16``).
 
 Pins (what fixes each function other than itself) live in
-tests/test_oracle_pins.py.  Every function here is pinned except
-``breakeven_length``, whose formula the pages do not print: parity unpinned.
+tests/test_oracle_pins.py.  Every function here is pinned.  The pages print
+no formula for ``breakeven_length``; it is pinned against a multiply-add
+count of this module's own ``project`` and ``sparse_scores``.
 """
 from __future__ import annotations
 
@@ -341,11 +342,12 @@ def qk_macs(T: int, d: int, k: int | None = None) -> int:
 def breakeven_length(d: int, k: int, G: int) -> float:
     """Sequence length beyond which AQUA's decode multiply-adds undercut dense attention.
 
-    Parity unpinned: the pages state that such a break-even point exists
-    (abstract; edgentiq, Key Advantages) but print no formula.  Reading: per
-    query head and decode step AQUA adds the query projection (d^2) and its
-    share of the key projection (d^2 / G) and saves (d - k) per token, so
-    T* = d^2 (1 + 1/G) / (d - k).
+    The pages state that such a break-even point exists (abstract; edgentiq,
+    Key Advantages) but print no formula.  Reading: per query head and decode
+    step AQUA adds the query projection (d^2) and its share of the key
+    projection (d^2 / G: one new key per KV head serves G query heads) and
+    saves (d - k) per token, so T* = d^2 (1 + 1/G) / (d - k).  Counted in
+    multiply-adds, not bytes.
     """
     if k >= d:
         return float("inf")

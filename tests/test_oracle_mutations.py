@@ -52,6 +52,10 @@ MUTANTS = [
      "recent window one token long"),
     ("h2o_decode_step", "acc += p", "acc = p", "score of the last head only"),
     ("h2o_decode_step", "s.score[i] += acc[i]", "s.score[i] = acc[i]", "score not cumulative"),
+    ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * d * 1.0", "break-even without the key projection share"),
+    ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * k * (1.0 + 1.0 / G)",
+     "break-even with d k instead of d^2 projection work"),
+    ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * d * (1.0 + G)", "break-even with G key projections"),
 ]
 
 

@@ -369,7 +369,83 @@ def test_qk_mac_count_matches_pages_25_percent():
     assert O.qk_macs(T, 128, 96) / O.qk_macs(T, 128) == 0.75
 
 
-def test_breakeven_is_finite_below_d():
-    # parity unpinned (no formula on the pages); only its domain is checked
-    assert O.breakeven_length(128, 128, 4) == float("inf")
-    assert O.breakeven_length(128, 96, 4) > 0
+class _MacCounter(np.ndarray):
+    """ndarray that adds the multiply-adds of every matmul it takes part in to
+    a shared tally (output elements times the contracted length)."""
+    tally = [0]
+
+    def __array_ufunc__(self, ufunc, method, *inputs, **kw):
+        args = [np.asarray(x) if isinstance(x, _MacCounter) else x for x in inputs]
+        res = getattr(ufunc, method)(*args, **kw)
+        if ufunc is np.matmul and method == "__call__":
+            _MacCounter.tally[0] += int(np.prod(np.shape(res))) * args[0].shape[-1]
+        return res.view(_MacCounter) if isinstance(res, np.ndarray) else res
+
+
+class _NumpyKeepingSubclasses:
+    """Stand-in for the oracle module's numpy whose asarray keeps array
+    subclasses (so the counter survives the oracle's input conversions)."""
+
+    def __getattr__(self, name):
+        return getattr(np, name)
+
+    @staticmethod
+    def asarray(a, dtype=None):
+        return np.asanyarray(a, dtype=dtype)
+
+
+def _counted_macs(fn):
+    _MacCounter.tally[0] = 0
+    fn()
+    return _MacCounter.tally[0]
+
+
+def test_breakeven_matches_the_oracles_own_operation_count():
+    """The break-even length is the first context length at which one AQUA
+    decode step costs fewer multiply-adds than dense attention, per query
+    head.  Both costs are COUNTED here on the oracle's own functions (every
+    matmul they execute, through a counting array type), not recomputed from
+    a formula: AQUA = the query projection + 1/G of the key projection (one
+    new key per KV head serves its G query heads) + the scores on the k
+    selected dimensions; dense = the textbook q . k over all d dimensions.
+    A search over T finds the first T where AQUA is cheaper; breakeven_length
+    must agree with it to within one token."""
+    saved = O.np
+    O.np = _NumpyKeepingSubclasses()
+    try:
+        _breakeven_search()
+    finally:
+        O.np = saved
+
+
+def _breakeven_search():
+    d = 128
+    rng = np.random.default_rng(3)
+    P = _rand_orthogonal(d, 4).view(_MacCounter)
+    K_all = rng.standard_normal((8192, d)).view(_MacCounter)
+    q = rng.standard_normal(d).view(_MacCounter)
+    k_new = rng.standard_normal(d).view(_MacCounter)
+    for k, G in [(96, 4), (64, 4), (32, 4), (96, 1), (120, 2), (64, 2)]:
+        def aqua(T):
+            def step():
+                qt = O.project(q, P)
+                S = O.select_dims(np.asarray(qt), k)
+                O.sparse_scores(qt, S, K_all[:T], 1.0)
+            kproj = _counted_macs(lambda: O.project(k_new, P))
+            return _counted_macs(step) + kproj / G
+
+        def dense(T):
+            return _counted_macs(lambda: K_all[:T] @ q)
+
+        assert aqua(1000) - aqua(999) == k and dense(1000) - dense(999) == d   # k, d per token
+        lo, hi = 1, 8192
+        assert aqua(hi) < dense(hi) and not aqua(lo) < dense(lo)
+        while hi - lo > 1:                 # first T with aqua(T) < dense(T) is hi
+            mid = (lo + hi) // 2
+            if aqua(mid) < dense(mid):
+                hi = mid
+            else:
+                lo = mid
+        T_star = O.breakeven_length(d, k, G)
+        assert abs(hi - T_star) <= 1, (k, G, hi, T_star)
+    assert O.breakeven_length(d, d, 4) == float("inf")   # no saving per token: no break-even
