@@ -44,34 +44,34 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "llama3.1-8b-decode"
 # chunked causal prefill: a 4096-token prompt in 512-token chunks (Llama-3.1-8B heads)
 PREFILL = dict(B=1, Hq=32, Hkv=8, L_total=4096, chunk=512, k=96)
+# the same prompt on a truncated cache (AQUA-Memory: the first m projected key
+# dimensions stored), k chosen within them
+PREFILL_TRUNC = dict(PREFILL, d_store=96, k=64)
 # truncated cache (first m projected dims stored), k within them, H2O budget of
 # `recent` newest + heavy hitters; absolute length runs from `budget` to T_end
 H2O_WL = dict(B=32, Hq=32, Hkv=8, m=96, k=64, budget=2048, recent=256, T_end=32768)
 # break-even sweep over the context length and k at the Llama decode shape (one
 # cache built at the largest T; shorter contexts rewind the lengths)
-T_SWEEP = dict(B=8, Hq=32, Hkv=8, kv="bf16", d_store=128, Ts=(512, 1024, 2048, 4096, 8192, 16384, 32768),
-               ks=(128, 96, 64, 32))
+T_SWEEP = dict(B=8, Hq=32, Hkv=8, kv="bf16", d_store=128, Ts=(2048, 8192, 32768), ks=(128, 96, 64, 32))
+T_SWEEP_FULL_TS = (512, 1024, 2048, 4096, 8192, 16384, 32768)
 L2_BYTES = 126e6
 FALLBACK_HBM_GBS = 6650.0
 
 
-def profile_traffic():
-    """DRAM bytes per launch of the attention kernel from the committed ncu summary,
-    or None when the kernel source changed since that capture."""
+def profile_traffic(kernel: str, source: str):
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu
+    traffic record (profiles/ncu_traffic.json, one entry per kernel with the
+    sha256 of the source it was captured from), or None when the kernel's
+    source changed since that capture."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "decode_attn_bf16_llama3.1-8b-decode.md")
-    src = os.path.join(ROOT, "sparse_dimension_attention_b200", "csrc", "decode.cu")
     try:
-        txt = open(prof).read()
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        if ("source sha256: " + digest) not in txt:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "ncu_traffic.json")))[kernel]
+        digest = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()
+        if rec.get("source_sha256") != digest:
             return None
-        for ln in txt.splitlines():
-            if ln.startswith("traffic_bytes_per_launch:"):
-                return int(ln.split(":")[1])
+        return int(rec["dram_bytes_per_launch"])
     except Exception:
         return None
-    return None
 
 
 def peaks():
@@ -307,6 +307,47 @@ class DecodeBench:
         wl, e = self.wl, self.esize
         return float(wl["B"] * wl["Hkv"] * 128 * e * 4)    # read k, v; write k~ column, v row
 
+    def bytes_attend(self, usz: np.ndarray, T: int) -> float:
+        """Algorithmic HBM bytes of the attention kernel alone: union rows of K~
+        and V rows per (b, g) and token, and the output write."""
+        wl, e = self.wl, self.esize
+        return float(T * np.sum(e * usz + e * 128) + wl["B"] * wl["Hq"] * 128 * e)
+
+    def kernel_times(self, K: int, k: int):
+        """Each kernel of the decode step timed alone with CUDA events on the
+        launching stream: K steps issued as aqua_decode_select (projection
+        kernel with the fused append) and aqua_decode_attend (attention
+        kernel), with an event before, between and after.  An event between
+        the two launches serialises the attention kernel behind the projection
+        kernel (no programmatic overlap), so each interval is one kernel's
+        duration.  A sleep kernel in front keeps the GPU busy while the host
+        enqueues all K steps, so no interval includes host launch gaps.
+        Returns the mean select and attend durations in ms."""
+        torch, aq, wl = self.torch, self.aq, self.wl
+        st = torch.cuda.current_stream()
+        self.rewind()
+        for s in range(3):                                   # warm (first launches configure the kernels)
+            aq.aqua_decode_select(self.cache.desc, self.q_d[s], self.P, wl["Hq"], k, self.ws,
+                                  k_new=self.k_d[s], v_new=self.v_d[s])
+            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True)
+        torch.cuda.synchronize()
+        self.rewind()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        torch.cuda._sleep(int(2e6 + K * 1e5))                # ~1 ms + 50 us per step of GPU time
+        for s in range(K):
+            i = s % self.n_in
+            ev[s][0].record(st)
+            aq.aqua_decode_select(self.cache.desc, self.q_d[i], self.P, wl["Hq"], k, self.ws,
+                                  k_new=self.k_d[i], v_new=self.v_d[i])
+            ev[s][1].record(st)
+            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True)
+            ev[s][2].record(st)
+        torch.cuda.synchronize()
+        sel = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+        att = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+        self.rewind()
+        return sel, att
+
     def timed_unfused(self, K: int, W: int, k: int):
         """The same steps as two public calls (aqua_project_keys, then aqua_decode_attn)."""
         torch = self.torch
@@ -368,42 +409,51 @@ class DecodeBench:
 
     def e2e(self, K: int, k: int):
         """Same steps through the public API from pinned host memory: per step one
-        H2D copy of the step's packed inputs (q, k_new, v_new), issued in front of
-        the step's calls, and the D2H copy of the step's output are part of the
-        timed region (captured with the calls into one CUDA graph).  The output
-        copy runs on a second stream from a double-buffered output, so it overlaps
-        the next step's kernels; the input copy does not overlap."""
+        H2D copy of the step's packed inputs (q, k_new, v_new) and one D2H copy
+        of the step's output are part of the timed region (captured with the
+        calls into one CUDA graph).  Both copies run on a second stream with
+        double buffers: the input copy of step s + 1 overlaps step s's kernels
+        (it waits until step s - 1, the last user of its buffer, is done), and
+        the output copy of step s overlaps step s + 1."""
         torch = self.torch
         st = torch.cuda.current_stream()
         cs = torch.cuda.Stream()
         wl = self.wl
         nq, nk = self.q_d[0].numel(), self.k_d[0].numel()
-        in_d = torch.empty_like(self.in_h[0], device="cuda")
-        qd = in_d[:nq].view(self.q_d[0].shape)
-        kd = in_d[nq:nq + nk].view(self.k_d[0].shape)
-        vd = in_d[nq + nk:].view(self.v_d[0].shape)
+        in_d = [torch.empty_like(self.in_h[0], device="cuda") for _ in range(2)]
+        views = [(x[:nq].view(self.q_d[0].shape), x[nq:nq + nk].view(self.k_d[0].shape),
+                  x[nq + nk:].view(self.v_d[0].shape)) for x in in_d]
         outs = [self.out, torch.empty_like(self.out)]
         outs_h = [self.out_h, torch.empty_like(self.out_h).pin_memory()]
 
-        def one(s, done, copied):
-            i = s % self.n_in
-            in_d.copy_(self.in_h[i], non_blocking=True)
-            if s >= 2:
-                st.wait_event(copied[s - 2])          # the output buffer's previous copy is out
-            self.aq.aqua_decode_attn(self.cache.desc, qd, self.P, wl["Hq"], k, outs[s % 2], self.ws, k_new=kd,
-                                     v_new=vd)
-            done[s].record(st)
-            with torch.cuda.stream(cs):
-                cs.wait_event(done[s])
-                outs_h[s % 2].copy_(outs[s % 2], non_blocking=True)
-                copied[s].record(cs)
-
         def run(n):
             done = [torch.cuda.Event() for _ in range(n)]
+            loaded = [torch.cuda.Event() for _ in range(n)]
             copied = [torch.cuda.Event() for _ in range(n)]
             cs.wait_stream(st)
+
+            def load(s):
+                with torch.cuda.stream(cs):
+                    if s >= 2:
+                        cs.wait_event(done[s - 2])            # step s - 2 no longer reads this buffer
+                    in_d[s % 2].copy_(self.in_h[s % self.n_in], non_blocking=True)
+                    loaded[s].record(cs)
+
+            load(0)
             for s in range(n):
-                one(s, done, copied)
+                if s + 1 < n:
+                    load(s + 1)
+                st.wait_event(loaded[s])
+                if s >= 2:
+                    st.wait_event(copied[s - 2])              # the output buffer's previous copy is out
+                qd, kd, vd = views[s % 2]
+                self.aq.aqua_decode_attn(self.cache.desc, qd, self.P, wl["Hq"], k, outs[s % 2], self.ws,
+                                         k_new=kd, v_new=vd)
+                done[s].record(st)
+                with torch.cuda.stream(cs):
+                    cs.wait_event(done[s])
+                    outs_h[s % 2].copy_(outs[s % 2], non_blocking=True)
+                    copied[s].record(cs)
             st.wait_stream(cs)
 
         self.rewind()
@@ -433,18 +483,20 @@ class DecodeBench:
 
 class PrefillBench:
     """A prompt pass = for every chunk: aqua_project_keys (append the chunk's keys
-    and values), then aqua_prefill_attn (selection + tcgen05 attention)."""
+    and values), then aqua_prefill_attn (selection + tcgen05 attention).  With
+    d_store < d the cache keeps the first d_store projected key dimensions."""
 
     def __init__(self, wl: dict, P):
         import torch
         import sparse_dimension_attention_b200 as aq
         self.aq, self.torch, self.wl, self.P = aq, torch, wl, P[:wl["Hkv"]].contiguous()
+        self.d_store = wl.get("d_store", 128)
         inp = synth.prefill_inputs(wl["L_total"], wl["Hq"], wl["Hkv"], bf16=True, B=wl["B"])
         bf = torch.bfloat16
         self.q = torch.from_numpy(inp["q"]).to(bf).cuda()          # [B, L, Hq, d]
         self.k = torch.from_numpy(inp["k"]).to(bf).cuda()          # [B, L, Hkv, d]
         self.v = torch.from_numpy(inp["v"]).to(bf).cuda()
-        self.cache = aq.AquaCache(wl["B"], wl["Hkv"], wl["L_total"] + 128)
+        self.cache = aq.AquaCache(wl["B"], wl["Hkv"], wl["L_total"] + 128, d_store=self.d_store)
         self.out = torch.empty((wl["B"], wl["chunk"], wl["Hq"], 128), dtype=bf, device="cuda")
         self.ws = torch.empty(aq.aqua_prefill_workspace_size(self.cache.desc, wl["Hq"], wl["chunk"]),
                               dtype=torch.uint8, device="cuda")
@@ -462,19 +514,23 @@ class PrefillBench:
             if ev is not None:
                 ev[c][1].record()
 
-    def flops(self, pos0: int):
-        """(dense causal flops, tensor-core flops issued) of one aqua_prefill_attn chunk call.
-        Dense causal: 2 d flops for q.k and 2 d for p.v per visible (row, token) per
-        query head.  Issued: the kernel's MMAs, bf16 high+low parts of the masked
-        query and of P, over every 128-token tile each 128-row CTA visits."""
+    def flops(self, pos0: int, k: int):
+        """(algorithmic, dense causal, tensor-core issued) flops of one
+        aqua_prefill_attn chunk call.  Algorithmic: 2 k flops for the scores on
+        the k selected dimensions and 2 d for p.v, per visible (row, token)
+        pair and query head.  Dense causal: 4 d per pair and head (standard
+        attention).  Issued: the kernel's MMAs, bf16 high + low parts of the
+        masked query (contraction d_store) and of P, over every 128-token tile
+        each 128-row CTA visits."""
         wl, C, d = self.wl, self.wl["chunk"], 128
         G = wl["Hq"] // wl["Hkv"]
         pairs = C * pos0 + C * (C + 1) // 2
+        alg = pairs * wl["Hq"] * (2.0 * k + 2.0 * d)
         dense = pairs * wl["Hq"] * 4.0 * d
         rpb = 128 // G
         tiles = sum(-(-(pos0 + min(C, (qb + 1) * rpb)) // 128) for qb in range(-(-C // rpb)))
-        issued = tiles * wl["Hkv"] * wl["B"] * (2 * 2.0 * 128 * 128 * d + 2 * 2.0 * 128 * 128 * 128)
-        return dense, issued
+        issued = tiles * wl["Hkv"] * wl["B"] * (2 * 2.0 * 128 * 128 * self.d_store + 2 * 2.0 * 128 * 128 * d)
+        return alg, dense, issued
 
     def timed(self, K: int, W: int, k: int):
         torch = self.torch
@@ -518,34 +574,52 @@ class PrefillBench:
         del g
         return e0.elapsed_time(e1) / K
 
-    def report(self, K: int, W: int, bf16_peak: float, peak_kind: str) -> dict:
+    def report(self, K: int, W: int, bf16_peak: float, peak_kind: str, dense_ref_ms: float | None = None,
+               workload: str = "chunked-prefill-4096") -> dict:
+        """The prompt at the workload's k against k = d_store (every stored
+        dimension kept: the masked contraction is dense) on the same cache, and
+        against dense_ref_ms (the full k = d pass on an untruncated cache) when
+        given.  roofline.frac uses the algorithmic flops."""
         wl = self.wl
+        k_dense = self.d_store
         eager_ms, attn_ms = self.timed(K, W, wl["k"])
-        dense_eager_ms, dense_attn = self.timed(K, W, 128)
+        dense_eager_ms, _ = self.timed(K, W, k_dense)
         prompt_ms = self.timed_graph(K, W, wl["k"])
-        dense_ms = self.timed_graph(K, W, 128)
-        fl = [self.flops(c * wl["chunk"]) for c in range(self.n_chunks)]
-        dense_f = sum(f[0] for f in fl)
-        issued_f = sum(f[1] for f in fl)
+        dense_ms = self.timed_graph(K, W, k_dense)
+        fl = [self.flops(c * wl["chunk"], wl["k"]) for c in range(self.n_chunks)]
+        alg_f = sum(f[0] for f in fl)
+        dense_f = sum(f[1] for f in fl)
+        issued_f = sum(f[2] for f in fl)
         t_attn = float(attn_ms.sum()) / 1e3
-        alg = dense_f / t_attn / 1e12
-        return {"workload": "chunked-prefill-4096", **wl, "d": 128,
+        alg = alg_f / t_attn / 1e12
+        line = {"workload": workload, **wl, "d": 128, "d_store": self.d_store,
                 "prompt_ms": prompt_ms, "tokens_per_s": wl["B"] * wl["L_total"] / (prompt_ms / 1e3),
                 "attn_call_us": [round(1e3 * x, 2) for x in attn_ms],
                 "roofline": {"bound": "tensor", "achieved": alg, "peak": bf16_peak, "unit": "TFLOP/s",
                              "frac": alg / bf16_peak, "peak_source": peak_kind + " bf16 burst",
-                             "achieved_note": "dense causal flops (4 d per visible pair and query head, "
-                                              "%.1f GFLOP per prompt) / summed aqua_prefill_attn call time "
-                                              "(selection + attention kernels)" % (dense_f / 1e9),
+                             "achieved_note": "algorithmic flops (2 k on the selected dimensions + 2 d for p.v per "
+                                              "visible pair and query head, %.1f GFLOP per prompt) / summed "
+                                              "aqua_prefill_attn call time" % (alg_f / 1e9),
+                             "dense_causal_tflops": dense_f / t_attn / 1e12,
+                             "dense_causal_note": "4 d flops per visible pair and query head (%.1f GFLOP)"
+                                                  % (dense_f / 1e9),
                              "issued_tflops": issued_f / t_attn / 1e12,
-                             "issued_note": "tcgen05 flops issued (bf16 high+low splits, whole 128-token tiles)"},
+                             "issued_note": "tcgen05 flops issued (bf16 high+low splits, contraction d_store for "
+                                            "the scores, whole 128-token tiles)"},
                 "prompt_ms_note": "whole prompt pass captured in one CUDA graph; eager (issued call by call "
                                   "from Python, per-chunk events) in prompt_ms_eager",
                 "prompt_ms_eager": eager_ms,
-                "dense_k128_prompt_ms": dense_ms,
-                "dense_k128_prompt_ms_eager": dense_eager_ms,
-                "speedup_vs_dense": dense_ms / prompt_ms,
+                "k_eq_dstore_prompt_ms": dense_ms,
+                "k_eq_dstore_prompt_ms_eager": dense_eager_ms,
+                "speedup_vs_k_eq_dstore": dense_ms / prompt_ms,
                 "l2": "not flushed: a chunk's K~/V (<= 16 MB) were written by the append just before"}
+        if dense_ref_ms is not None:
+            line["dense_ref_prompt_ms"] = dense_ref_ms
+            line["speedup_vs_dense"] = dense_ref_ms / prompt_ms
+            line["speedup_note"] = "dense_ref: k = d = 128 on an untruncated cache (standard attention's work)"
+        else:
+            line["speedup_vs_dense"] = dense_ms / prompt_ms
+        return line
 
 
 class H2OBench:
@@ -588,24 +662,26 @@ class H2OBench:
         aq.aqua_h2o_update(self.cache.desc, self.sc, self.lse, wl["Hq"], wl["budget"], wl["recent"], self.ev)
         self.n_steps += 1
 
-    def bytes_step(self, usz: float) -> float:
+    def bytes_step(self, usz: float, score_roundtrip: bool = True) -> float:
         """Algorithmic HBM bytes of one step at n = budget+1 attended tokens per (b, g):
-        K~ union rows and V rows, the scores write and read-back, the cumulative
-        score/position arrays, the append, q and the output."""
+        K~ union rows and V rows, the cumulative score/position arrays, the
+        append, q and the output; with score_roundtrip also the per-head scores
+        the decode step writes and the H2O update reads back (a consequence of
+        splitting the step into two kernels, not of the method)."""
         wl = self.wl
         B, Hq, Hkv, n = wl["B"], wl["Hq"], wl["Hkv"], wl["budget"] + 1
         units = B * Hkv
         attn = units * n * (2.0 * usz + 2 * 128)
-        scores = 2.0 * B * Hq * n * 4                       # written by the decode, read by the update
+        scores = 2.0 * B * Hq * n * 4 if score_roundtrip else 0.0
         h2o = units * n * (4 + 4 + 4)                       # score read + write, pos read
         move = units * (wl["m"] + 128) * 2 * 2              # victim slot <- last slot
         append = units * (128 * 2 * 2 + wl["m"] * 2 + 128 * 2)
         qo = B * Hq * 128 * 2 * 2
         return attn + scores + h2o + move + append + qo
 
-    def report(self, W: int, K: int = 200) -> dict:
-        """Steady state from T_abs = budget to T_end (runs shorter than 100 main
-        steps replay the 256-step graph only K // 4 + 1 times)."""
+    def report(self, W: int, hbm_peak: float) -> dict:
+        """Steady state over the whole absolute-length range, from T_abs =
+        budget + (warm-up steps) to T_end: 256-step graphs replayed back to back."""
         torch, wl = self.torch, self.wl
         G = wl["Hq"] // wl["Hkv"]
         for _ in range(W):
@@ -626,8 +702,6 @@ class H2OBench:
         torch.cuda.synchronize()
         t_abs0 = wl["budget"] + self.n_steps                               # tokens seen so far
         reps = max(1, (wl["T_end"] - t_abs0) // self.GRAPH_STEPS)
-        if K < 100:
-            reps = min(reps, K // 4 + 1)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(reps):
@@ -640,24 +714,31 @@ class H2OBench:
         n_len = int(self.cache.len[0].item())
         status = self.aq.aqua_status(self.cache.desc)
         by = self.bytes_step(float(np.mean(usz)))
-        return {"workload": "truncated-h2o-decode", **wl, "d": 128,
+        by_nrt = self.bytes_step(float(np.mean(usz)), score_roundtrip=False)
+        gbs = by * K / (ms / 1e3) / 1e9
+        gbs_nrt = by_nrt * K / (ms / 1e3) / 1e9
+        return {"workload": "truncated-h2o-decode", **wl, "d": 128, "T_end": t_abs0 + K,
+                "T_end_config": wl["T_end"],
                 "steps": K, "T_abs_range": [t_abs0, t_abs0 + K], "cache_len_after": n_len, "status": status,
                 "queries_per_s": wl["B"] * K / (ms / 1e3), "ms_per_step": ms / K,
-                "mean_union": float(np.mean(usz)), "bytes_per_step": by,
-                "hbm_gbs": by * K / (ms / 1e3) / 1e9,
+                "mean_union": float(np.mean(usz)), "bytes_per_step": by, "hbm_gbs": gbs, "frac": gbs / hbm_peak,
+                "bytes_per_step_no_score_roundtrip": by_nrt, "hbm_gbs_no_score_roundtrip": gbs_nrt,
+                "frac_no_score_roundtrip": gbs_nrt / hbm_peak,
                 "launch": "%d-step CUDA graph replayed %d times; 3 launches per step" % (self.GRAPH_STEPS, reps),
                 "l2": "no flush: each step streams %.0f MB, above the 126 MB L2" % (by / 1e6)}
 
 
-def t_sweep(P, K: int, W: int, world: int) -> dict:
+def t_sweep(P, K: int, W: int, world: int, Ts=None) -> dict:
     """Decode step time over context lengths T and selection sizes k at the
     Llama decode shape, against k = d at the same T (the same kernels: at k = d
     the selection keeps every dimension, so the comparison isolates what the
-    smaller union saves against the fixed per-step costs).  Also the pages'
-    flop break-even T* = d^2 (1 + 1/G) / (d - k) of AQUA against dense attention
-    per query head, for reference."""
+    smaller union saves against the fixed per-step costs).  Each point also
+    carries the speedup its bytes allow, 2d / (|U| + d) (K~ union rows + V
+    against K~ + V), and the pages' flop break-even T* = d^2 (1 + 1/G) / (d - k)
+    of AQUA against dense attention per query head."""
     tw = dict(T_SWEEP)
-    Ts, ks = tw.pop("Ts"), tw.pop("ks")
+    Ts, ks = Ts or tw.pop("Ts"), tw.pop("ks")
+    tw.pop("Ts", None)
     wl = dict(tw, T=max(Ts), k=ks[0])
     tb = DecodeBench(wl, K, W, P=P)
     unions = {kk: tb.union_sizes(kk, min(K, 8)) for kk in ks}
@@ -676,10 +757,11 @@ def t_sweep(P, K: int, W: int, world: int) -> dict:
             rows.append({"T": T, "k": kk, "decode_us": us, "mean_union": float(u.mean()),
                          "decode_gbs": sum(by) / (t_ms / 1e3) / 1e9,
                          "speedup_vs_k_d": (dense_us / us) if dense_us else None,
+                         "byte_bound_speedup": 2.0 * d / (float(u.mean()) + d),
                          "l2_resident": by[0] < L2_BYTES})
     del tb
     return {"workload": "llama3.1-8b-decode T x k sweep", "B": wl["B"], "Hq": wl["Hq"], "Hkv": wl["Hkv"],
-            "rows": rows, "launch": "K steps in one CUDA graph per (T, k)",
+            "steps_per_point": K, "rows": rows, "launch": "K steps in one CUDA graph per (T, k)",
             "flop_breakeven_T": {str(kk): d * d * (1 + 1 / G) / (d - kk) for kk in ks if kk < d},
             "note": "l2_resident: a step's algorithmic bytes fit in the 126 MB L2 (no flush between steps)"}
 
@@ -764,10 +846,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--no-extras", action="store_true", help="only the main decode line")
-    ap.add_argument("--extras", default="sweep,long,prefill,h2o",
-                    help="comma list of extra lines: sweep (k sweep), long (long context), prefill (chunked "
-                         "prefill), h2o (truncated cache + H2O steady state); tsweep (break-even sweep over "
-                         "T and k, not in the default)")
+    ap.add_argument("--extras", default="sweep,tsweep,long,prefill,h2o",
+                    help="comma list of extra lines: sweep (k sweep), tsweep (break-even sweep over T in "
+                         "{2048, 8192, 32768} and k), tsweep_full (T from 512 to 32768), long (long context), "
+                         "prefill (chunked prefill, full and truncated cache), h2o (truncated cache + H2O steady "
+                         "state)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -791,12 +874,17 @@ def main():
     value = whole_job_rate(wl["B"], K, world, total_ms)
     T_steps = [wl["T"] + s for s in range(K)]
     dec_bytes = [bench.bytes_decode(usz[s % usz.shape[0]], T_steps[s]) for s in range(K)]
-    achieved = (sum(dec_bytes) + K * bench.bytes_append()) / (sum(step_ms) / 1e3) / 1e9
     step_gbs = (sum(dec_bytes) + K * bench.bytes_append()) / (total_ms / 1e3) / 1e9
+    # the dominant kernel alone: the attention kernel's algorithmic bytes over its own duration
+    Kk = min(K, 50)
+    sel_ms, att_ms = bench.kernel_times(Kk, wl["k"])
+    att_bytes = float(np.mean([bench.bytes_attend(usz[s % usz.shape[0]], T_steps[s]) for s in range(Kk)]))
+    att_gbs = att_bytes / (att_ms / 1e3) / 1e9
     unfused_ms = bench.timed_unfused(min(K, 100), W, wl["k"])
     eager_ms, _, _ = bench.timed(min(K, 100), W, wl["k"], world, clocks=False, graph=False)
     e2e_ms, h2d, d2h = bench.e2e(K, wl["k"])
     e2e_ms = max_over_ranks(e2e_ms, world)
+    kname = "decode_attn_bf16_kernel" if wl["kv"] == "bf16" else "decode_attn_f32_kernel"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -810,20 +898,28 @@ def main():
                    "inputs": "synthetic anisotropic Q/K (Llama-3.1-8B shape), P from GPU SVD calibration"},
         "hbm_gbs": step_gbs,
         "mean_union": float(usz.mean()),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": profile_traffic(),
-                     "traffic_note": "ncu DRAM read+write bytes of one decode_attn_bf16_kernel launch "
-                                     "(profiles/decode_attn_bf16_llama3.1-8b-decode.md); null if the kernel changed",
-                     "kernel": "aqua_decode_attn step (qproj_topk_kernel with fused append + decode_attn_bf16_kernel)",
+        "roofline": {"bound": "hbm", "achieved": att_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": att_gbs / hbm_peak,
+                     "traffic": profile_traffic(kname, "sparse_dimension_attention_b200/csrc/decode.cu"),
+                     "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the "
+                                     "kernel (profiles/ncu_traffic.json); null when its source changed since",
+                     "kernel": kname, "kernel_us": 1e3 * att_ms, "bytes_per_launch": att_bytes,
+                     "achieved_note": "algorithmic bytes of the attention kernel (K~ union rows + V rows per "
+                                      "(b, KV head) and token, output write) / its mean duration alone (CUDA "
+                                      "events around aqua_decode_attend, %d steps)" % Kk,
                      "peak_source": peak_kind,
-                     "step_us": 1e3 * statistics.mean(step_ms)},
+                     "select_kernel_us": 1e3 * sel_ms,
+                     "step_us": 1e3 * ms_step, "step_gbs": step_gbs, "step_frac": step_gbs / hbm_peak,
+                     "step_note": "whole step (both kernels, programmatically overlapped, in one CUDA graph): "
+                                  "all algorithmic bytes incl. the append / step time"},
         "launch": "K steps captured in one CUDA graph (kernels chained with programmatic dependent launch)",
         "eager_step_us": 1e3 * eager_ms / min(K, 100),
         "unfused_step_us": 1e3 * unfused_ms,
         "e2e": {"value": whole_job_rate(wl["B"], K, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "note": "aqua_decode_attn from pinned host buffers; each step's input copy precedes its kernels, "
-                        "its output copy overlaps the next step (second stream, two output buffers)"},
+                "note": "aqua_decode_attn from pinned host buffers; per step one packed input copy and one output "
+                        "copy, both double-buffered on a second stream (input of step s+1 and output of step s "
+                        "overlap the step's kernels)"},
         "gpu_launches": 2 * K,
         "clocks": clk,
     }
@@ -837,7 +933,8 @@ def main():
             by = [bench.bytes_decode(u[s % u.shape[0]], T_steps[s]) + bench.bytes_append() for s in range(K)]
             sweep.append({"k": kk, "queries_per_s": world * wl["B"] * K / (t_ms / 1e3), "ms_per_step": t_ms / K,
                           "decode_us": 1e3 * statistics.mean(d_ms), "mean_union": float(u.mean()),
-                          "decode_gbs": sum(by) / (sum(d_ms) / 1e3) / 1e9})
+                          "decode_gbs": sum(by) / (sum(d_ms) / 1e3) / 1e9,
+                          "byte_bound_speedup": 256.0 / (float(u.mean()) + 128.0)})
         dense = sweep[0]["decode_us"]
         for r in sweep:
             r["speedup_vs_dense"] = dense / r["decode_us"]
@@ -845,8 +942,8 @@ def main():
     P = bench.P
     del bench
     torch.cuda.empty_cache()
-    if "tsweep" in extras:
-        line["t_sweep"] = t_sweep(P, min(K, 50), W, world)
+    if "tsweep" in extras or "tsweep_full" in extras:
+        line["t_sweep"] = t_sweep(P, min(K, 20), W, world, Ts=T_SWEEP_FULL_TS if "tsweep_full" in extras else None)
         torch.cuda.empty_cache()
     if "long" in extras:
         lwl = WORKLOADS["long-context-decode"]
@@ -868,11 +965,15 @@ def main():
         line["prefill"] = pb.report(min(K, 20), W, bf16_peak, peak_kind)
         del pb
         torch.cuda.empty_cache()
+        pb = PrefillBench(PREFILL_TRUNC, P)
+        line["prefill_truncated"] = pb.report(min(K, 20), W, bf16_peak, peak_kind,
+                                              dense_ref_ms=line["prefill"]["k_eq_dstore_prompt_ms"],
+                                              workload="chunked-prefill-4096-truncated-cache")
+        del pb
+        torch.cuda.empty_cache()
     if "h2o" in extras:
         hb = H2OBench(H2O_WL, P)
-        r = hb.report(W, K)
-        r["frac"] = r["hbm_gbs"] / hbm_peak
-        line["truncated_h2o"] = r
+        line["truncated_h2o"] = hb.report(W, hbm_peak)
         del hb
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)

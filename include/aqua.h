@@ -149,7 +149,15 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
 
 /*
  * One decode step of AQUA attention for every sequence and query head, over
- * the len[b] cached tokens.
+ * the len[b] cached tokens.  It follows the online phase of the method
+ * (abstract: queries and keys are projected, a sparse subset of dimensions is
+ * chosen by the query's magnitude, the attention scores use only those
+ * dimensions; edgentiq, "How AQUA Works: A Two-Phase Approach", Online
+ * Inference): q~ = q P; S_h = the k dimensions with the largest |q~_j| (ties
+ * to the lower index); s_t = sum over j in S_h of q~_j k~_t[j] / sqrt(d);
+ * softmax over the visible tokens; o_h = sum_t p_t v_t over the unprojected
+ * values.  The 1/sqrt(d) scale, the tie rule and the unprojected V are the
+ * workload statement's readings where the pages are silent.
  *   q          [B][Hq][d]  cache dtype; query head h uses KV head h / (Hq/Hkv)
  *   k_new, v_new  nullable [B][Hkv][d] cache dtype: the step's new key and
  *              value.  When given they are appended, exactly as
@@ -170,6 +178,8 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  *   qproj_out  nullable [B][Hq][d] f32: the projected query q~ the selection used
  *   scores_out nullable [B][Hq][Tcap] f32: score of every cached slot (scaled)
  *   lse_out    nullable [B][Hq] f32: log-sum-exp of the scores
+ *   workspace  device, 256-byte aligned, >= aqua_decode_workspace_size bytes;
+ *              caller-owned scratch, contents need no initialisation
  * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4}.  A sequence with
  * len[b] = 0 gets a zero output and lse = -inf.
  * Errors: AQUA_ERR_ARG if only one of k_new, v_new is given or the cache is full.
@@ -179,6 +189,37 @@ AQUA_API int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_ne
                               const float* P, int Hq, int k, float scale, void* out, int out_dtype,
                               int32_t* sel_out, float* qproj_out, float* scores_out, float* lse_out,
                               void* workspace, size_t workspace_bytes, aqua_stream_t stream);
+
+/*
+ * The decode step of aqua_decode_attn as two calls on the same stream, which
+ * together enqueue exactly the two kernels aqua_decode_attn enqueues and give
+ * bit-identical results:
+ *   aqua_decode_select  the online selection (abstract: project the query, pick
+ *                       the dimensions by the query's magnitude): q~ = q P,
+ *                       top-k of |q~| per query head, the group's union of
+ *                       kept dimensions and the masked queries, written to the
+ *                       workspace; with k_new/v_new also the append (slot
+ *                       len[b], cache->max_len += 1; len[b] itself advances at
+ *                       the end of aqua_decode_attend).
+ *   aqua_decode_attend  the sparse-dimension attention over that selection
+ *                       (edgentiq, "How AQUA Works", Online Inference: scores
+ *                       on the selected dimensions, softmax, weighted sum of
+ *                       the values), split over the SMs and merged.
+ * Use: a caller that wants to schedule or time the two halves separately (an
+ * event between them serialises the second behind the first; back to back
+ * they overlap as in aqua_decode_attn).  The workspace carries the selection
+ * from the first call to the second; neither it nor the cache may be touched
+ * in between.  `appended` must be 1 exactly when the preceding
+ * aqua_decode_select was given k_new/v_new.  Arguments as aqua_decode_attn;
+ * each call checks the arguments it uses (AQUA_ERR_ARG for appended not 0/1,
+ * or 1 with an empty cache).
+ */
+AQUA_API int aqua_decode_select(aqua_cache* cache, const void* q, const void* k_new, const void* v_new,
+                                const float* P, int Hq, int k, float scale, int32_t* sel_out, float* qproj_out,
+                                void* workspace, size_t workspace_bytes, aqua_stream_t stream);
+AQUA_API int aqua_decode_attend(aqua_cache* cache, int Hq, int appended, void* out, int out_dtype,
+                                float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
+                                aqua_stream_t stream);
 
 /*
  * The decode step of aqua_decode_attn for callers that cannot provide device
@@ -208,10 +249,17 @@ AQUA_API int aqua_decode_attn_static(aqua_cache* cache, const void* q, const voi
  * pos0 .. pos0+L-1 of every sequence (their keys must already be appended, so
  * len[b] >= pos0 + L).  Row i of sequence b attends to slots 0 .. pos0+i; each
  * (row, head) selects its own k dimensions; the dimension-masked Q K~^T and
- * P V run on the tensor cores.
+ * P V run on the tensor cores.  The pages describe only the per-query step
+ * (abstract; edgentiq, "How AQUA Works", Online Inference); chunked causal
+ * prefill applies that step to every prompt row, as the workload statement's
+ * prefill configuration (a 4096-token prompt in 512-token chunks, causal)
+ * asks.  Row i's result equals a decode step at position pos0+i.
  *   q    [B][L][Hq][d] cache dtype (bf16 only)
  *   out  [B][L][Hq][d] out_dtype
- *   sel_out nullable [B][L][Hq][k] int32
+ *   sel_out   nullable [B][L][Hq][k] int32: selected dimensions, ascending
+ *   qproj_out nullable [B][L][Hq][d] f32: the projected queries q~ the selection
+ *             used (computed on the tensor cores with P split into three bf16
+ *             parts, f32 accumulation), 16-byte aligned
  *   workspace  device, 256-byte aligned, >= aqua_prefill_workspace_size bytes
  *              (a small reserved block: projection, selection and attention
  *              run in one kernel and keep their intermediates on chip)
@@ -221,7 +269,7 @@ AQUA_API int aqua_decode_attn_static(aqua_cache* cache, const void* q, const voi
  */
 AQUA_API size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L);
 AQUA_API int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, const float* P,
-                      int Hq, int k, float scale, void* out, int out_dtype, int32_t* sel_out,
+                      int Hq, int k, float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out,
                       void* workspace, size_t workspace_bytes, aqua_stream_t stream);
 
 /*

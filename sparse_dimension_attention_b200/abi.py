@@ -28,7 +28,8 @@ EXPORTED = (
     "aqua_last_error", "aqua_version", "aqua_status",
     "aqua_calibrate_workspace_size", "aqua_calibrate",
     "aqua_project_keys",
-    "aqua_decode_workspace_size", "aqua_decode_attn", "aqua_decode_attn_static",
+    "aqua_decode_workspace_size", "aqua_decode_attn", "aqua_decode_select", "aqua_decode_attend",
+    "aqua_decode_attn_static",
     "aqua_prefill_workspace_size", "aqua_prefill_attn",
     "aqua_h2o_update",
     "aqua_selftest_wait_timeout",
@@ -75,10 +76,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "aqua_project_keys": (c_int, [C, P, P, P, c_int, P]),
         "aqua_decode_workspace_size": (c_size_t, [C, c_int]),
         "aqua_decode_attn": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
+        "aqua_decode_select": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, P, P, c_size_t, P]),
+        "aqua_decode_attend": (c_int, [C, c_int, c_int, P, c_int, P, P, P, c_size_t, P]),
         "aqua_decode_attn_static": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P]),
         "aqua_selftest_wait_timeout": (c_int, [C, ctypes.c_ulonglong, P]),
         "aqua_prefill_workspace_size": (c_size_t, [C, c_int, c_int]),
-        "aqua_prefill_attn": (c_int, [C, P, c_int, c_int, P, c_int, c_int, c_float, P, c_int, P, P, c_size_t, P]),
+        "aqua_prefill_attn": (c_int, [C, P, c_int, c_int, P, c_int, c_int, c_float, P, c_int, P, P, P, c_size_t, P]),
         "aqua_h2o_update": (c_int, [C, P, P, c_int, c_int, c_int, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -161,6 +164,23 @@ def aqua_decode_attn(cache: aqua_cache, q, P, Hq: int, k: int, out, workspace, s
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def aqua_decode_select(cache: aqua_cache, q, P, Hq: int, k: int, workspace, scale: float = 0.0, k_new=None,
+                       v_new=None, sel_out=None, qproj_out=None, stream=None) -> None:
+    """First half of a decode step: projection, top-k, group union (and the append)."""
+    _check(load_library().aqua_decode_select(
+        ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(P), Hq, k, scale, _ptr(sel_out),
+        _ptr(qproj_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def aqua_decode_attend(cache: aqua_cache, Hq: int, out, workspace, appended: bool = False, scores_out=None,
+                       lse_out=None, stream=None) -> None:
+    """Second half of a decode step: attention over the selection aqua_decode_select left in the workspace."""
+    out_dtype = AQUA_BF16 if str(out.dtype) == "torch.bfloat16" else AQUA_F32
+    _check(load_library().aqua_decode_attend(
+        ctypes.byref(cache), Hq, int(bool(appended)), _ptr(out), out_dtype, _ptr(scores_out), _ptr(lse_out),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def aqua_decode_attn_static(cache: aqua_cache, q, P, Hq: int, k: int, out, scale: float = 0.0, k_new=None,
                             v_new=None, sel_out=None, qproj_out=None, scores_out=None, lse_out=None,
                             stream=None) -> None:
@@ -177,11 +197,11 @@ def aqua_prefill_workspace_size(cache: aqua_cache, Hq: int, L: int) -> int:
 
 
 def aqua_prefill_attn(cache: aqua_cache, q, pos0: int, L: int, P, Hq: int, k: int, out, workspace,
-                      scale: float = 0.0, sel_out=None, stream=None) -> None:
+                      scale: float = 0.0, sel_out=None, qproj_out=None, stream=None) -> None:
     out_dtype = AQUA_BF16 if str(out.dtype) == "torch.bfloat16" else AQUA_F32
     _check(load_library().aqua_prefill_attn(
         ctypes.byref(cache), _ptr(q), pos0, L, _ptr(P), Hq, k, scale, _ptr(out), out_dtype, _ptr(sel_out),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+        _ptr(qproj_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def aqua_h2o_update(cache: aqua_cache, scores, lse, Hq: int, budget: int, recent: int, evicted_out=None,

@@ -6,7 +6,10 @@
 #include <cstdio>
 
 #include <cudaTypedefs.h>
+#include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "aqua_internal.cuh"
 
@@ -22,6 +25,8 @@ int set_error(int code, const char* fmt, ...) {
   return code;
 }
 
+void clear_error() { g_err[0] = '\0'; }
+
 int check_launch(const char* what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -31,12 +36,32 @@ int check_launch(const char* what) {
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  static int cache[64] = {0};
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  static std::atomic<int> cache[64];
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 148;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+int set_smem_limit(const void* kernel, int bytes, const char* name) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "%s: cudaGetDevice: %s", name, cudaGetErrorString(e));
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> limit_set;   // (kernel, device) -> bytes
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(kernel, dev);
+  const auto it = limit_set.find(key);
+  if (it != limit_set.end() && it->second >= bytes) return AQUA_OK;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess)
+    return set_error(AQUA_ERR_CUDA, "cudaFuncSetAttribute(%s, %d bytes): %s", name, bytes, cudaGetErrorString(e));
+  limit_set[key] = bytes;
+  return AQUA_OK;
 }
 
 namespace {
@@ -87,13 +112,10 @@ int encode_tmap_bf16_3d(CUtensorMap* map, const void* base, const uint64_t dims[
 // launchers (defined next to their kernels)
 int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
                         cudaStream_t st);
-size_t decode_workspace_bytes(int n_units, int G);
-int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale,
-                  void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
-                  float* lse_out, const void* k_new, const void* v_new, void* ws, cudaStream_t st);
 size_t prefill_workspace_bytes(const aqua_cache* c, int Hq, int L);
 int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const float* P, int Hq, int k,
-                   float scale, void* out, int out_dtype, int32_t* sel_out, void* ws, cudaStream_t st);
+                   float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out, void* ws,
+                   cudaStream_t st);
 int launch_h2o_update(aqua_cache* c, const float* scores, const float* lse, int Hq, int budget, int recent,
                       int32_t* evicted_out, cudaStream_t st);
 size_t calibrate_workspace_bytes(int n, int d);
@@ -136,13 +158,68 @@ int check_out_dtype(int out_dtype) {
   return AQUA_OK;
 }
 
+// Head grouping shared by every decode entry point.
+int check_heads(const aqua_cache* c, int Hq, const char* who) {
+  if (Hq < 1 || Hq % c->Hkv != 0)
+    return set_error(AQUA_ERR_ARG, "%s: Hq=%d not a multiple of Hkv=%d", who, Hq, c->Hkv);
+  const int G = Hq / c->Hkv;
+  if (G != 1 && G != 2 && G != 4) return set_error(AQUA_ERR_UNSUPPORTED, "%s: Hq/Hkv=%d not in {1,2,4}", who, G);
+  return AQUA_OK;
+}
+
+// Arguments of the selection phase (query projection, top-k, optional append).
+int check_select_args(const aqua_cache* c, const aqua::DecodeArgs& a, const char* who) {
+  if (a.q == nullptr || a.P == nullptr) return set_error(AQUA_ERR_ARG, "%s: NULL q or P", who);
+  if (a.k < 1 || a.k > c->d_store)
+    return set_error(AQUA_ERR_ARG, "%s: k=%d outside [1, d_store=%d]", who, a.k, c->d_store);
+  if (!aligned(a.q, 16) || !aligned(a.P, 16)) return set_error(AQUA_ERR_ARG, "%s: q, P must be 16-byte aligned", who);
+  if ((a.k_new == nullptr) != (a.v_new == nullptr))
+    return set_error(AQUA_ERR_ARG, "%s: k_new and v_new must both be given or both be NULL", who);
+  if (a.k_new != nullptr) {
+    if ((long long)c->max_len + 1 > c->Tcap)
+      return set_error(AQUA_ERR_ARG, "%s: appending to a full cache (max_len %d, Tcap %d)", who, c->max_len, c->Tcap);
+    if (!aligned(a.k_new, 16) || !aligned(a.v_new, 16))
+      return set_error(AQUA_ERR_ARG, "%s: k_new, v_new must be 16-byte aligned", who);
+  }
+  return AQUA_OK;
+}
+
+// Arguments of the attention phase (output, optional scores and lse).
+int check_attend_args(const aqua::DecodeArgs& a, const char* who) {
+  int rc = check_out_dtype(a.out_dtype);
+  if (rc != AQUA_OK) return rc;
+  if (a.out == nullptr) return set_error(AQUA_ERR_ARG, "%s: NULL out", who);
+  if (!aligned(a.out, 16)) return set_error(AQUA_ERR_ARG, "%s: out must be 16-byte aligned", who);
+  return AQUA_OK;
+}
+
+int check_workspace(const aqua_cache* c, int Hq, const void* ws, size_t ws_bytes, const char* who) {
+  if (ws == nullptr) return set_error(AQUA_ERR_ARG, "%s: NULL workspace", who);
+  if (!aligned(ws, 256)) return set_error(AQUA_ERR_ARG, "%s: workspace must be 256-byte aligned", who);
+  const size_t need = aqua::decode_workspace_bytes(c->B * c->Hkv, Hq / c->Hkv);
+  if (ws_bytes < need) return set_error(AQUA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws_bytes, need);
+  return AQUA_OK;
+}
+
 }  // namespace
+
+namespace aqua {
+// Every argument check of aqua_decode_attn except the workspace; also used by
+// aqua_decode_attn_static, so both reject the same calls with the same codes.
+int check_decode_args(const aqua_cache* c, const DecodeArgs& a, const char* who) {
+  int rc = validate_cache(c);
+  if (rc == AQUA_OK) rc = check_heads(c, a.Hq, who);
+  if (rc == AQUA_OK) rc = check_attend_args(a, who);
+  if (rc == AQUA_OK) rc = check_select_args(c, a, who);
+  return rc;
+}
+}  // namespace aqua
 
 extern "C" {
 
 const char* aqua_last_error(void) { return aqua::g_err; }
 
-int aqua_version(void) { return 2; }
+int aqua_version(void) { return 3; }
 
 int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream) {
   if (cache == nullptr || cache->ctrl == nullptr || status_out == nullptr)
@@ -209,37 +286,53 @@ int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_new, const 
                      float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
                      aqua_stream_t stream) {
   aqua::g_err[0] = '\0';
-  int rc = validate_cache(cache);
+  aqua::DecodeArgs a;
+  a.q = q; a.k_new = k_new; a.v_new = v_new; a.P = P; a.Hq = Hq; a.k = k; a.scale = scale;
+  a.out = out; a.out_dtype = out_dtype; a.sel_out = sel_out; a.qproj_out = qproj_out;
+  a.scores_out = scores_out; a.lse_out = lse_out; a.ws = workspace; a.appended = k_new != nullptr;
+  int rc = aqua::check_decode_args(cache, a, "aqua_decode_attn");
+  if (rc == AQUA_OK) rc = check_workspace(cache, Hq, workspace, workspace_bytes, "aqua_decode_attn");
   if (rc != AQUA_OK) return rc;
-  if ((rc = check_out_dtype(out_dtype)) != AQUA_OK) return rc;
-  if (q == nullptr || P == nullptr || out == nullptr || workspace == nullptr)
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: NULL q, P, out or workspace");
-  if (Hq < 1 || Hq % cache->Hkv != 0)
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: Hq=%d not a multiple of Hkv=%d", Hq, cache->Hkv);
-  const int G = Hq / cache->Hkv;
-  if (G != 1 && G != 2 && G != 4)
-    return set_error(AQUA_ERR_UNSUPPORTED, "aqua_decode_attn: Hq/Hkv=%d not in {1,2,4}", G);
-  if (k < 1 || k > cache->d_store)
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k=%d outside [1, d_store=%d]", k, cache->d_store);
-  if (!aligned(q, 16) || !aligned(P, 16) || !aligned(out, 16) || !aligned(workspace, 256))
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: q, P, out 16-byte and workspace 256-byte alignment required");
-  const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, G);
-  if (workspace_bytes < need)
-    return set_error(AQUA_ERR_WORKSPACE, "aqua_decode_attn: workspace %zu < %zu bytes", workspace_bytes, need);
-  if ((k_new == nullptr) != (v_new == nullptr))
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k_new and v_new must both be given or both be NULL");
-  if (k_new != nullptr) {
-    if ((long long)cache->max_len + 1 > cache->Tcap)
-      return set_error(AQUA_ERR_ARG, "aqua_decode_attn: appending to a full cache (max_len %d, Tcap %d)",
-                       cache->max_len, cache->Tcap);
-    if (!aligned(k_new, 16) || !aligned(v_new, 16))
-      return set_error(AQUA_ERR_ARG, "aqua_decode_attn: k_new, v_new must be 16-byte aligned");
-  }
-  if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)cache->d);
-  rc = aqua::launch_decode(cache, q, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, scores_out, lse_out,
-                           k_new, v_new, workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt((float)cache->d);
+  rc = aqua::launch_decode(cache, a, aqua::kPhaseSelect | aqua::kPhaseAttend, reinterpret_cast<cudaStream_t>(stream));
   if (rc == AQUA_OK && k_new != nullptr) cache->max_len += 1;
   return rc;
+}
+
+int aqua_decode_select(aqua_cache* cache, const void* q, const void* k_new, const void* v_new, const float* P,
+                       int Hq, int k, float scale, int32_t* sel_out, float* qproj_out, void* workspace,
+                       size_t workspace_bytes, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  aqua::DecodeArgs a;
+  a.q = q; a.k_new = k_new; a.v_new = v_new; a.P = P; a.Hq = Hq; a.k = k; a.scale = scale;
+  a.sel_out = sel_out; a.qproj_out = qproj_out; a.ws = workspace; a.appended = k_new != nullptr;
+  int rc = validate_cache(cache);
+  if (rc == AQUA_OK) rc = check_heads(cache, Hq, "aqua_decode_select");
+  if (rc == AQUA_OK) rc = check_select_args(cache, a, "aqua_decode_select");
+  if (rc == AQUA_OK) rc = check_workspace(cache, Hq, workspace, workspace_bytes, "aqua_decode_select");
+  if (rc != AQUA_OK) return rc;
+  if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt((float)cache->d);
+  rc = aqua::launch_decode(cache, a, aqua::kPhaseSelect, reinterpret_cast<cudaStream_t>(stream));
+  if (rc == AQUA_OK && k_new != nullptr) cache->max_len += 1;
+  return rc;
+}
+
+int aqua_decode_attend(aqua_cache* cache, int Hq, int appended, void* out, int out_dtype, float* scores_out,
+                       float* lse_out, void* workspace, size_t workspace_bytes, aqua_stream_t stream) {
+  aqua::g_err[0] = '\0';
+  aqua::DecodeArgs a;
+  a.Hq = Hq; a.out = out; a.out_dtype = out_dtype; a.scores_out = scores_out; a.lse_out = lse_out;
+  a.ws = workspace; a.appended = appended;
+  int rc = validate_cache(cache);
+  if (rc == AQUA_OK) rc = check_heads(cache, Hq, "aqua_decode_attend");
+  if (rc == AQUA_OK) rc = check_attend_args(a, "aqua_decode_attend");
+  if (rc == AQUA_OK && appended != 0 && appended != 1)
+    rc = set_error(AQUA_ERR_ARG, "aqua_decode_attend: appended=%d (0 or 1)", appended);
+  if (rc == AQUA_OK && appended && cache->max_len < 1)
+    rc = set_error(AQUA_ERR_ARG, "aqua_decode_attend: appended=1 with max_len 0 (no selection appended a token)");
+  if (rc == AQUA_OK) rc = check_workspace(cache, Hq, workspace, workspace_bytes, "aqua_decode_attend");
+  if (rc != AQUA_OK) return rc;
+  return aqua::launch_decode(cache, a, aqua::kPhaseAttend, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L) {
@@ -248,7 +341,7 @@ size_t aqua_prefill_workspace_size(const aqua_cache* cache, int Hq, int L) {
 }
 
 int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, const float* P, int Hq, int k,
-                      float scale, void* out, int out_dtype, int32_t* sel_out, void* workspace,
+                      float scale, void* out, int out_dtype, int32_t* sel_out, float* qproj_out, void* workspace,
                       size_t workspace_bytes, aqua_stream_t stream) {
   aqua::g_err[0] = '\0';
   int rc = validate_cache(cache);
@@ -263,13 +356,14 @@ int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, c
     return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: k=%d outside [1, d_store=%d]", k, cache->d_store);
   if (L < 1 || pos0 < 0 || (long long)pos0 + L > cache->Tcap)
     return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: pos0=%d L=%d outside Tcap=%d", pos0, L, cache->Tcap);
-  if (!aligned(q, 16) || !aligned(P, 16) || !aligned(out, 16) || !aligned(workspace, 256))
-    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: alignment");
+  if (!aligned(q, 16) || !aligned(P, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+      !aligned(qproj_out, 16))
+    return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: q, P, out, qproj_out 16-byte and workspace 256-byte alignment required");
   const size_t need = aqua::prefill_workspace_bytes(cache, Hq, L);
   if (workspace_bytes < need)
     return set_error(AQUA_ERR_WORKSPACE, "aqua_prefill_attn: workspace %zu < %zu bytes", workspace_bytes, need);
   if (!(scale > 0.f)) scale = 1.0f / std::sqrt((float)cache->d);
-  return aqua::launch_prefill(cache, q, pos0, L, P, Hq, k, scale, out, out_dtype, sel_out, workspace,
+  return aqua::launch_prefill(cache, q, pos0, L, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, workspace,
                               reinterpret_cast<cudaStream_t>(stream));
 }
 

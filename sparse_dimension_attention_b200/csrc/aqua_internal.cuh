@@ -24,8 +24,42 @@ enum CtrlWord { kCtrlStatus = 0, kCtrlAppendTicket = 1, kCtrlH2OTicket = 2, kCtr
 
 // ---------------------------------------------------------------- host side errors
 int set_error(int code, const char* fmt, ...);
+void clear_error();   // empties the thread's last-error text (at the start of each entry point)
 int check_launch(const char* what);
 int device_sm_count();
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the CURRENT device.
+// cudaFuncSetAttribute acts per device, so the library records, per (kernel,
+// device), the limit already set (thread-safe); later calls cost one lookup.
+int set_smem_limit(const void* kernel, int bytes, const char* name);
+template <typename... KArgs>
+int set_smem_limit(void (*kernel)(KArgs...), int bytes, const char* name) {
+  return set_smem_limit(reinterpret_cast<const void*>(kernel), bytes, name);
+}
+
+// Arguments of a decode step (aqua_decode_attn, or its two phases
+// aqua_decode_select / aqua_decode_attend; see include/aqua.h).
+struct DecodeArgs {
+  const void* q = nullptr;
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const float* P = nullptr;
+  int Hq = 0, k = 0;
+  float scale = 0.f;
+  void* out = nullptr;
+  int out_dtype = 0;
+  int32_t* sel_out = nullptr;
+  float* qproj_out = nullptr;
+  float* scores_out = nullptr;
+  float* lse_out = nullptr;
+  void* ws = nullptr;
+  int appended = 0;   // the step appends its token (k_new/v_new given to the selection phase)
+};
+enum DecodePhase { kPhaseSelect = 1, kPhaseAttend = 2 };
+size_t decode_workspace_bytes(int n_units, int G);
+// Every host-side argument check of a whole decode step except the workspace
+// (AQUA_OK or the status, with the message set).
+int check_decode_args(const aqua_cache* c, const DecodeArgs& a, const char* who);
+int launch_decode(const aqua_cache* c, const DecodeArgs& a, int phases, cudaStream_t st);
 // 2-D tiled tensor map over a row-major bf16 matrix [rows][cols] (cols contiguous,
 // row stride in bytes), box [box_rows][box_cols]; swizzle128 selects the 128-byte
 // shared-memory swizzle.  Returns AQUA_OK or AQUA_ERR_CUDA.

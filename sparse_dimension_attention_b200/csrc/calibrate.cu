@@ -223,12 +223,7 @@ int launch_calibrate(const float* X, int n, float* P_out, float* sigma_out, void
   gram_sum_kernel<<<D, D, 0, st>>>(part, nb, A);
   if ((rc = check_launch("gram_sum_kernel")) != AQUA_OK) return rc;
   const int smem = D * LDA * (int)sizeof(double);
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(jacobi_kernel)");
-    configured = true;
-  }
+  if ((rc = set_smem_limit(jacobi_kernel, smem, "jacobi_kernel")) != AQUA_OK) return rc;
   jacobi_kernel<<<1, kJacobiThreads, smem, st>>>(A, V, P_out, sigma_out);
   return check_launch("jacobi_kernel");
 }

@@ -125,6 +125,22 @@ __device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, flo
     static_cast<float*>(p.out)[idx] = v;
 }
 
+// Sequences with no tokens have no tiles: attention over zero tokens is the
+// empty sum, output 0 and lse = -inf.  The attention CTAs share these units
+// (unit u goes to CTA u mod grid).  Only steps without an append can meet one.
+template <int G>
+__device__ __forceinline__ void write_empty_units(const DecodeParams& p) {
+  if (p.len_add != 0) return;
+  const int n_units = p.B * p.Hkv;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const int b = u / p.Hkv;
+    if (seq_len(p.len, b, p.Tcap) > 0) continue;
+    const size_t bhq0 = (size_t)b * p.Hq + (size_t)(u % p.Hkv) * G;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_val(p, bhq0 * D + i, 0.f);
+    if (p.lse_out != nullptr && threadIdx.x < G) p.lse_out[bhq0 + threadIdx.x] = -INFINITY;
+  }
+}
+
 // ============================================================================
 // query projection + magnitude top-k + group union
 // ============================================================================
@@ -322,11 +338,6 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
   if (p.qproj_out) p.qproj_out[bh * D + i] = qt;
   qs[hw][i] = keep ? qt * p.scale_log2 : 0.f;
 
-  // sequences with no tokens: zero output, lse = -inf
-  if (sl == 0 && !append && seq_len(p.len, b, p.Tcap) <= 0) {
-    for (int j = lane; j < D; j += 32) store_val(p, bh * D + j, 0.f);
-    if (p.lse_out && lane == 0) p.lse_out[bh] = -INFINITY;
-  }
   named_bar_sync(1, NPT);
 
   if (p.sel_out && keep) {                      // kept dims of the head in ascending order
@@ -830,6 +841,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   }
   pdl_launch_dependents();
   pdl_wait();   // the projection kernel (and its append) must be complete
+  write_empty_units<G>(p);
   if (!has_work) {
     if (tid == 0) step_done(p);
     return;
@@ -1223,6 +1235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
   }
   pdl_launch_dependents();
   pdl_wait();
+  write_empty_units<G>(p);
   Sched Sd;
   if (!make_schedule<TT, NTHREADS>(p, sch + 8, sch, Sd)) {
     if (tid == 0) step_done(p);
@@ -1485,15 +1498,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 // host launch
 // ============================================================================
 template <typename T, int G, int MINB>
-cudaError_t launch_qproj_variant(const DecodeParams& p, int n_units, int smem, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(qproj_topk_kernel<T, G, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  return launch_pdl(qproj_topk_kernel<T, G, MINB>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), smem, st, p);
+int launch_qproj_variant(const DecodeParams& p, int n_units, int smem, cudaStream_t st) {
+  const int rc = set_smem_limit(qproj_topk_kernel<T, G, MINB>, smem, "qproj_topk_kernel");
+  if (rc != AQUA_OK) return rc;
+  const cudaError_t e =
+      launch_pdl(qproj_topk_kernel<T, G, MINB>, dim3(n_units), dim3(QprojCfg<G>::WARPS * 32), smem, st, p);
+  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
+  return check_launch("qproj_topk_kernel");
 }
 
 template <typename T, int G>
@@ -1504,56 +1515,50 @@ int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
   // With more units, two CTAs share each SM (registers capped to fit), rather
   // than a second wave.
   constexpr int kOwnSm = 116 * 1024;
-  const cudaError_t e = n_units <= device_sm_count()
-                            ? launch_qproj_variant<T, G, 1>(p, n_units, kOwnSm, st)
-                            : launch_qproj_variant<T, G, 2>(p, n_units, D * D * 4, st);
-  if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "qproj_topk_kernel: %s", cudaGetErrorString(e));
-  return check_launch("qproj_topk_kernel");
+  return n_units <= device_sm_count() ? launch_qproj_variant<T, G, 1>(p, n_units, kOwnSm, st)
+                                      : launch_qproj_variant<T, G, 2>(p, n_units, D * D * 4, st);
 }
 
 template <int G>
-int launch_decode_bf16(const aqua_cache* c, const DecodeParams& p, int n_units, int C, cudaStream_t st) {
+int launch_attn_bf16(const aqua_cache* c, const DecodeParams& p, int C, cudaStream_t st) {
   using S = SmemBF16<G>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(decode_attn_bf16_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES) !=
-        cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(decode_attn_bf16_kernel)");
-    configured = true;
-  }
+  int rc = set_smem_limit(decode_attn_bf16_kernel<G>, S::BYTES, "decode_attn_bf16_kernel");
+  if (rc != AQUA_OK) return rc;
   // The tensor map depends only on the V buffer and its row count; reuse the
   // last encoding while they are unchanged (encoding costs host time every step).
   static thread_local const void* last_base = nullptr;
   static thread_local uint64_t last_rows = 0;
   static thread_local CUtensorMap tmap;
   const uint64_t rows = (uint64_t)c->B * c->Hkv * c->Tcap;
-  int rc = AQUA_OK;
   if (last_base != c->v || last_rows != rows) {
     if ((rc = encode_tmap_bf16_2d(&tmap, c->v, D, rows, D * 2, 64, S::TT, true)) != AQUA_OK) return rc;
     last_base = c->v;
     last_rows = rows;
   }
-  if ((rc = launch_qproj<__nv_bfloat16, G>(p, n_units, st)) != AQUA_OK) return rc;
   const cudaError_t e = launch_pdl(decode_attn_bf16_kernel<G>, dim3(C), dim3(NTHREADS_BF16), S::BYTES, st, tmap, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_bf16_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attn_bf16_kernel");
 }
 
 template <int G>
-int launch_decode_f32(const DecodeParams& p, int n_units, int C, cudaStream_t st) {
+int launch_attn_f32(const DecodeParams& p, int C, cudaStream_t st) {
   using S = SmemF32<G>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(decode_attn_f32_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES) !=
-        cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(decode_attn_f32_kernel)");
-    configured = true;
-  }
-  int rc = launch_qproj<float, G>(p, n_units, st);
+  const int rc = set_smem_limit(decode_attn_f32_kernel<G>, S::BYTES, "decode_attn_f32_kernel");
   if (rc != AQUA_OK) return rc;
   const cudaError_t e = launch_pdl(decode_attn_f32_kernel<G>, dim3(C), dim3(NTHREADS), S::BYTES, st, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_f32_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attn_f32_kernel");
+}
+
+template <int G>
+int launch_phases(const aqua_cache* c, const DecodeParams& p, int n_units, int C, int phases, cudaStream_t st) {
+  const bool bf = c->dtype == AQUA_BF16;
+  int rc = AQUA_OK;
+  if (phases & kPhaseSelect)
+    rc = bf ? launch_qproj<__nv_bfloat16, G>(p, n_units, st) : launch_qproj<float, G>(p, n_units, st);
+  if (rc == AQUA_OK && (phases & kPhaseAttend))
+    rc = bf ? launch_attn_bf16<G>(c, p, C, st) : launch_attn_f32<G>(p, C, st);
+  return rc;
 }
 
 }  // namespace
@@ -1572,13 +1577,14 @@ size_t decode_workspace_bytes(int n_units, int G) {
   return off;
 }
 
-int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale,
-                  void* out, int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out,
-                  float* lse_out, const void* k_new, const void* v_new, void* ws, cudaStream_t st) {
-  const int G = Hq / c->Hkv;
+// One decode step, or one of its phases: kPhaseSelect launches the projection
+// and selection kernel (with the fused append when a.k_new is given),
+// kPhaseAttend the attention kernel over the selection in the workspace.
+int launch_decode(const aqua_cache* c, const DecodeArgs& a, int phases, cudaStream_t st) {
+  const int G = a.Hq / c->Hkv;
   const int n_units = c->B * c->Hkv;
   DecodeParams p;
-  unsigned char* base = static_cast<unsigned char*>(ws);
+  unsigned char* base = static_cast<unsigned char*>(a.ws);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     void* ptr = base + off;
@@ -1593,21 +1599,21 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.counters = static_cast<int32_t*>(take((size_t)n_units * 4));
   p.part_ml = static_cast<float*>(take(nseg * G * 2 * 4));
   p.part_o = static_cast<float*>(take(nseg * G * D * 4));
-  p.q = q;
-  p.P = P;
+  p.q = a.q;
+  p.P = a.P;
   p.len = c->len;
   p.kproj = c->k_proj;
   p.v = c->v;
-  p.out = out;
-  p.sel_out = sel_out;
-  p.qproj_out = qproj_out;
-  p.scores_out = scores_out;
-  p.lse_out = lse_out;
+  p.out = a.out;
+  p.sel_out = a.sel_out;
+  p.qproj_out = a.qproj_out;
+  p.scores_out = a.scores_out;
+  p.lse_out = a.lse_out;
   p.ctrl = c->ctrl;
-  p.k_new = k_new;
-  p.v_new = v_new;
+  p.k_new = (phases & kPhaseSelect) ? a.k_new : nullptr;
+  p.v_new = (phases & kPhaseSelect) ? a.v_new : nullptr;
   p.len_w = c->len;
-  p.len_add = (k_new != nullptr) ? 1 : 0;
+  p.len_add = a.appended ? 1 : 0;
   // the projection kernel gives each of its CTAs an SM of its own when there
   // are no more units than SMs; that many attention CTAs then start late
   p.n_late = n_units <= device_sm_count() ? n_units : 0;
@@ -1615,25 +1621,27 @@ int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, in
   p.pos = c->pos;
   p.score = c->score;
   p.B = c->B;
-  p.Hq = Hq;
+  p.Hq = a.Hq;
   p.Hkv = c->Hkv;
   p.d_store = c->d_store;
   p.Tcap = c->Tcap;
-  p.k = k;
-  p.out_bf16 = out_dtype == AQUA_BF16;
-  p.scale_log2 = scale * kLog2e;
+  p.k = a.k;
+  p.out_bf16 = a.out_dtype == AQUA_BF16;
+  p.scale_log2 = a.scale * kLog2e;
   const bool bf = c->dtype == AQUA_BF16;
   const int TT = bf ? SmemBF16<1>::TT : SmemF32<1>::TT;
-  const int max_len = c->max_len + (k_new != nullptr ? 1 : 0);
+  // host bound of the tokens attended: the selection phase has not yet counted
+  // the token it appends in cache->max_len, the attention phase alone has
+  const int max_len = c->max_len + ((phases & kPhaseSelect) && a.appended ? 1 : 0);
   const long long tiles_ub = (long long)n_units * ((max_len + TT - 1) / TT);
   long long C = device_sm_count();
   if (C > tiles_ub) C = tiles_ub;
   if (C < 1) C = 1;
   if (C > kMaxCtas) C = kMaxCtas;
   switch (G) {
-    case 1: return bf ? launch_decode_bf16<1>(c, p, n_units, (int)C, st) : launch_decode_f32<1>(p, n_units, (int)C, st);
-    case 2: return bf ? launch_decode_bf16<2>(c, p, n_units, (int)C, st) : launch_decode_f32<2>(p, n_units, (int)C, st);
-    case 4: return bf ? launch_decode_bf16<4>(c, p, n_units, (int)C, st) : launch_decode_f32<4>(p, n_units, (int)C, st);
+    case 1: return launch_phases<1>(c, p, n_units, (int)C, phases, st);
+    case 2: return launch_phases<2>(c, p, n_units, (int)C, phases, st);
+    case 4: return launch_phases<4>(c, p, n_units, (int)C, phases, st);
     default: return set_error(AQUA_ERR_UNSUPPORTED, "decode: Hq/Hkv = %d not in {1,2,4}", G);
   }
 }

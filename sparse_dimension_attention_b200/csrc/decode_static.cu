@@ -28,11 +28,6 @@
 
 namespace aqua {
 
-size_t decode_workspace_bytes(int n_units, int G);
-int launch_decode(const aqua_cache* c, const void* q, const float* P, int Hq, int k, float scale, void* out,
-                  int out_dtype, int32_t* sel_out, float* qproj_out, float* scores_out, float* lse_out,
-                  const void* k_new, const void* v_new, void* ws, cudaStream_t st);
-
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
@@ -69,20 +64,25 @@ extern "C" int aqua_decode_attn_static(aqua_cache* cache, const void* q, const v
                                        int32_t* sel_out, float* qproj_out, float* scores_out, float* lse_out,
                                        aqua_stream_t stream) {
   using aqua::set_error;
-  // The same checks as aqua_decode_attn, which this forwards to with the
-  // built-in scratch in place of a workspace: first the size against the array.
-  if (cache == nullptr) return set_error(AQUA_ERR_ARG, "aqua_decode_attn_static: cache descriptor is NULL");
-  if (cache->Hkv < 1 || Hq < 1 || Hq % cache->Hkv != 0 || cache->B < 1)
-    return set_error(AQUA_ERR_ARG, "aqua_decode_attn_static: Hq=%d, Hkv=%d, B=%d", Hq, cache->Hkv, cache->B);
+  aqua::clear_error();
+  // Every argument check of aqua_decode_attn, in the same order and with the
+  // same status codes; then the scratch this shape needs against the array.
+  aqua::DecodeArgs a;
+  a.q = q; a.k_new = k_new; a.v_new = v_new; a.P = P; a.Hq = Hq; a.k = k; a.scale = scale;
+  a.out = out; a.out_dtype = out_dtype; a.sel_out = sel_out; a.qproj_out = qproj_out;
+  a.scores_out = scores_out; a.lse_out = lse_out; a.appended = k_new != nullptr;
+  int rc = aqua::check_decode_args(cache, a, "aqua_decode_attn_static");
+  if (rc != AQUA_OK) return rc;
   const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv);
   if (need > aqua::kStaticScratchBytes)
     return set_error(AQUA_ERR_WORKSPACE,
                      "aqua_decode_attn_static: this shape needs %zu bytes of scratch; the built-in array holds %zu "
                      "(use aqua_decode_attn with a workspace)",
                      need, aqua::kStaticScratchBytes);
-  void* ws = nullptr;
-  const int rc = aqua::static_scratch(&ws);
+  rc = aqua::static_scratch(&a.ws);
   if (rc != AQUA_OK) return rc;
-  return aqua_decode_attn(cache, q, k_new, v_new, P, Hq, k, scale, out, out_dtype, sel_out, qproj_out, scores_out,
-                          lse_out, ws, aqua::kStaticScratchBytes, stream);
+  if (!(a.scale > 0.f)) a.scale = 1.0f / std::sqrt((float)cache->d);
+  rc = aqua::launch_decode(cache, a, aqua::kPhaseSelect | aqua::kPhaseAttend, reinterpret_cast<cudaStream_t>(stream));
+  if (rc == AQUA_OK && k_new != nullptr) cache->max_len += 1;
+  return rc;
 }

@@ -136,6 +136,7 @@ struct PrefillParams {
   const float* P;            // [Hkv][D][D]
   void* out;                 // [B][L][Hq][D]
   int32_t* sel_out;          // nullable [B][L][Hq][k]
+  float* qproj_out;          // nullable [B][L][Hq][D]: the q~ the selection used
   int32_t* ctrl;
   int B, L, Hq, Hkv, d_store, Tcap, k, pos0;
   int out_bf16;
@@ -540,11 +541,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       if (ok) {
         // second pass over this half of q~ (still in TMEM): masked, scaled, split, K-major swizzled rows
+        float* qpo = (p.qproj_out != nullptr && live)
+                         ? p.qproj_out + (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * D + d0
+                         : nullptr;
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 32) {
           float v[32];
           tmem_ld32(tm_O + lane_base + d0 + c0, v);
           tmem_wait_ld();
+          if (qpo != nullptr) {                       // the exact f32 values the keys above came from
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(qpo + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          }
           const uint32_t word = selm[c0 >> 5];
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {            // 8 dims = one 16-byte chunk
@@ -719,19 +728,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 template <int G>
 int launch_prefill_g(const aqua_cache* c, const PrefillParams& p, const void* q, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(prefill_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::BYTES) !=
-        cudaSuccess)
-      return check_launch("cudaFuncSetAttribute(prefill)");
-    configured = true;
-  }
+  int rc = set_smem_limit(prefill_attn_kernel<G>, AttnSmem::BYTES, "prefill_attn_kernel");
+  if (rc != AQUA_OK) return rc;
   CUtensorMap tq, tk, tv;
   // q [B*L][Hq][D]: box {64 dims, G heads, 128/G positions} = the CTA's 128 rows in (position, head) order
   const uint64_t qdims[3] = {(uint64_t)D, (uint64_t)p.Hq, (uint64_t)p.B * p.L};
   const uint64_t qstr[2] = {(uint64_t)D * 2, (uint64_t)p.Hq * D * 2};
   const uint32_t qbox[3] = {64u, (uint32_t)G, (uint32_t)(PM / G)};
-  int rc = encode_tmap_bf16_3d(&tq, q, qdims, qstr, qbox, true);
+  rc = encode_tmap_bf16_3d(&tq, q, qdims, qstr, qbox, true);
   if (rc == AQUA_OK)
     rc = encode_tmap_bf16_2d(&tk, c->k_proj, (uint64_t)c->Tcap, (uint64_t)c->B * c->Hkv * c->d_store,
                              (uint64_t)c->Tcap * 2, 64, (uint32_t)c->d_store, true);
@@ -751,13 +755,14 @@ size_t prefill_workspace_bytes(const aqua_cache*, int, int) {
 }
 
 int launch_prefill(const aqua_cache* c, const void* q, int pos0, int L, const float* P, int Hq, int k, float scale,
-                   void* out, int out_dtype, int32_t* sel_out, void*, cudaStream_t st) {
+                   void* out, int out_dtype, int32_t* sel_out, float* qproj_out, void*, cudaStream_t st) {
   if (c->d_store % 16 != 0)
     return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: d_store %d must be a multiple of 16", c->d_store);
   PrefillParams p;
   p.P = P;
   p.out = out;
   p.sel_out = sel_out;
+  p.qproj_out = qproj_out;
   p.ctrl = c->ctrl;
   p.B = c->B;
   p.L = L;

@@ -149,13 +149,8 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
   dim3 grid((L + kTokPerCta - 1) / kTokPerCta, c->Hkv, c->B);
   const int smem = D * D * 4;
   if (c->dtype == AQUA_BF16) {
-    static bool configured = false;
-    if (!configured) {
-      if (cudaFuncSetAttribute(project_keys_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               smem) != cudaSuccess)
-        return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
-      configured = true;
-    }
+    const int rc = set_smem_limit(project_keys_kernel<__nv_bfloat16>, smem, "project_keys_kernel");
+    if (rc != AQUA_OK) return rc;
     const cudaError_t e = launch_pdl(
         project_keys_kernel<__nv_bfloat16>, grid, dim3(256), smem, st, static_cast<const __nv_bfloat16*>(k_new),
         static_cast<const __nv_bfloat16*>(v_new), P, static_cast<__nv_bfloat16*>(c->k_proj),
@@ -163,13 +158,8 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
         c->Tcap);
     if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "project_keys_kernel: %s", cudaGetErrorString(e));
   } else {
-    static bool configured = false;
-    if (!configured) {
-      if (cudaFuncSetAttribute(project_keys_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return check_launch("cudaFuncSetAttribute(project_keys_kernel)");
-      configured = true;
-    }
+    const int rc = set_smem_limit(project_keys_kernel<float>, smem, "project_keys_kernel");
+    if (rc != AQUA_OK) return rc;
     const cudaError_t e = launch_pdl(project_keys_kernel<float>, grid, dim3(256), smem, st,
                                      static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
                                      static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs,

@@ -49,7 +49,7 @@ def test_struct_layout():
 
 
 def test_version(lib):
-    assert aq.aqua_version() == 2
+    assert aq.aqua_version() == 3
 
 
 def _desc(**kw):
@@ -106,6 +106,53 @@ def test_decode_argument_checks(lib):
     assert full.max_len == 64
 
 
+def test_decode_phases_argument_checks(lib):
+    """aqua_decode_select / aqua_decode_attend check the arguments each one uses."""
+    c = _desc(max_len=10)
+    ws = lib.aqua_decode_workspace_size(ctypes.byref(c), 8)
+    sel = lambda **kw: lib.aqua_decode_select(
+        ctypes.byref(kw.get("c", c)), kw.get("q", 0x5000), kw.get("kn", None), kw.get("vn", None), 0x7000,
+        kw.get("Hq", 8), kw.get("k", 96), 0.0, None, None, kw.get("ws", 0x10000), kw.get("wsb", ws), None)
+    att = lambda **kw: lib.aqua_decode_attend(
+        ctypes.byref(kw.get("c", c)), kw.get("Hq", 8), kw.get("app", 0), kw.get("out", 0x8000),
+        kw.get("od", abi.AQUA_BF16), None, None, kw.get("ws", 0x10000), kw.get("wsb", ws), None)
+    assert sel(q=None) == abi.AQUA_ERR_ARG
+    assert sel(k=0) == abi.AQUA_ERR_ARG
+    assert sel(Hq=16) == abi.AQUA_ERR_UNSUPPORTED
+    assert sel(kn=0x9000) == abi.AQUA_ERR_ARG
+    assert sel(wsb=ws - 1) == abi.AQUA_ERR_WORKSPACE
+    assert att(app=2) == abi.AQUA_ERR_ARG
+    assert att(c=_desc(max_len=0), app=1) == abi.AQUA_ERR_ARG       # nothing was appended
+    assert att(out=None) == abi.AQUA_ERR_ARG
+    assert att(od=9) == abi.AQUA_ERR_UNSUPPORTED
+    assert att(Hq=7) == abi.AQUA_ERR_ARG
+    assert att(ws=0x10010) == abi.AQUA_ERR_ARG
+    assert c.max_len == 10
+
+
+def test_static_decode_checks_match_the_workspace_entry_point(lib):
+    """aqua_decode_attn_static rejects bad calls with aqua_decode_attn's codes,
+    before it compares the shape's scratch with its built-in array."""
+    def both(c, Hq, k=96, od=abi.AQUA_BF16, q=0x5000):
+        ws_call = lib.aqua_decode_attn(ctypes.byref(c), q, None, None, 0x7000, Hq, k, 0.0, 0x8000, od, None, None,
+                                       None, None, 0x10000, 1 << 40, None)
+        st_call = lib.aqua_decode_attn_static(ctypes.byref(c), q, None, None, 0x7000, Hq, k, 0.0, 0x8000, od, None,
+                                              None, None, None, None)
+        return ws_call, st_call
+    big = _desc(B=512, Hkv=8)
+    assert both(big, 64) == (abi.AQUA_ERR_UNSUPPORTED, abi.AQUA_ERR_UNSUPPORTED)   # group of 8, not scratch
+    assert both(big, 12) == (abi.AQUA_ERR_ARG, abi.AQUA_ERR_ARG)
+    assert both(big, 32, k=0) == (abi.AQUA_ERR_ARG, abi.AQUA_ERR_ARG)
+    assert both(big, 32, od=4) == (abi.AQUA_ERR_UNSUPPORTED, abi.AQUA_ERR_UNSUPPORTED)
+    assert both(_desc(d=64), 8) == (abi.AQUA_ERR_UNSUPPORTED, abi.AQUA_ERR_UNSUPPORTED)
+    assert both(big, 32, q=None) == (abi.AQUA_ERR_ARG, abi.AQUA_ERR_ARG)
+    # a valid call whose scratch exceeds the 8 MiB array
+    st = lib.aqua_decode_attn_static(ctypes.byref(big), 0x5000, None, None, 0x7000, 32, 96, 0.0, 0x8000,
+                                     abi.AQUA_BF16, None, None, None, None, None)
+    assert st == abi.AQUA_ERR_WORKSPACE
+    assert "8388608" in lib.aqua_last_error().decode()
+
+
 def test_decode_workspace_grows_with_units(lib):
     a = lib.aqua_decode_workspace_size(ctypes.byref(_desc(B=1, Hkv=1)), 4)
     b = lib.aqua_decode_workspace_size(ctypes.byref(_desc(B=8, Hkv=8)), 32)
@@ -136,10 +183,12 @@ def test_prefill_argument_checks(lib):
     c = _desc()
     ws = lib.aqua_prefill_workspace_size(ctypes.byref(c), 8, 32)
     assert lib.aqua_prefill_attn(ctypes.byref(c), 0x5000, 40, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
-                                 None, 0x10000, ws, None) == abi.AQUA_ERR_ARG   # pos0 + L > Tcap
+                                 None, None, 0x10000, ws, None) == abi.AQUA_ERR_ARG   # pos0 + L > Tcap
     c32 = _desc(dtype=abi.AQUA_F32)
     assert lib.aqua_prefill_attn(ctypes.byref(c32), 0x5000, 0, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
-                                 None, 0x10000, ws, None) == abi.AQUA_ERR_UNSUPPORTED
+                                 None, None, 0x10000, ws, None) == abi.AQUA_ERR_UNSUPPORTED
+    assert lib.aqua_prefill_attn(ctypes.byref(c), 0x5000, 0, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
+                                 None, 0x9004, 0x10000, ws, None) == abi.AQUA_ERR_ARG  # qproj_out misaligned
 
 
 def test_calibrate_argument_checks(lib):

@@ -290,3 +290,51 @@ def test_decode_bf16_more_units_than_sms():
     cache, res, ref, _ = _decode_case(B, 2 * Hkv, Hkv, max(lens) - 1, 48, lens=lens)
     _check_outputs(res, ref, "bf16", lens)
     check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 48)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_select_then_attend_equals_one_call(fused):
+    """aqua_decode_select + aqua_decode_attend (back to back, and with a
+    synchronisation between them) give bit-identical outputs, selections,
+    log-sum-exps and caches to aqua_decode_attn, with and without the fused
+    append of the step's token; one sequence is empty."""
+    B, Hq, Hkv, T, k = 3, 8, 2, 700, 64
+    P64, P32 = calib_P(Hkv)
+    inp = synth.decode_inputs(B, Hq, Hkv, T, bf16=True, steps=2)
+    caches = [aq.AquaCache(B, Hkv, 720) for _ in range(3)]
+    for c in caches:
+        Pt = fill_cache(c, inp["k_hist"], inp["v_hist"], P32)
+        if not fused:
+            c.len[1] = 0                                   # an empty sequence
+    res = []
+    for mode, c in enumerate(caches):
+        ws = torch.zeros(aq.aqua_decode_workspace_size(c.desc, Hq), dtype=torch.uint8, device="cuda")
+        r = []
+        for s in range(2):
+            q = tdev(inp["q"][s], torch.bfloat16)
+            kn = tdev(inp["k_new"][s], torch.bfloat16) if fused else None
+            vn = tdev(inp["v_new"][s], torch.bfloat16) if fused else None
+            out = torch.full((B, Hq, 128), 7.0, dtype=torch.float32, device="cuda")
+            lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+            sel = torch.empty((B, Hq, k), dtype=torch.int32, device="cuda")
+            if mode == 0:
+                aq.aqua_decode_attn(c.desc, q, Pt, Hq, k, out, ws, k_new=kn, v_new=vn, lse_out=lse, sel_out=sel)
+            else:
+                aq.aqua_decode_select(c.desc, q, Pt, Hq, k, ws, k_new=kn, v_new=vn, sel_out=sel)
+                if mode == 2:
+                    torch.cuda.synchronize()
+                aq.aqua_decode_attend(c.desc, Hq, out, ws, appended=fused, lse_out=lse)
+            r.append((out.clone(), lse.clone(), sel.clone()))
+        torch.cuda.synchronize()
+        res.append(r)
+    for mode in (1, 2):
+        for s in range(2):
+            for a, b in zip(res[0][s], res[mode][s]):
+                assert torch.equal(a, b), (mode, s)
+        for name in ("k_proj", "v", "len", "n_abs"):
+            assert torch.equal(getattr(caches[0], name), getattr(caches[mode], name)), name
+        assert caches[0].max_len == caches[mode].max_len
+    if not fused:
+        assert torch.all(res[1][1][0][1] == 0) and torch.all(torch.isneginf(res[1][1][1][1]))
+    for c in caches:
+        assert aq.aqua_status(c.desc) == aq.AQUA_OK

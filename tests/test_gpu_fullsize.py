@@ -19,7 +19,7 @@ import bench
 import synth
 from oracle import aqua_oracle as O
 import sparse_dimension_attention_b200 as aq
-from aqua_testlib import calib_P, rel_err_rows, tdev
+from aqua_testlib import calib_P, check_selection, rel_err_rows, tdev
 
 pytestmark = pytest.mark.gpu
 
@@ -122,6 +122,22 @@ def test_prompt_graph_last_chunk_sampled_rows(prompt, k):
         ref, _ = O.prefill(inp["q"][0, p:p + 1], p, P64, Kt, V, k, out_dtype="bf16")
         err = rel_err_rows(out[i], ref[0])
         assert np.max(err) <= TOL_BF16_OUT, (i, np.max(err))
+    # the last chunk once more, eagerly, exporting its selection and q~: the
+    # output is bit-identical to the graph's, and every (row, head) selection
+    # is exactly the oracle's on the kernel's own q~ (and on the f64 q~ away
+    # from near ties)
+    Hq, G = wl["Hq"], wl["Hq"] // wl["Hkv"]
+    o2 = torch.empty_like(pb.out)
+    sel = torch.full((1, C, Hq, k), -1, dtype=torch.int32, device="cuda")
+    qp = torch.empty((1, C, Hq, 128), dtype=torch.float32, device="cuda")
+    aq.aqua_prefill_attn(pb.cache.desc, pb.q[:, pos0:pos0 + C], pos0, C, pb.P, Hq, k, o2, pb.ws, sel_out=sel,
+                         qproj_out=qp)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, pb.out)
+    qt64 = np.einsum("lhi,hij->lhj", inp["q"][0, pos0:pos0 + C].astype(np.float64), P64[np.arange(Hq) // G])
+    ref_sel = np.stack([[O.select_dims(qt64[i, h], k) for h in range(Hq)] for i in range(C)])
+    near = check_selection(sel.cpu().numpy()[0], qp.cpu().numpy()[0], ref_sel, qt64, k)
+    assert near <= C * Hq // 1000, near
 
 
 def _h2o_oracle_state(inp, P64, b, Hkv, n0, m):
