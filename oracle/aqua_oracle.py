@@ -157,6 +157,18 @@ def default_scale(d: int) -> float:
 # ----------------------------------------------------------------------------
 # cache building and the decode / prefill steps
 # ----------------------------------------------------------------------------
+#
+# AQUA-Memory on the values.  The edgentiq blog ("AQUA-Memory: Dual Savings")
+# says the lowest-importance dimensions are dropped before the key AND value
+# vectors are stored.  The pages give no formula; the plainest reading, taken
+# here: values are projected by the same orthogonal P as the keys of their KV
+# head, the first m_v projected dimensions are stored, V^ = store((v P)[:m_v]),
+# and the attention output is brought back to the value space by the
+# transpose of those columns, o = (sum_t p_t V^_t) P[:, :m_v]^T.  With m_v = d
+# this is exactly the unpruned output (P P^T = I); for m_v < d it is the
+# unpruned output projected onto the span of P's first m_v columns (up to the
+# storage rounding of V^).  Without v_projected the values are unprojected,
+# as the workload statement asks for the main path.
 
 def build_key_cache(k, P, kv_dtype: str, m: int | None = None) -> np.ndarray:
     """Projected-key cache K~ = store(k P)[..., :m] for keys k [..., Hkv, d] and P [Hkv, d, d].
@@ -174,14 +186,36 @@ def build_key_cache(k, P, kv_dtype: str, m: int | None = None) -> np.ndarray:
     return store(kt[..., :m], kv_dtype)
 
 
+def build_value_cache(v, P, kv_dtype: str, m_v: int | None = None) -> np.ndarray:
+    """Pruned projected-value cache V^ = store((v P)[..., :m_v]) for values v [..., Hkv, d].
+
+    AQUA-Memory on the values (see the reading above): same P as the keys of
+    the KV head, the first m_v projected dimensions kept.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    P = np.asarray(P, dtype=np.float64)
+    m_v = v.shape[-1] if m_v is None else m_v
+    vt = np.einsum("...gi,gij->...gj", v, P)
+    return store(vt[..., :m_v], kv_dtype)
+
+
+def unproject_values(o_hat, P_g) -> np.ndarray:
+    """o = o^ P[:, :m_v]^T: an output over the m_v stored projected value
+    dimensions, brought back to the d value dimensions."""
+    o_hat = np.asarray(o_hat, dtype=np.float64)
+    m_v = o_hat.shape[-1]
+    return o_hat @ np.asarray(P_g, dtype=np.float64)[:, :m_v].T
+
+
 def decode(q, P, Kt, V, lens, k: int, scale: float | None = None, m: int | None = None,
-           out_dtype: str = "f64"):
+           out_dtype: str = "f64", v_projected: bool = False):
     """One AQUA decode step for every (sequence, query head).
 
     q   [B, Hq, d]          queries (their new keys are already in the cache);
     P   [Hkv, d, d]         projection per KV head (query head h uses P[h // G]);
     Kt  [B, Hkv, T, m]      projected-key cache (token-major), T >= lens[b];
-    V   [B, Hkv, T, d]      unprojected values;
+    V   [B, Hkv, T, d]      unprojected values, or with v_projected the pruned
+                            projected values V^ [B, Hkv, T, m_v] (build_value_cache);
     lens[B]                 visible tokens per sequence.
     Returns dict: out [B, Hq, d], sel [B, Hq, k], qt [B, Hq, d], lse [B, Hq],
     probs list-of-lists [b][h] -> [lens[b]].
@@ -203,6 +237,8 @@ def decode(q, P, Kt, V, lens, k: int, scale: float | None = None, m: int | None 
             g = h // G
             qt = project(q[b, h], P[g])
             o, p, l, S = attend_one(qt, k, Kt[b, g, :T], V[b, g, :T], scale, m)
+            if v_projected:
+                o = unproject_values(o, P[g])
             out[b, h], sel[b, h], qts[b, h], lse[b, h], probs[b][h] = o, S, qt, l, p
     if out_dtype == "bf16":
         out = round_bf16(out)
@@ -212,10 +248,11 @@ def decode(q, P, Kt, V, lens, k: int, scale: float | None = None, m: int | None 
 
 
 def prefill(q, pos0: int, P, Kt, V, k: int, scale: float | None = None, m: int | None = None,
-            out_dtype: str = "f64"):
+            out_dtype: str = "f64", v_projected: bool = False):
     """Causal AQUA attention for a chunk of queries at absolute positions pos0 .. pos0+L-1.
 
-    q [L, Hq, d]; Kt [Hkv, >= pos0+L, m]; V [Hkv, >= pos0+L, d] (one sequence).
+    q [L, Hq, d]; Kt [Hkv, >= pos0+L, m]; V [Hkv, >= pos0+L, d] (one sequence),
+    or with v_projected the pruned projected values [Hkv, >= pos0+L, m_v].
     Row i sees tokens 0 .. pos0+i.  Each (row, head) selects its own k
     dimensions, exactly as a decode step at that position would.
     Returns (out [L, Hq, d], sel [L, Hq, k]).
@@ -234,6 +271,8 @@ def prefill(q, pos0: int, P, Kt, V, k: int, scale: float | None = None, m: int |
             g = h // G
             qt = project(q[i, h], P[g])
             o, _, _, S = attend_one(qt, k, Kt[g, :T], V[g, :T], scale, m)
+            if v_projected:
+                o = unproject_values(o, P[g])
             out[i, h], sel[i, h] = o, S
     if out_dtype == "bf16":
         out = round_bf16(out)
@@ -282,11 +321,13 @@ class H2OSeq:
 
 
 def h2o_decode_step(seqs, q_b, k_new_b, v_new_b, t_abs: int, P, k: int, budget: int, recent: int,
-                    kv_dtype: str, m: int | None = None, scale: float | None = None):
+                    kv_dtype: str, m: int | None = None, scale: float | None = None, m_v: int | None = None):
     """One decode step of one sequence with H2O eviction.
 
     seqs: list over KV heads of H2OSeq (modified in place); q_b [Hq, d];
     k_new_b, v_new_b [Hkv, d]; the new token has absolute position t_abs.
+    With m_v the values are kept as pruned projected values (AQUA-Memory on
+    the values; the retained rows in seqs are then V^ rows).
     Returns out [Hq, d] (float64) and the evicted positions per KV head.
     """
     q_b = np.asarray(q_b, dtype=np.float64)
@@ -303,14 +344,17 @@ def h2o_decode_step(seqs, q_b, k_new_b, v_new_b, t_abs: int, P, k: int, budget: 
         s.pos.append(t_abs)
         s.score.append(0.0)
         s.kt.append(kt_new)
-        s.v.append(np.asarray(v_new_b[g], dtype=np.float64))
+        if m_v is None:
+            s.v.append(np.asarray(v_new_b[g], dtype=np.float64))
+        else:
+            s.v.append(store(project(v_new_b[g], P[g])[:m_v], kv_dtype))
         Kt = np.array(s.kt)
         Vv = np.array(s.v)
         acc = np.zeros(len(s.pos))
         for h in range(g * G, (g + 1) * G):
             qt = project(q_b[h], P[g])
             o, p, _, _ = attend_one(qt, k, Kt, Vv, scale, m)
-            out[h] = o
+            out[h] = o if m_v is None else unproject_values(o, P[g])
             acc += p
         for i in range(len(s.pos)):
             s.score[i] += acc[i]

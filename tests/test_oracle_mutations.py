@@ -52,6 +52,17 @@ MUTANTS = [
      "recent window one token long"),
     ("h2o_decode_step", "acc += p", "acc = p", "score of the last head only"),
     ("h2o_decode_step", "s.score[i] += acc[i]", "s.score[i] = acc[i]", "score not cumulative"),
+    ("build_value_cache", "return store(vt[..., :m_v], kv_dtype)",
+     "return store(vt[..., v.shape[-1] - m_v:], kv_dtype)", "trailing value dimensions kept"),
+    ("build_value_cache", 'np.einsum("...gi,gij->...gj", v, P)', 'np.einsum("...gi,gji->...gj", v, P)',
+     "values projected by the transpose of P"),
+    ("build_value_cache", "return store(vt[..., :m_v], kv_dtype)", "return store(v[..., :m_v], kv_dtype)",
+     "values pruned without the projection"),
+    ("unproject_values", "[:, :m_v].T", "[:m_v, :]", "back-projection by rows of P instead of columns"),
+    ("decode", "o = unproject_values(o, P[g])", "o = unproject_values(o, P[0])",
+     "back-projection with another KV head's P"),
+    ("h2o_decode_step", "unproject_values(o, P[g])", "unproject_values(o, P[0])",
+     "H2O back-projection with another KV head's P"),
     ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * d * 1.0", "break-even without the key projection share"),
     ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * k * (1.0 + 1.0 / G)",
      "break-even with d k instead of d^2 projection work"),

@@ -263,6 +263,110 @@ def test_truncated_cache_build_and_decode_keep_the_leading_dims():
     np.testing.assert_array_equal(O.build_key_cache(kk, P[None], "f64", d), O.build_key_cache(kk, P[None], "f64"))
 
 
+# --------------------------------------------------------------------------- value pruning (AQUA-Memory)
+
+def _vp_case(seed, Hq=4, Hkv=2, T=50, d=128):
+    rng = np.random.default_rng(seed)
+    P = np.stack([_rand_orthogonal(d, seed + 1 + g) for g in range(Hkv)])
+    q = rng.standard_normal((1, Hq, d))
+    kk = rng.standard_normal((1, T, Hkv, d))
+    vv = rng.standard_normal((1, T, Hkv, d))
+    Kt = O.build_key_cache(kk, P, "f64").transpose(0, 2, 1, 3)
+    return P, q, kk, vv, Kt
+
+
+def _vp_decode(P, q, Kt, vv, m_v, k=64, store="f64"):
+    Vh = O.build_value_cache(vv, P, store, m_v).transpose(0, 2, 1, 3)
+    assert Vh.shape[-1] == m_v
+    return O.decode(q, P, Kt, Vh, [vv.shape[1]], k, v_projected=True)
+
+
+def test_value_pruning_at_full_width_is_the_unpruned_output():
+    """m_v = d: V P P^T = V for orthogonal P, so projecting the values and
+    bringing the output back changes nothing."""
+    P, q, kk, vv, Kt = _vp_case(30)
+    plain = O.decode(q, P, Kt, vv.transpose(0, 2, 1, 3), [vv.shape[1]], 64)
+    pruned = _vp_decode(P, q, Kt, vv, 128)
+    np.testing.assert_allclose(pruned["out"], plain["out"], rtol=1e-12, atol=1e-13)
+
+
+def test_value_pruning_projects_the_output_onto_the_kept_subspace():
+    """By linearity, pruning every value to the span of P's first m_v columns
+    and summing equals summing first and projecting the unpruned output onto
+    that span: o_pruned = o P_m P_m^T (computed here the other way round, from
+    the unpruned decode).  The probabilities do not depend on the values."""
+    P, q, kk, vv, Kt = _vp_case(31)
+    plain = O.decode(q, P, Kt, vv.transpose(0, 2, 1, 3), [vv.shape[1]], 64)
+    G = q.shape[1] // P.shape[0]
+    for m_v in (96, 64, 1):
+        pruned = _vp_decode(P, q, Kt, vv, m_v)
+        for h in range(q.shape[1]):
+            Pm = P[h // G][:, :m_v]
+            expect = (plain["out"][0, h] @ Pm) @ Pm.T
+            np.testing.assert_allclose(pruned["out"][0, h], expect, rtol=1e-11, atol=1e-12)
+        np.testing.assert_array_equal(pruned["sel"], plain["sel"])
+        np.testing.assert_allclose(pruned["lse"], plain["lse"], rtol=1e-14)
+
+
+def test_value_pruning_sign_invariance():
+    """Flipping the sign of columns of P flips the same stored value
+    dimensions and their back-projection columns: the output is unchanged."""
+    P, q, kk, vv, Kt = _vp_case(32)
+    P2 = P.copy()
+    P2[:, :, [0, 3, 70, 95, 100]] *= -1
+    Kt2 = O.build_key_cache(kk, P2, "f64").transpose(0, 2, 1, 3)
+    a = _vp_decode(P, q, Kt, vv, 96)
+    b = _vp_decode(P2, q, Kt2, vv, 96)
+    np.testing.assert_allclose(b["out"], a["out"], rtol=1e-12, atol=1e-13)
+
+
+def test_value_pruning_is_lossless_for_values_in_the_kept_subspace():
+    """Values built inside the span of each KV head's first m_v columns of P
+    lose nothing: the pruned output equals the unpruned one."""
+    P, q, kk, _, Kt = _vp_case(33)
+    m_v = 80
+    coeff = np.random.default_rng(34).standard_normal((1, kk.shape[1], P.shape[0], m_v))
+    vv = np.einsum("btgj,gij->btgi", coeff, P[:, :, :m_v])
+    plain = O.decode(q, P, Kt, vv.transpose(0, 2, 1, 3), [vv.shape[1]], 64)
+    pruned = _vp_decode(P, q, Kt, vv, m_v)
+    np.testing.assert_allclose(pruned["out"], plain["out"], rtol=1e-11, atol=1e-12)
+
+
+def test_value_pruning_storage_rounds_the_projected_values():
+    """bf16 storage: V^ is the RNE rounding of (v P)[:m_v] (not of v)."""
+    P, q, kk, vv, Kt = _vp_case(35)
+    Vh = O.build_value_cache(vv, P, "bf16", 96)
+    exact = np.einsum("btgi,gij->btgj", vv, P)[..., :96]
+    np.testing.assert_array_equal(Vh, O.round_bf16(exact))
+
+
+def test_h2o_with_value_pruning():
+    """H2O steps with pruned values: the evictions are those of plain H2O (they
+    depend on the keys only) and every output is the plain output projected
+    onto the kept value subspace; at m_v = d the outputs are the plain ones."""
+    d, Hq, Hkv, n0, k = 128, 4, 2, 12, 48
+    rng = np.random.default_rng(36)
+    P = np.stack([_rand_orthogonal(d, 37 + g) for g in range(Hkv)])
+    kk = rng.standard_normal((n0 + 6, Hkv, d))
+    vv = rng.standard_normal((n0 + 6, Hkv, d))
+    q = rng.standard_normal((6, Hq, d))
+    for m_v in (96, 128):
+        def seqs(project_v):
+            return [O.H2OSeq(pos=list(range(n0)), score=[0.0] * n0,
+                             kt=list(O.build_key_cache(kk[:n0, g][:, None], P[g][None], "f64")[:, 0]),
+                             v=list(O.build_value_cache(vv[:n0, g][:, None], P[g][None], "f64", m_v)[:, 0])
+                             if project_v else list(vv[:n0, g]))
+                    for g in range(Hkv)]
+        a, b = seqs(False), seqs(True)
+        for s in range(6):
+            oa, ea = O.h2o_decode_step(a, q[s], kk[n0 + s], vv[n0 + s], n0 + s, P, k, 14, 3, "f64")
+            ob, eb = O.h2o_decode_step(b, q[s], kk[n0 + s], vv[n0 + s], n0 + s, P, k, 14, 3, "f64", m_v=m_v)
+            assert ea == eb
+            for h in range(Hq):
+                Pm = P[h // (Hq // Hkv)][:, :m_v]
+                np.testing.assert_allclose(ob[h], (oa[h] @ Pm) @ Pm.T, rtol=1e-11, atol=1e-12)
+
+
 # --------------------------------------------------------------------------- prefill vs decode
 
 def test_prefill_row_equals_decode_and_chunk_invariance():
