@@ -40,6 +40,9 @@ WORKLOADS = {
     "long-context-decode": dict(B=1, Hq=32, Hkv=8, T=131072, k=96, kv="bf16", d_store=128),
     # tiny f32 case (launch-bound)
     "tiny-f32-decode": dict(B=1, Hq=4, Hkv=1, T=1024, k=96, kv="f32", d_store=128),
+    # AQUA-Memory at the Llama decode shape: the first 96 projected key AND value
+    # dimensions stored, k = 64 chosen within the keys' 96
+    "aqua-memory-decode": dict(B=8, Hq=32, Hkv=8, T=8192, k=64, kv="bf16", d_store=96, dv_store=96),
 }
 DEFAULT_WORKLOAD = "llama3.1-8b-decode"
 # chunked causal prefill: a 4096-token prompt in 512-token chunks (Llama-3.1-8B heads)
@@ -242,7 +245,9 @@ class DecodeBench:
         # history of T-1 tokens so the first step attends T
         inp = synth.decode_inputs(B, Hq, Hkv, T - 1, bf16=(kv == "bf16"), steps=n_steps)
         self.T0 = T - 1
-        self.cache = aq.AquaCache(B, Hkv, T + n_steps + 64, d_store=wl["d_store"], dtype=self.dt)
+        self.cache = aq.AquaCache(B, Hkv, T + n_steps + 64, d_store=wl["d_store"], dtype=self.dt,
+                                  dv_store=wl.get("dv_store"))
+        self.vcols = wl.get("dv_store") or 128          # stored value dims
         chunk = 4096
         for s in range(0, T - 1, chunk):
             e = min(T - 1, s + chunk)
@@ -298,20 +303,21 @@ class DecodeBench:
 
     def bytes_decode(self, usz: np.ndarray, T: int) -> float:
         """Algorithmic HBM bytes of one aqua_decode_attn call at T tokens per sequence:
-        union rows of K~ and V rows (per (b, g) and token), q read, output write."""
+        union rows of K~ and stored V rows (per (b, g) and token), q read, output write."""
         wl, e = self.wl, self.esize
         d = 128
-        return float(T * np.sum(e * usz + e * d) + wl["B"] * wl["Hq"] * d * e * 2)
+        return float(T * np.sum(e * usz + e * self.vcols) + wl["B"] * wl["Hq"] * d * e * 2)
 
     def bytes_append(self) -> float:
         wl, e = self.wl, self.esize
-        return float(wl["B"] * wl["Hkv"] * 128 * e * 4)    # read k, v; write k~ column, v row
+        # read k, v; write the k~ column and the (projected) value row
+        return float(wl["B"] * wl["Hkv"] * (128 * e * 2 + wl["d_store"] * e + self.vcols * e))
 
     def bytes_attend(self, usz: np.ndarray, T: int) -> float:
         """Algorithmic HBM bytes of the attention kernel alone: union rows of K~
-        and V rows per (b, g) and token, and the output write."""
+        and stored V rows per (b, g) and token, and the output write."""
         wl, e = self.wl, self.esize
-        return float(T * np.sum(e * usz + e * 128) + wl["B"] * wl["Hq"] * 128 * e)
+        return float(T * np.sum(e * usz + e * self.vcols) + wl["B"] * wl["Hq"] * 128 * e)
 
     def kernel_times(self, K: int, k: int):
         """Each kernel of the decode step timed alone with CUDA events on the
@@ -329,7 +335,7 @@ class DecodeBench:
         for s in range(3):                                   # warm (first launches configure the kernels)
             aq.aqua_decode_select(self.cache.desc, self.q_d[s], self.P, wl["Hq"], k, self.ws,
                                   k_new=self.k_d[s], v_new=self.v_d[s])
-            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True)
+            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True, P=self.P)
         torch.cuda.synchronize()
         self.rewind()
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -340,7 +346,7 @@ class DecodeBench:
             aq.aqua_decode_select(self.cache.desc, self.q_d[i], self.P, wl["Hq"], k, self.ws,
                                   k_new=self.k_d[i], v_new=self.v_d[i])
             ev[s][1].record(st)
-            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True)
+            aq.aqua_decode_attend(self.cache.desc, wl["Hq"], self.out, self.ws, appended=True, P=self.P)
             ev[s][2].record(st)
         torch.cuda.synchronize()
         sel = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
@@ -846,8 +852,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--k", type=int, default=None)
     ap.add_argument("--no-extras", action="store_true", help="only the main decode line")
-    ap.add_argument("--extras", default="sweep,tsweep,long,prefill,h2o",
-                    help="comma list of extra lines: sweep (k sweep), tsweep (break-even sweep over T in "
+    ap.add_argument("--extras", default="sweep,memory,tsweep,long,prefill,h2o",
+                    help="comma list of extra lines: sweep (k sweep), memory (keys and values stored at 96 "
+                         "projected dims), tsweep (break-even sweep over T in "
                          "{2048, 8192, 32768} and k), tsweep_full (T from 512 to 32768), long (long context), "
                          "prefill (chunked prefill, full and truncated cache), h2o (truncated cache + H2O steady "
                          "state)")
@@ -942,6 +949,27 @@ def main():
     P = bench.P
     del bench
     torch.cuda.empty_cache()
+    if "memory" in extras:
+        mwl = WORKLOADS["aqua-memory-decode"]
+        mb = DecodeBench(mwl, K, W, P=P)
+        mu = mb.union_sizes(mwl["k"], min(K, 8))
+        t_ms, d_ms, _ = mb.timed(K, W, mwl["k"], world, clocks=False)
+        t_ms = max_over_ranks(t_ms, world)
+        by = [mb.bytes_decode(mu[s % mu.shape[0]], T_steps[s]) + mb.bytes_append() for s in range(K)]
+        gbs = sum(by) / (t_ms / 1e3) / 1e9
+        dense_us = line["k_sweep"][0]["decode_us"] if "k_sweep" in line else None
+        us = 1e3 * t_ms / K
+        line["aqua_memory"] = {"workload": "aqua-memory-decode", **mwl, "d": 128, "ms_per_step": t_ms / K,
+                               "queries_per_s": world * mwl["B"] * K / (t_ms / 1e3), "decode_us": us,
+                               "mean_union": float(mu.mean()), "bytes_per_step": float(np.mean(by)),
+                               "decode_gbs": gbs, "frac": gbs / hbm_peak,
+                               "speedup_vs_dense": dense_us / us if dense_us else None,
+                               "byte_bound_speedup": 256.0 / (float(mu.mean()) + mwl["dv_store"]),
+                               "note": "keys and values both stored at their first 96 projected dims; dense = the "
+                                       "k = d = 128 step on the full cache (k_sweep[0]); 3 launches per step (the "
+                                       "third brings the output back from the projected value dims)"}
+        del mb
+        torch.cuda.empty_cache()
     if "tsweep" in extras or "tsweep_full" in extras:
         line["t_sweep"] = t_sweep(P, min(K, 20), W, world, Ts=T_SWEEP_FULL_TS if "tsweep_full" in extras else None)
         torch.cuda.empty_cache()

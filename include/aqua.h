@@ -70,7 +70,12 @@ enum aqua_dtype { AQUA_F32 = 0, AQUA_BF16 = 1 };
  *                                           tokens.  d_store = m < d keeps only the
  *                                           first m projected dimensions
  *                                           (AQUA-Memory static truncation).
- *   v       [B][Hkv][Tcap][d]        dtype  unprojected values, token-major.
+ *   v       [B][Hkv][Tcap][dv]       dtype  values, token-major.  dv_store = 0: the
+ *                                           unprojected values (dv = d).  dv_store > 0
+ *                                           (AQUA-Memory on the values): the first
+ *                                           dv = dv_store dimensions of v P, the
+ *                                           projected value; outputs are brought back
+ *                                           as o = o^ P[:, :dv_store]^T.
  *   len     [B]                      int32  tokens (slots) in use per sequence.
  *   n_abs   [B]                      int32  tokens ever appended per sequence (the
  *                                           absolute position of the next token);
@@ -85,6 +90,12 @@ enum aqua_dtype { AQUA_F32 = 0, AQUA_BF16 = 1 };
  *                                           word read by aqua_status.
  *   max_len  host int: an upper bound of every len[b]; aqua_project_keys adds L,
  *            aqua_h2o_update lowers it to the budget.
+ *   dv_store host int: 0, or the number of projected value dimensions stored
+ *            (a multiple of 16, at most d).  The edgentiq blog ("AQUA-Memory:
+ *            Dual Savings") drops the lowest-importance dimensions of both keys
+ *            and values before caching; the reading taken: values use the KV
+ *            head's P like the keys and the first dv_store projected dimensions
+ *            are kept.  Prefill requires dv_store = 0.
  *   Tcap must be a multiple of 16; dtype is AQUA_BF16 or AQUA_F32 for both k_proj and v.
  */
 typedef struct aqua_cache {
@@ -98,6 +109,7 @@ typedef struct aqua_cache {
   int B, Hkv, d, d_store, Tcap;
   int max_len;
   int dtype;
+  int dv_store;
 } aqua_cache;
 
 /* Thread-local text of the last failure on this host thread ("" if none). */
@@ -133,7 +145,8 @@ AQUA_API int aqua_calibrate(const float* X, int n, int d, float* P_out, float* s
  * k~ = k_new[b][l][g] . P[g] is computed in f32, its first d_store dimensions
  * are rounded to the cache dtype (bf16: round-to-nearest-even) and written into
  * slot len[b] + l of k_proj (dimension-major); v_new is copied into the same
- * slot of v.  If pos/score are present the slot's position is n_abs[b] + l and
+ * slot of v (with dv_store > 0: v~ = v_new P[g] in f32, its first dv_store
+ * dimensions rounded to the cache dtype).  If pos/score are present the slot's position is n_abs[b] + l and
  * its score 0.  Afterwards len[b] += L and n_abs[b] += L on the device, and
  * cache->max_len += L on the host.
  *   k_new, v_new  [B][L][Hkv][d]  cache dtype
@@ -210,16 +223,18 @@ AQUA_API int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_ne
  * they overlap as in aqua_decode_attn).  The workspace carries the selection
  * from the first call to the second; neither it nor the cache may be touched
  * in between.  `appended` must be 1 exactly when the preceding
- * aqua_decode_select was given k_new/v_new.  Arguments as aqua_decode_attn;
+ * aqua_decode_select was given k_new/v_new.  P may be NULL for
+ * aqua_decode_attend unless cache->dv_store > 0 (the output's back-projection
+ * reads it).  Arguments as aqua_decode_attn;
  * each call checks the arguments it uses (AQUA_ERR_ARG for appended not 0/1,
  * or 1 with an empty cache).
  */
 AQUA_API int aqua_decode_select(aqua_cache* cache, const void* q, const void* k_new, const void* v_new,
                                 const float* P, int Hq, int k, float scale, int32_t* sel_out, float* qproj_out,
                                 void* workspace, size_t workspace_bytes, aqua_stream_t stream);
-AQUA_API int aqua_decode_attend(aqua_cache* cache, int Hq, int appended, void* out, int out_dtype,
-                                float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
-                                aqua_stream_t stream);
+AQUA_API int aqua_decode_attend(aqua_cache* cache, const float* P, int Hq, int appended, void* out,
+                                int out_dtype, float* scores_out, float* lse_out, void* workspace,
+                                size_t workspace_bytes, aqua_stream_t stream);
 
 /*
  * The decode step of aqua_decode_attn for callers that cannot provide device

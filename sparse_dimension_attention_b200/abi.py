@@ -48,7 +48,7 @@ class aqua_cache(ctypes.Structure):
         ("k_proj", c_void_p), ("v", c_void_p), ("len", c_void_p), ("n_abs", c_void_p),
         ("pos", c_void_p), ("score", c_void_p), ("ctrl", c_void_p),
         ("B", c_int), ("Hkv", c_int), ("d", c_int), ("d_store", c_int), ("Tcap", c_int),
-        ("max_len", c_int), ("dtype", c_int),
+        ("max_len", c_int), ("dtype", c_int), ("dv_store", c_int),
     ]
 
 
@@ -77,7 +77,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "aqua_decode_workspace_size": (c_size_t, [C, c_int]),
         "aqua_decode_attn": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P, c_size_t, P]),
         "aqua_decode_select": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, P, P, c_size_t, P]),
-        "aqua_decode_attend": (c_int, [C, c_int, c_int, P, c_int, P, P, P, c_size_t, P]),
+        "aqua_decode_attend": (c_int, [C, P, c_int, c_int, P, c_int, P, P, P, c_size_t, P]),
         "aqua_decode_attn_static": (c_int, [C, P, P, P, P, c_int, c_int, c_float, P, c_int, P, P, P, P, P]),
         "aqua_selftest_wait_timeout": (c_int, [C, ctypes.c_ulonglong, P]),
         "aqua_prefill_workspace_size": (c_size_t, [C, c_int, c_int]),
@@ -172,13 +172,14 @@ def aqua_decode_select(cache: aqua_cache, q, P, Hq: int, k: int, workspace, scal
         _ptr(qproj_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
-def aqua_decode_attend(cache: aqua_cache, Hq: int, out, workspace, appended: bool = False, scores_out=None,
-                       lse_out=None, stream=None) -> None:
-    """Second half of a decode step: attention over the selection aqua_decode_select left in the workspace."""
+def aqua_decode_attend(cache: aqua_cache, Hq: int, out, workspace, appended: bool = False, P=None,
+                       scores_out=None, lse_out=None, stream=None) -> None:
+    """Second half of a decode step: attention over the selection aqua_decode_select left in the
+    workspace (P is needed only with projected values)."""
     out_dtype = AQUA_BF16 if str(out.dtype) == "torch.bfloat16" else AQUA_F32
     _check(load_library().aqua_decode_attend(
-        ctypes.byref(cache), Hq, int(bool(appended)), _ptr(out), out_dtype, _ptr(scores_out), _ptr(lse_out),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+        ctypes.byref(cache), _ptr(P), Hq, int(bool(appended)), _ptr(out), out_dtype, _ptr(scores_out),
+        _ptr(lse_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def aqua_decode_attn_static(cache: aqua_cache, q, P, Hq: int, k: int, out, scale: float = 0.0, k_new=None,

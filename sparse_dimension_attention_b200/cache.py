@@ -13,18 +13,21 @@ from . import abi
 class AquaCache:
     """Projected-key cache (dimension-major), value cache (token-major) and lengths.
 
-    k_proj [B, Hkv, d_store, Tcap], v [B, Hkv, Tcap, d], len [B], n_abs [B];
-    with h2o=True also pos [B, Hkv, Tcap] (int32) and score [B, Hkv, Tcap] (f32).
+    k_proj [B, Hkv, d_store, Tcap], v [B, Hkv, Tcap, d] (with dv_store: the
+    first dv_store projected value dims, [B, Hkv, Tcap, dv_store]), len [B],
+    n_abs [B]; with h2o=True also pos [B, Hkv, Tcap] (int32) and score
+    [B, Hkv, Tcap] (f32).
     """
 
     def __init__(self, B: int, Hkv: int, Tcap: int, d: int = 128, d_store: int | None = None,
-                 dtype: torch.dtype = torch.bfloat16, h2o: bool = False, device="cuda"):
+                 dtype: torch.dtype = torch.bfloat16, h2o: bool = False, device="cuda", dv_store: int | None = None):
         d_store = d if d_store is None else d_store
         if Tcap % 16:
             Tcap += 16 - Tcap % 16
         self.B, self.Hkv, self.d, self.d_store, self.Tcap, self.dtype = B, Hkv, d, d_store, Tcap, dtype
+        self.dv_store = dv_store or 0
         self.k_proj = torch.zeros((B, Hkv, d_store, Tcap), dtype=dtype, device=device)
-        self.v = torch.zeros((B, Hkv, Tcap, d), dtype=dtype, device=device)
+        self.v = torch.zeros((B, Hkv, Tcap, self.dv_store or d), dtype=dtype, device=device)
         self.len = torch.zeros((B,), dtype=torch.int32, device=device)
         self.n_abs = torch.zeros((B,), dtype=torch.int32, device=device)
         self.ctrl = torch.zeros((abi.AQUA_CTRL_WORDS,), dtype=torch.int32, device=device)
@@ -34,7 +37,7 @@ class AquaCache:
             self.k_proj.data_ptr(), self.v.data_ptr(), self.len.data_ptr(), self.n_abs.data_ptr(),
             self.pos.data_ptr() if h2o else None, self.score.data_ptr() if h2o else None,
             self.ctrl.data_ptr(), B, Hkv, d, d_store, Tcap, 0,
-            abi.AQUA_BF16 if dtype == torch.bfloat16 else abi.AQUA_F32)
+            abi.AQUA_BF16 if dtype == torch.bfloat16 else abi.AQUA_F32, self.dv_store)
 
     @property
     def max_len(self) -> int:

@@ -149,6 +149,8 @@ int validate_cache(const aqua_cache* c) {
     return set_error(AQUA_ERR_ARG, "cache: pos requires score and n_abs");
   if ((long long)c->B * c->Hkv > (1LL << 24))
     return set_error(AQUA_ERR_UNSUPPORTED, "cache: B*Hkv too large");
+  if (c->dv_store < 0 || c->dv_store > c->d || c->dv_store % 16 != 0)
+    return set_error(AQUA_ERR_ARG, "cache: dv_store %d must be 0 or a multiple of 16 up to d", c->dv_store);
   return AQUA_OK;
 }
 
@@ -196,7 +198,7 @@ int check_attend_args(const aqua::DecodeArgs& a, const char* who) {
 int check_workspace(const aqua_cache* c, int Hq, const void* ws, size_t ws_bytes, const char* who) {
   if (ws == nullptr) return set_error(AQUA_ERR_ARG, "%s: NULL workspace", who);
   if (!aligned(ws, 256)) return set_error(AQUA_ERR_ARG, "%s: workspace must be 256-byte aligned", who);
-  const size_t need = aqua::decode_workspace_bytes(c->B * c->Hkv, Hq / c->Hkv);
+  const size_t need = aqua::decode_workspace_bytes(c->B * c->Hkv, Hq / c->Hkv, c->dv_store > 0);
   if (ws_bytes < need) return set_error(AQUA_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", who, ws_bytes, need);
   return AQUA_OK;
 }
@@ -219,7 +221,7 @@ extern "C" {
 
 const char* aqua_last_error(void) { return aqua::g_err; }
 
-int aqua_version(void) { return 3; }
+int aqua_version(void) { return 4; }
 
 int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream) {
   if (cache == nullptr || cache->ctrl == nullptr || status_out == nullptr)
@@ -278,7 +280,7 @@ int aqua_project_keys(aqua_cache* cache, const void* k_new, const void* v_new, c
 
 size_t aqua_decode_workspace_size(const aqua_cache* cache, int Hq) {
   if (validate_cache(cache) != AQUA_OK || Hq < 1 || Hq % cache->Hkv != 0) return 0;
-  return aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv);
+  return aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv, cache->dv_store > 0);
 }
 
 int aqua_decode_attn(aqua_cache* cache, const void* q, const void* k_new, const void* v_new, const float* P,
@@ -317,17 +319,20 @@ int aqua_decode_select(aqua_cache* cache, const void* q, const void* k_new, cons
   return rc;
 }
 
-int aqua_decode_attend(aqua_cache* cache, int Hq, int appended, void* out, int out_dtype, float* scores_out,
-                       float* lse_out, void* workspace, size_t workspace_bytes, aqua_stream_t stream) {
+int aqua_decode_attend(aqua_cache* cache, const float* P, int Hq, int appended, void* out, int out_dtype,
+                       float* scores_out, float* lse_out, void* workspace, size_t workspace_bytes,
+                       aqua_stream_t stream) {
   aqua::g_err[0] = '\0';
   aqua::DecodeArgs a;
-  a.Hq = Hq; a.out = out; a.out_dtype = out_dtype; a.scores_out = scores_out; a.lse_out = lse_out;
+  a.P = P; a.Hq = Hq; a.out = out; a.out_dtype = out_dtype; a.scores_out = scores_out; a.lse_out = lse_out;
   a.ws = workspace; a.appended = appended;
   int rc = validate_cache(cache);
   if (rc == AQUA_OK) rc = check_heads(cache, Hq, "aqua_decode_attend");
   if (rc == AQUA_OK) rc = check_attend_args(a, "aqua_decode_attend");
   if (rc == AQUA_OK && appended != 0 && appended != 1)
     rc = set_error(AQUA_ERR_ARG, "aqua_decode_attend: appended=%d (0 or 1)", appended);
+  if (rc == AQUA_OK && cache->dv_store > 0 && (P == nullptr || !aligned(P, 16)))
+    rc = set_error(AQUA_ERR_ARG, "aqua_decode_attend: projected values (dv_store > 0) need a 16-byte aligned P");
   if (rc == AQUA_OK && appended && cache->max_len < 1)
     rc = set_error(AQUA_ERR_ARG, "aqua_decode_attend: appended=1 with max_len 0 (no selection appended a token)");
   if (rc == AQUA_OK) rc = check_workspace(cache, Hq, workspace, workspace_bytes, "aqua_decode_attend");
@@ -350,6 +355,8 @@ int aqua_prefill_attn(const aqua_cache* cache, const void* q, int pos0, int L, c
   if (q == nullptr || P == nullptr || out == nullptr || workspace == nullptr)
     return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: NULL q, P, out or workspace");
   if (cache->dtype != AQUA_BF16) return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: bf16 cache only");
+  if (cache->dv_store != 0)
+    return set_error(AQUA_ERR_UNSUPPORTED, "aqua_prefill_attn: projected values (dv_store > 0) are decode-only");
   if (Hq < 1 || Hq % cache->Hkv != 0)
     return set_error(AQUA_ERR_ARG, "aqua_prefill_attn: Hq=%d not a multiple of Hkv=%d", Hq, cache->Hkv);
   if (k < 1 || k > cache->d_store)

@@ -55,7 +55,8 @@ struct DecodeArgs {
   int appended = 0;   // the step appends its token (k_new/v_new given to the selection phase)
 };
 enum DecodePhase { kPhaseSelect = 1, kPhaseAttend = 2 };
-size_t decode_workspace_bytes(int n_units, int G);
+// scratch of a decode step; with projected values also the pre-projection outputs
+size_t decode_workspace_bytes(int n_units, int G, bool projected_values);
 // Every host-side argument check of a whole decode step except the workspace
 // (AQUA_OK or the status, with the message set).
 int check_decode_args(const aqua_cache* c, const DecodeArgs& a, const char* who);

@@ -79,6 +79,8 @@ struct DecodeParams {
   int32_t* pos;
   float* score;
   int B, Hq, Hkv, d_store, Tcap, k;
+  int dv;                 // 0: unprojected values of D dims; > 0: the first dv projected value dims
+  float* ohat;            // dv > 0: [B][Hq][D] outputs over the projected value dims (workspace)
   int len_add;            // 1 with a fused append: the step attends len[b] + 1 tokens
   int n_late;             // attention CTAs (the last ones) expected to start after the projection kernel
   int out_bf16;
@@ -125,6 +127,16 @@ __device__ __forceinline__ void store_val(const DecodeParams& p, size_t idx, flo
     static_cast<float*>(p.out)[idx] = v;
 }
 
+// A final output element.  With projected values (dv > 0) the result over the
+// stored projected dimensions goes to the workspace; vproj_out_kernel then
+// brings it back to the value space (o = o^ P[:, :dv]^T) and writes out.
+__device__ __forceinline__ void store_result(const DecodeParams& p, size_t idx, float v) {
+  if (p.dv > 0)
+    p.ohat[idx] = v;
+  else
+    store_val(p, idx, v);
+}
+
 // Sequences with no tokens have no tiles: attention over zero tokens is the
 // empty sum, output 0 and lse = -inf.  The attention CTAs share these units
 // (unit u goes to CTA u mod grid).  Only steps without an append can meet one.
@@ -136,7 +148,7 @@ __device__ __forceinline__ void write_empty_units(const DecodeParams& p) {
     const int b = u / p.Hkv;
     if (seq_len(p.len, b, p.Tcap) > 0) continue;
     const size_t bhq0 = (size_t)b * p.Hq + (size_t)(u % p.Hkv) * G;
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_val(p, bhq0 * D + i, 0.f);
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) store_result(p, bhq0 * D + i, 0.f);
     if (p.lse_out != nullptr && threadIdx.x < G) p.lse_out[bhq0 + threadIdx.x] = -INFINITY;
   }
 }
@@ -170,6 +182,7 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
   __shared__ __align__(16) float qs[G][D];       // q rows, later the kept scaled q~
   __shared__ __align__(16) float part[NPW][G][D];
   __shared__ __align__(16) float knew_s[D];
+  __shared__ __align__(16) float vnew_s[D];     // the new value row (projected when dv > 0)
   __shared__ uint32_t masks[G][NWQ];
   __shared__ int neq[G][NWQ];
   __shared__ __align__(8) uint64_t pbars[kPChunks];
@@ -226,7 +239,10 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
       return;
     }
 #pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) knew_s[4 * lane + s2] = kx[s2];
+    for (int s2 = 0; s2 < 4; ++s2) {
+      knew_s[4 * lane + s2] = kx[s2];
+      vnew_s[4 * lane + s2] = Elem<T>::load(&vx[s2]);
+    }
     __syncwarp();
     float kt[4];
     project_row_smem(Ps, knew_s, lane, kt);
@@ -236,9 +252,20 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
       const int jd = 4 * lane + s2;
       if (jd < p.d_store) kp[(size_t)jd * p.Tcap] = Elem<T>::from_f32(kt[s2]);
     }
-    T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * D;
+    if (p.dv > 0) {
+      // projected value v~ = v P, first dv dims (same projection routine and order as the key)
+      float vt[4];
+      project_row_smem(Ps, vnew_s, lane, vt);
+      T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * p.dv;
+      if (4 * lane < p.dv) {
 #pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = vx[s2];
+        for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = Elem<T>::from_f32(vt[s2]);
+      }
+    } else {
+      T* vp = const_cast<T*>(static_cast<const T*>(p.v)) + ((size_t)u * p.Tcap + slot) * D;
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2) vp[4 * lane + s2] = vx[s2];
+    }
     if (p.pos != nullptr && lane == 0) {
       p.pos[(size_t)u * p.Tcap + slot] = nabs;
       p.score[(size_t)u * p.Tcap + slot] = 0.f;
@@ -661,7 +688,7 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
         if (x == h) lh = Lh[x];
       const float o = Oacc[h * D + dim];
       if (hh.seg < 0)
-        store_val(p, (bhq0 + h) * D + dim, o / lh);
+        store_result(p, (bhq0 + h) * D + dim, o / lh);
       else
         p.part_o[((size_t)hh.seg * G + h) * D + dim] = o;
     }
@@ -727,7 +754,7 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
     }
     const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
     const size_t bhq0 = (size_t)b * p.Hq + g * G;
-    store_val(p, (bhq0 + h) * D + dim, O / Lsum);
+    store_result(p, (bhq0 + h) * D + dim, O / Lsum);
     if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M + log2f(Lsum)) * kLn2;
   }
   if (tid == 0) p.counters[hh.u] = 0;
@@ -753,6 +780,19 @@ struct SmemBF16 {
   static_assert(KROW_BF16 >= 2 * TT + G * 4, "a K~ row's padding holds the row's G masked queries");
 };
 
+// The V tile of TT = 128 tokens as tensor copies of 64-dim halves, 128B-swizzled
+// (dims past the stored ones are filled with zeros by the copy); with projected
+// values of at most 64 dims only the first half is copied (the consumers never
+// read the second).
+__device__ __forceinline__ void issue_v_tile(unsigned char* st, const CUtensorMap* tmap, int row, uint64_t* bar,
+                                             uint64_t pol, int vcols) {
+  constexpr int VHALF = 128 * 128;
+  const bool two = vcols > 64;
+  mbar_arrive_expect_tx(bar, (two ? 2 : 1) * VHALF);
+  tma_load_2d(st, tmap, 0, row, bar, pol);
+  if (two) tma_load_2d(st + VHALF, tmap, 64, row, bar, pol);
+}
+
 template <int G>
 __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     decode_attn_bf16_kernel(const __grid_constant__ CUtensorMap tmap_v, DecodeParams p) {
@@ -769,6 +809,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const int vcols = p.dv > 0 ? p.dv : D;       // stored value dims (V row length)
   if (tid == 0) s_last[1] = 0;
 
   // the K~ rows of every stage start zeroed: union padding rows and never-copied
@@ -821,12 +862,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       const int pt = tid - NCT;
       const uint64_t pol = policy_evict_first();
       unsigned char* st = smem + (size_t)it * S::STAGE;
-      if (pt == 0) {
-        mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
-        const int row = W0.u * p.Tcap + t0;
-        tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
-        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
-      }
+      if (pt == 0) issue_v_tile(st, &tmap_v, W0.u * p.Tcap + t0, &full[it], pol, vcols);
       const int chunk = pt & 15, r0 = pt >> 4;
       const __nv_bfloat16* kbase =
           static_cast<const __nv_bfloat16*>(p.kproj) + (size_t)W0.u * p.d_store * p.Tcap + t0 + chunk * 8;
@@ -866,10 +902,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         if (it < n_nat) continue;
         const StageHdr h0 = W0.header(Sd, t, TT);
         unsigned char* st = smem + (size_t)it * S::STAGE;
-        mbar_arrive_expect_tx(&full[it], 2 * S::VHALF);
-        const int row = h0.u * p.Tcap + h0.t0;
-        tma_load_2d(st, &tmap_v, 0, row, &full[it], pol);
-        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[it], pol);
+        issue_v_tile(st, &tmap_v, h0.u * p.Tcap + h0.t0, &full[it], pol, vcols);
       }
     }
     // union rows of the current unit and, loaded ahead, of the next one
@@ -905,12 +938,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       }
       const StageHdr hh = W.header(Sd, t, TT);
       unsigned char* st = smem + (size_t)s * S::STAGE;
-      if (pt == 0 && it >= NSTAGE) {
-        mbar_arrive_expect_tx(&full[s], 2 * S::VHALF);
-        const int row = hh.u * p.Tcap + hh.t0;
-        tma_load_2d(st, &tmap_v, 0, row, &full[s], pol);
-        tma_load_2d(st + S::VHALF, &tmap_v, 64, row, &full[s], pol);
-      }
+      if (pt == 0 && it >= NSTAGE) issue_v_tile(st, &tmap_v, hh.u * p.Tcap + hh.t0, &full[s], pol, vcols);
       const int nch = (hh.nvalid + 7) / 8;                  // 16-byte groups of 8 tokens
       if (chunk < nch) {
         const __nv_bfloat16* kbase =
@@ -1099,13 +1127,14 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       for (int e = 0; e < 4; ++e) split_bf16(pv[e], ph[e], pl[e]);
       const uint32_t pa[4] = {pack_bf16(ph[0], ph[1]), pack_bf16(pl[0], pl[1]), pack_bf16(ph[2], ph[3]),
                               pack_bf16(pl[2], pl[3])};
-      // ---- o += P V over 128 dims (16 n-tiles of 8)
+      // ---- o += P V over the stored value dims (16 n-tiles of 8 for 128 dims)
       {
         const int mtx = lane >> 3, r8 = lane & 7;
         const int tok = tb + (mtx & 1) * 8 + r8;
         const unsigned char* vrow = st + tok * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
+          if (16 * j >= vcols) break;            // past the stored projected value dims
           const int dim0 = 16 * j + (mtx >> 1) * 8;
           const int chunk = (dim0 & 63) >> 3;
           uint32_t bfr[4];
@@ -1225,6 +1254,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const int vcols = p.dv > 0 ? p.dv : D;       // stored value dims (V row length)
 
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -1274,7 +1304,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
       }
       const StageHdr hh = W.header(Sd, t, TT);
       const uint32_t kbytes = (uint32_t)((hh.nvalid + 3) / 4 * 16);
-      const uint32_t vbytes = (uint32_t)hh.nvalid * D * 4;
+      const uint32_t vbytes = (uint32_t)hh.nvalid * vcols * 4;
       unsigned char* st = smem + (size_t)s * S::STAGE;
       if (lane == 0) {
         hdr[s] = hh;
@@ -1288,7 +1318,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
         if (r < hh.nU) bulk_g2s(st + (size_t)r * TT * 4, kbase + (size_t)urow[i] * p.Tcap, kbytes, &full[s], pol);
       }
       if (lane == 0) {
-        const float* vsrc = static_cast<const float*>(p.v) + ((size_t)hh.u * p.Tcap + hh.t0) * D;
+        const float* vsrc = static_cast<const float*>(p.v) + ((size_t)hh.u * p.Tcap + hh.t0) * vcols;
         bulk_g2s(st + S::KBYTES, vsrc, vbytes, &full[s], pol);
       }
     }
@@ -1443,8 +1473,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 #pragma unroll 4
     for (int j = 0; j < TPW; ++j) {
       const int tok = warp * TPW + j;
-      if (tok < hh.nvalid) {
-        const float4 vf = *reinterpret_cast<const float4*>(Vs + (size_t)tok * D + 4 * lane);
+      if (tok < hh.nvalid && 4 * lane < vcols) {   // V rows hold vcols dims ([TT][vcols] in the stage)
+        const float4 vf = *reinterpret_cast<const float4*>(Vs + (size_t)tok * vcols + 4 * lane);
         float pv[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) pv[h] = psm[tok * G + h];
@@ -1495,6 +1525,46 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 }
 
 // ============================================================================
+// projected values: back to the value space
+// ============================================================================
+// With projected values (AQUA-Memory on the values) the attention kernels
+// leave, per query head, o^ over the dv stored projected value dims in the
+// workspace; the output is o[i] = sum_{j < dv} o^[j] P[g][i][j] (o^ times the
+// transpose of P's first dv columns).  One CTA per (b, g) unit, four warps;
+// warp w computes output dims w, w + 4, ...: its lanes read row i of P
+// (contiguous, L2-resident) and the G heads' o^ from shared memory, then a
+// warp sum.  Launched as a programmatic dependent of the attention kernel.
+template <int G>
+__global__ void __launch_bounds__(128) vproj_out_kernel(DecodeParams p) {
+  __shared__ float oh[G][D];
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv, g = u % p.Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t bhq0 = (size_t)b * p.Hq + (size_t)g * G;
+  const float* Pg = p.P + (size_t)g * D * D;
+  pdl_wait();   // the attention kernel's o^ must be complete
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) oh[i / D][i % D] = __ldcg(p.ohat + bhq0 * D + i);
+  __syncthreads();
+  for (int i = warp; i < D; i += 4) {
+    float acc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+    for (int j = lane; j < p.dv; j += 32) {
+      const float pij = __ldg(Pg + (size_t)i * D + j);
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(oh[h][j], pij, acc[h]);
+    }
+    float mine = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float sum = warp_sum(acc[h]);
+      if (lane == h) mine = sum;
+    }
+    if (lane < G) store_val(p, (bhq0 + lane) * D + i, mine);
+  }
+}
+
+// ============================================================================
 // host launch
 // ============================================================================
 template <typename T, int G, int MINB>
@@ -1529,11 +1599,14 @@ int launch_attn_bf16(const aqua_cache* c, const DecodeParams& p, int C, cudaStre
   static thread_local const void* last_base = nullptr;
   static thread_local uint64_t last_rows = 0;
   static thread_local CUtensorMap tmap;
+  static thread_local uint64_t last_cols = 0;
   const uint64_t rows = (uint64_t)c->B * c->Hkv * c->Tcap;
-  if (last_base != c->v || last_rows != rows) {
-    if ((rc = encode_tmap_bf16_2d(&tmap, c->v, D, rows, D * 2, 64, S::TT, true)) != AQUA_OK) return rc;
+  const uint64_t cols = c->dv_store > 0 ? (uint64_t)c->dv_store : (uint64_t)D;   // V row length
+  if (last_base != c->v || last_rows != rows || last_cols != cols) {
+    if ((rc = encode_tmap_bf16_2d(&tmap, c->v, cols, rows, cols * 2, 64, S::TT, true)) != AQUA_OK) return rc;
     last_base = c->v;
     last_rows = rows;
+    last_cols = cols;
   }
   const cudaError_t e = launch_pdl(decode_attn_bf16_kernel<G>, dim3(C), dim3(NTHREADS_BF16), S::BYTES, st, tmap, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_bf16_kernel: %s", cudaGetErrorString(e));
@@ -1558,12 +1631,17 @@ int launch_phases(const aqua_cache* c, const DecodeParams& p, int n_units, int C
     rc = bf ? launch_qproj<__nv_bfloat16, G>(p, n_units, st) : launch_qproj<float, G>(p, n_units, st);
   if (rc == AQUA_OK && (phases & kPhaseAttend))
     rc = bf ? launch_attn_bf16<G>(c, p, C, st) : launch_attn_f32<G>(p, C, st);
+  if (rc == AQUA_OK && (phases & kPhaseAttend) && p.dv > 0) {
+    const cudaError_t e = launch_pdl(vproj_out_kernel<G>, dim3(n_units), dim3(128), 0, st, p);
+    if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "vproj_out_kernel: %s", cudaGetErrorString(e));
+    rc = check_launch("vproj_out_kernel");
+  }
   return rc;
 }
 
 }  // namespace
 
-size_t decode_workspace_bytes(int n_units, int G) {
+size_t decode_workspace_bytes(int n_units, int G, bool projected_values) {
   size_t off = 0;
   auto take = [&](size_t bytes) { off += (bytes + 255) & ~size_t(255); };
   const size_t nseg = (size_t)n_units + kMaxCtas;
@@ -1574,6 +1652,7 @@ size_t decode_workspace_bytes(int n_units, int G) {
   take((size_t)n_units * 4);          // counters
   take(nseg * G * 2 * 4);             // part_ml
   take(nseg * G * D * 4);             // part_o
+  if (projected_values) take((size_t)n_units * G * D * 4);   // ohat
   return off;
 }
 
@@ -1599,6 +1678,8 @@ int launch_decode(const aqua_cache* c, const DecodeArgs& a, int phases, cudaStre
   p.counters = static_cast<int32_t*>(take((size_t)n_units * 4));
   p.part_ml = static_cast<float*>(take(nseg * G * 2 * 4));
   p.part_o = static_cast<float*>(take(nseg * G * D * 4));
+  p.dv = c->dv_store;
+  p.ohat = c->dv_store > 0 ? static_cast<float*>(take((size_t)n_units * G * D * 4)) : nullptr;
   p.q = a.q;
   p.P = a.P;
   p.len = c->len;

@@ -73,7 +73,7 @@ extern "C" int aqua_decode_attn_static(aqua_cache* cache, const void* q, const v
   a.scores_out = scores_out; a.lse_out = lse_out; a.appended = k_new != nullptr;
   int rc = aqua::check_decode_args(cache, a, "aqua_decode_attn_static");
   if (rc != AQUA_OK) return rc;
-  const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv);
+  const size_t need = aqua::decode_workspace_bytes(cache->B * cache->Hkv, Hq / cache->Hkv, cache->dv_store > 0);
   if (need > aqua::kStaticScratchBytes)
     return set_error(AQUA_ERR_WORKSPACE,
                      "aqua_decode_attn_static: this shape needs %zu bytes of scratch; the built-in array holds %zu "

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
                                                               int32_t* ctrl, const float* __restrict__ scores,
                                                               const float* __restrict__ lse, int32_t* evicted_out,
                                                               int B, int Hq, int Hkv, int d_store, int Tcap,
-                                                              int budget, int recent) {
+                                                              int budget, int recent, int vcols) {
   __shared__ Cand wbest[kThreads / 32];
   __shared__ int s_victim, s_vpos, is_last;
   const int u = blockIdx.x;
@@ -62,11 +62,11 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   // they move into the victim's slot if one is evicted
   const int last = n - 1;
   T* kp = kproj + (size_t)u * d_store * Tcap;
-  T* vp = vcache + ub * D;
+  T* vp = vcache + ub * vcols;                        // V rows of vcols elements (projected values: dv)
   T klast = T(0.f), vlast = T(0.f);
   if (n > budget) {
     if (threadIdx.x < d_store) klast = kp[(size_t)threadIdx.x * Tcap + last];
-    if (threadIdx.x < D) vlast = vp[(size_t)last * D + threadIdx.x];
+    if (threadIdx.x < vcols) vlast = vp[(size_t)last * vcols + threadIdx.x];
   }
   Cand best{INFINITY, 0, -1};
   for (int tb = threadIdx.x; tb < n; tb += kThreads * kTokPerThread) {
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
     // move the last slot into the evicted one
     static_assert(kThreads >= D, "one thread per key dimension and value element");
     if (threadIdx.x < d_store) kp[(size_t)threadIdx.x * Tcap + v] = klast;
-    if (threadIdx.x < D) vp[(size_t)v * D + threadIdx.x] = vlast;
+    if (threadIdx.x < vcols) vp[(size_t)v * vcols + threadIdx.x] = vlast;
     if (threadIdx.x == 0) {
       pos[ub + v] = pos[ub + last];
       score[ub + v] = score[ub + last];
@@ -161,12 +161,12 @@ int launch_h2o_g(aqua_cache* c, const float* scores, const float* lse, int Hq, i
     e = launch_pdl(h2o_update_kernel<__nv_bfloat16, G>, dim3(n_units), dim3(kThreads), 0, st,
                    static_cast<__nv_bfloat16*>(c->k_proj), static_cast<__nv_bfloat16*>(c->v), c->len,
                    (const int32_t*)c->n_abs, c->pos, c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq,
-                   c->Hkv, c->d_store, c->Tcap, budget, recent);
+                   c->Hkv, c->d_store, c->Tcap, budget, recent, c->dv_store > 0 ? c->dv_store : D);
   } else {
     e = launch_pdl(h2o_update_kernel<float, G>, dim3(n_units), dim3(kThreads), 0, st,
                    static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, (const int32_t*)c->n_abs,
                    c->pos, c->score, c->ctrl, scores, lse, evicted_out, c->B, Hq, c->Hkv, c->d_store, c->Tcap,
-                   budget, recent);
+                   budget, recent, c->dv_store > 0 ? c->dv_store : D);
   }
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "h2o_update_kernel: %s", cudaGetErrorString(e));
   return AQUA_OK;

@@ -34,6 +34,12 @@ template <typename T> struct Vec4;
 template <> struct Vec4<float> { using type = float4; };
 template <> struct Vec4<__nv_bfloat16> { using type = uint2; };
 
+// four floats rounded to T (RNE for bf16) as one vector
+__device__ __forceinline__ float4 to_vec4(const float (&y)[4], float*) { return make_float4(y[0], y[1], y[2], y[3]); }
+__device__ __forceinline__ uint2 to_vec4(const float (&y)[4], __nv_bfloat16*) {
+  return make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
+}
+
 // grid (ceil(L/32), Hkv, B), block 256: P[g] is staged in shared memory by one
 // bulk copy; warp w projects tokens blockIdx.x*32 + 4w .. 4w+3 of (b, g) with
 // one pass over P, the projected keys are staged as a [dim][32 token] tile and
@@ -53,10 +59,12 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
                                                            T* __restrict__ kproj, T* __restrict__ vcache,
                                                            int32_t* len, int32_t* n_abs, int32_t* pos,
                                                            float* score, int32_t* ctrl, int B, int L,
-                                                           int Hkv, int d_store, int Tcap) {
+                                                           int Hkv, int d_store, int Tcap, int dv) {
   using V4 = typename Vec4<T>::type;
-  extern __shared__ __align__(128) float Ps[];              // [D][D]
+  extern __shared__ __align__(128) float Ps[];              // [D][D], then (dv > 0) the value rows
   __shared__ __align__(16) float xs[kWarps][kTokPerWarp][D];  // the warp's key rows
+  // the warp's value rows, projected too when dv > 0: [kWarps][kTokPerWarp][D] after P
+  float (*xv)[kTokPerWarp][D] = reinterpret_cast<float (*)[kTokPerWarp][D]>(Ps + D * D);
   __shared__ T kt[D][kTokPerCta];                           // projected keys, dimension-major
   __shared__ __align__(8) uint64_t pbar;
   __shared__ int is_last;
@@ -86,6 +94,11 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
       vrow[t] = *reinterpret_cast<const V4*>(v_new + row * D + 4 * lane);
     }
     *reinterpret_cast<float4*>(&xs[warp][t][4 * lane]) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+    if (dv > 0) {
+      float vv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (l < ntok) load4<T>(reinterpret_cast<const T*>(&vrow[t]), vv);
+      *reinterpret_cast<float4*>(&xv[warp][t][4 * lane]) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+    }
   }
   __syncwarp();
   const bool ok = mbar_wait_bounded(&pbar, 0);
@@ -98,6 +111,12 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
     for (int t = 0; t < kTokPerWarp; ++t)
 #pragma unroll
       for (int s = 0; s < 4; ++s) kt[4 * lane + s][warp * kTokPerWarp + t] = Elem<T>::from_f32(y[t][s]);
+    if (dv > 0) {
+      // projected values v~ = v P (AQUA-Memory on the values), rounded to the cache type in registers
+      project_rows_smem<kTokPerWarp>(Ps, &xv[warp][0][0], lane, y);
+#pragma unroll
+      for (int t = 0; t < kTokPerWarp; ++t) vrow[t] = to_vec4(y[t], static_cast<T*>(nullptr));
+    }
   }
   pdl_wait();
   // Lengths are read before this CTA takes its ticket below; the last CTA
@@ -113,7 +132,8 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
       const int l = warp * kTokPerWarp + t;
       if (l < ntok) {
         const int slot = base + l0 + l;
-        *reinterpret_cast<V4*>(vcache + (unit * Tcap + slot) * D + 4 * lane) = vrow[t];
+        const int vcols = dv > 0 ? dv : D;                   // V row length
+        if (4 * lane < vcols) *reinterpret_cast<V4*>(vcache + (unit * Tcap + slot) * vcols + 4 * lane) = vrow[t];
         if (pos != nullptr && lane == 0) {
           pos[unit * Tcap + slot] = abase + l0 + l;
           score[unit * Tcap + slot] = 0.f;
@@ -147,7 +167,7 @@ __global__ void __launch_bounds__(256) project_keys_kernel(const T* __restrict__
 int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, const float* P, int L,
                         cudaStream_t st) {
   dim3 grid((L + kTokPerCta - 1) / kTokPerCta, c->Hkv, c->B);
-  const int smem = D * D * 4;
+  const int smem = D * D * 4 + (c->dv_store > 0 ? kWarps * kTokPerWarp * D * 4 : 0);
   if (c->dtype == AQUA_BF16) {
     const int rc = set_smem_limit(project_keys_kernel<__nv_bfloat16>, smem, "project_keys_kernel");
     if (rc != AQUA_OK) return rc;
@@ -155,7 +175,7 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
         project_keys_kernel<__nv_bfloat16>, grid, dim3(256), smem, st, static_cast<const __nv_bfloat16*>(k_new),
         static_cast<const __nv_bfloat16*>(v_new), P, static_cast<__nv_bfloat16*>(c->k_proj),
         static_cast<__nv_bfloat16*>(c->v), c->len, c->n_abs, c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store,
-        c->Tcap);
+        c->Tcap, c->dv_store);
     if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "project_keys_kernel: %s", cudaGetErrorString(e));
   } else {
     const int rc = set_smem_limit(project_keys_kernel<float>, smem, "project_keys_kernel");
@@ -163,7 +183,8 @@ int launch_project_keys(aqua_cache* c, const void* k_new, const void* v_new, con
     const cudaError_t e = launch_pdl(project_keys_kernel<float>, grid, dim3(256), smem, st,
                                      static_cast<const float*>(k_new), static_cast<const float*>(v_new), P,
                                      static_cast<float*>(c->k_proj), static_cast<float*>(c->v), c->len, c->n_abs,
-                                     c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap);
+                                     c->pos, c->score, c->ctrl, c->B, L, c->Hkv, c->d_store, c->Tcap,
+                                     c->dv_store);
     if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "project_keys_kernel: %s", cudaGetErrorString(e));
   }
   return check_launch("project_keys_kernel");

@@ -42,14 +42,15 @@ def test_exports_nothing_else(lib):
 
 
 def test_struct_layout():
-    # 7 pointers followed by 7 ints on LP64
-    assert ctypes.sizeof(abi.aqua_cache) == 7 * 8 + 7 * 4 + 4   # trailing padding to 8
+    # 7 pointers followed by 8 ints on LP64
+    assert ctypes.sizeof(abi.aqua_cache) == 7 * 8 + 8 * 4
     assert abi.aqua_cache.B.offset == 56
     assert abi.aqua_cache.dtype.offset == 56 + 6 * 4
+    assert abi.aqua_cache.dv_store.offset == 56 + 7 * 4
 
 
 def test_version(lib):
-    assert aq.aqua_version() == 3
+    assert aq.aqua_version() == 4
 
 
 def _desc(**kw):
@@ -68,6 +69,9 @@ def _desc(**kw):
     ("k_proj", None, abi.AQUA_ERR_ARG),
     ("k_proj", 0x1004, abi.AQUA_ERR_ARG),       # misaligned
     ("max_len", 65, abi.AQUA_ERR_ARG),
+    ("dv_store", 8, abi.AQUA_ERR_ARG),         # not a multiple of 16
+    ("dv_store", 144, abi.AQUA_ERR_ARG),
+    ("dv_store", -16, abi.AQUA_ERR_ARG),
 ])
 def test_project_keys_rejects_bad_cache(lib, field, value, code):
     c = _desc(**{field: value})
@@ -114,7 +118,7 @@ def test_decode_phases_argument_checks(lib):
         ctypes.byref(kw.get("c", c)), kw.get("q", 0x5000), kw.get("kn", None), kw.get("vn", None), 0x7000,
         kw.get("Hq", 8), kw.get("k", 96), 0.0, None, None, kw.get("ws", 0x10000), kw.get("wsb", ws), None)
     att = lambda **kw: lib.aqua_decode_attend(
-        ctypes.byref(kw.get("c", c)), kw.get("Hq", 8), kw.get("app", 0), kw.get("out", 0x8000),
+        ctypes.byref(kw.get("c", c)), kw.get("P", None), kw.get("Hq", 8), kw.get("app", 0), kw.get("out", 0x8000),
         kw.get("od", abi.AQUA_BF16), None, None, kw.get("ws", 0x10000), kw.get("wsb", ws), None)
     assert sel(q=None) == abi.AQUA_ERR_ARG
     assert sel(k=0) == abi.AQUA_ERR_ARG
@@ -127,6 +131,12 @@ def test_decode_phases_argument_checks(lib):
     assert att(od=9) == abi.AQUA_ERR_UNSUPPORTED
     assert att(Hq=7) == abi.AQUA_ERR_ARG
     assert att(ws=0x10010) == abi.AQUA_ERR_ARG
+    cv = _desc(max_len=10, dv_store=96)
+    wsv = lib.aqua_decode_workspace_size(ctypes.byref(cv), 8)
+    assert wsv > ws                                                   # room for the pre-projection outputs
+    assert att(c=cv, wsb=wsv) == abi.AQUA_ERR_ARG                     # projected values need P
+    assert att(c=cv, P=0x7004, wsb=wsv) == abi.AQUA_ERR_ARG          # misaligned P
+    assert att(c=cv, wsb=ws, P=0x7000) == abi.AQUA_ERR_WORKSPACE
     assert c.max_len == 10
 
 
@@ -184,6 +194,9 @@ def test_prefill_argument_checks(lib):
     ws = lib.aqua_prefill_workspace_size(ctypes.byref(c), 8, 32)
     assert lib.aqua_prefill_attn(ctypes.byref(c), 0x5000, 40, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
                                  None, None, 0x10000, ws, None) == abi.AQUA_ERR_ARG   # pos0 + L > Tcap
+    cv = _desc(dv_store=64)
+    assert lib.aqua_prefill_attn(ctypes.byref(cv), 0x5000, 0, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
+                                 None, None, 0x10000, ws, None) == abi.AQUA_ERR_UNSUPPORTED   # decode-only
     c32 = _desc(dtype=abi.AQUA_F32)
     assert lib.aqua_prefill_attn(ctypes.byref(c32), 0x5000, 0, 32, 0x7000, 8, 96, 0.0, 0x8000, abi.AQUA_BF16,
                                  None, None, 0x10000, ws, None) == abi.AQUA_ERR_UNSUPPORTED
