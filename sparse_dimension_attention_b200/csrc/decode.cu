@@ -570,7 +570,18 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   Split* sp_s = reinterpret_cast<Split*>(sch + 32);
   if (tid == 0) *sp_s = sp;
   const int C = sp.C;
-  if (c >= C) return false;
+  if (c >= C) {
+    // an idle CTA (the grid is sized from the host's length bound, the split
+    // from the actual lengths): an empty schedule, never walked
+    S.N = N;
+    S.NV = NV;
+    S.sp = sp_s;
+    S.C = C;
+    S.my_start = S.my_end = 0;
+    S.u0 = 0;
+    S.ts0 = S.sb0 = S.vs0 = 0;
+    return false;
+  }
   const long long a = split_start(c, sp), e = split_start(c + 1, sp);   // this CTA's positions
   if (tid == 0 && e == NV) sch[1] = N;    // the last CTA's tiles run to the end
   {
@@ -848,11 +859,12 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   // the masked queries in dimension order (zero for dims no head kept), which
   // is the same sum as over the union rows.
   int n_nat = 0;
-  {
+  if (has_work) {
+    // (a CTA without work has no schedule: make_schedule leaves Sd unset for it)
     UnitWalker W0;
     W0.start<TT>(p, Sd, false);
     const int u_first = W0.u;
-    for (int it = 0; has_work && it < NSTAGE && it < n_tiles; ++it) {
+    for (int it = 0; it < NSTAGE && it < n_tiles; ++it) {
       const long long t = Sd.my_start + it;
       W0.seek<TT>(p, Sd, t, false);
       const int t0 = (int)(t - W0.ts) * TT;

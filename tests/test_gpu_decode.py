@@ -70,9 +70,14 @@ def test_decode_bf16_ragged_lengths(T):
     _check_outputs(res, ref, "bf16", lens)
 
 
-def test_decode_bf16_per_sequence_lengths_and_empty():
+@pytest.mark.parametrize("G", [4, 2, 1])
+def test_decode_bf16_per_sequence_lengths_and_empty(G):
+    """Per-sequence lengths with an empty sequence.  The attention grid is sized
+    from the host's length bound (8 tiles per unit) while the split uses the
+    actual lengths (49 CTAs' worth of positions), so the last CTAs of the grid
+    are idle and must not walk a schedule."""
     lens = [1000, 37, 0, 513]
-    cache, res, ref, _ = _decode_case(4, 8, 2, 1000, 64, lens=lens)
+    cache, res, ref, _ = _decode_case(4, 2 * G, 2, 1000, 64, lens=lens)
     live = [i for i, L in enumerate(lens) if L > 0]
     _check_outputs({"out": res["out"][live], "lse": res["lse"][live]},
                    {"out": ref["out"][live], "lse": ref["lse"][live]}, "bf16", None)
