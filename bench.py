@@ -539,6 +539,11 @@ class PrefillBench:
         return alg, dense, issued
 
     def timed(self, K: int, W: int, k: int):
+        """Eager passes with CUDA events around every attention call.  A sleep
+        kernel in front of each pass keeps the GPU busy while the host enqueues
+        the whole pass, so an interval is the kernel's own duration, not a host
+        launch gap (the event between the append and the attention call still
+        serialises the two)."""
         torch = self.torch
         for _ in range(W):
             self.one_pass(k)
@@ -548,6 +553,7 @@ class PrefillBench:
         for _ in range(K):
             ev = [(E(), E()) for _ in range(self.n_chunks)]
             p0, p1 = E(), E()
+            torch.cuda._sleep(int(2e6))                   # ~1 ms of GPU time while the host enqueues
             p0.record()
             self.one_pass(k, ev)
             p1.record()

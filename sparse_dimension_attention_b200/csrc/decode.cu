@@ -791,17 +791,17 @@ struct SmemBF16 {
   static_assert(KROW_BF16 >= 2 * TT + G * 4, "a K~ row's padding holds the row's G masked queries");
 };
 
-// The V tile of TT = 128 tokens as tensor copies of 64-dim halves, 128B-swizzled
-// (dims past the stored ones are filled with zeros by the copy); with projected
-// values of at most 64 dims only the first half is copied (the consumers never
-// read the second).
+// The V tile of TT = 128 tokens as two tensor copies of 64-dim halves,
+// 128B-swizzled.  With projected values the tensor map's rows hold the dv
+// stored dims and the copy fills the dims past them with zeros (a half that
+// starts past dv is all zeros), so the PV products run over all 128 dims with
+// no bound in the loop.
 __device__ __forceinline__ void issue_v_tile(unsigned char* st, const CUtensorMap* tmap, int row, uint64_t* bar,
-                                             uint64_t pol, int vcols) {
+                                             uint64_t pol) {
   constexpr int VHALF = 128 * 128;
-  const bool two = vcols > 64;
-  mbar_arrive_expect_tx(bar, (two ? 2 : 1) * VHALF);
+  mbar_arrive_expect_tx(bar, 2 * VHALF);
   tma_load_2d(st, tmap, 0, row, bar, pol);
-  if (two) tma_load_2d(st + VHALF, tmap, 64, row, bar, pol);
+  tma_load_2d(st + VHALF, tmap, 64, row, bar, pol);
 }
 
 template <int G>
@@ -820,7 +820,6 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int vcols = p.dv > 0 ? p.dv : D;       // stored value dims (V row length)
   if (tid == 0) s_last[1] = 0;
 
   // the K~ rows of every stage start zeroed: union padding rows and never-copied
@@ -874,7 +873,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       const int pt = tid - NCT;
       const uint64_t pol = policy_evict_first();
       unsigned char* st = smem + (size_t)it * S::STAGE;
-      if (pt == 0) issue_v_tile(st, &tmap_v, W0.u * p.Tcap + t0, &full[it], pol, vcols);
+      if (pt == 0) issue_v_tile(st, &tmap_v, W0.u * p.Tcap + t0, &full[it], pol);
       const int chunk = pt & 15, r0 = pt >> 4;
       const __nv_bfloat16* kbase =
           static_cast<const __nv_bfloat16*>(p.kproj) + (size_t)W0.u * p.d_store * p.Tcap + t0 + chunk * 8;
@@ -914,7 +913,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         if (it < n_nat) continue;
         const StageHdr h0 = W0.header(Sd, t, TT);
         unsigned char* st = smem + (size_t)it * S::STAGE;
-        issue_v_tile(st, &tmap_v, h0.u * p.Tcap + h0.t0, &full[it], pol, vcols);
+        issue_v_tile(st, &tmap_v, h0.u * p.Tcap + h0.t0, &full[it], pol);
       }
     }
     // union rows of the current unit and, loaded ahead, of the next one
@@ -950,7 +949,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       }
       const StageHdr hh = W.header(Sd, t, TT);
       unsigned char* st = smem + (size_t)s * S::STAGE;
-      if (pt == 0 && it >= NSTAGE) issue_v_tile(st, &tmap_v, hh.u * p.Tcap + hh.t0, &full[s], pol, vcols);
+      if (pt == 0 && it >= NSTAGE) issue_v_tile(st, &tmap_v, hh.u * p.Tcap + hh.t0, &full[s], pol);
       const int nch = (hh.nvalid + 7) / 8;                  // 16-byte groups of 8 tokens
       if (chunk < nch) {
         const __nv_bfloat16* kbase =
@@ -1139,14 +1138,13 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       for (int e = 0; e < 4; ++e) split_bf16(pv[e], ph[e], pl[e]);
       const uint32_t pa[4] = {pack_bf16(ph[0], ph[1]), pack_bf16(pl[0], pl[1]), pack_bf16(ph[2], ph[3]),
                               pack_bf16(pl[2], pl[3])};
-      // ---- o += P V over the stored value dims (16 n-tiles of 8 for 128 dims)
+      // ---- o += P V over 128 dims (16 n-tiles of 8; zeros past dv with projected values)
       {
         const int mtx = lane >> 3, r8 = lane & 7;
         const int tok = tb + (mtx & 1) * 8 + r8;
         const unsigned char* vrow = st + tok * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (16 * j >= vcols) break;            // past the stored projected value dims
           const int dim0 = 16 * j + (mtx >> 1) * 8;
           const int chunk = (dim0 & 63) >> 3;
           uint32_t bfr[4];
@@ -1542,38 +1540,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
 // With projected values (AQUA-Memory on the values) the attention kernels
 // leave, per query head, o^ over the dv stored projected value dims in the
 // workspace; the output is o[i] = sum_{j < dv} o^[j] P[g][i][j] (o^ times the
-// transpose of P's first dv columns).  One CTA per (b, g) unit, four warps;
-// warp w computes output dims w, w + 4, ...: its lanes read row i of P
-// (contiguous, L2-resident) and the G heads' o^ from shared memory, then a
-// warp sum.  Launched as a programmatic dependent of the attention kernel.
+// transpose of P's first dv columns).  One CTA of 128 threads per (b, g) unit:
+// the first dv columns of P[g] are staged in shared memory by coalesced loads
+// before the dependency wait (rows padded to dv + 1 floats, so that thread i
+// reading row i is free of bank conflicts), then thread i computes output dim
+// i of the G heads.  Launched as a programmatic dependent of the attention
+// kernel.
+constexpr int kVprojThreads = 128;
+__host__ __device__ constexpr int vproj_smem_bytes(int dv) { return D * (dv + 1) * 4; }
+
 template <int G>
-__global__ void __launch_bounds__(128) vproj_out_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kVprojThreads) vproj_out_kernel(DecodeParams p) {
+  extern __shared__ float Pm[];                 // [D][dv + 1]: P[g][i][j], j < dv
   __shared__ float oh[G][D];
   const int u = blockIdx.x;
   const int b = u / p.Hkv, g = u % p.Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int dv = p.dv, ld = dv + 1;
   const size_t bhq0 = (size_t)b * p.Hq + (size_t)g * G;
   const float* Pg = p.P + (size_t)g * D * D;
-  pdl_wait();   // the attention kernel's o^ must be complete
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) oh[i / D][i % D] = __ldcg(p.ohat + bhq0 * D + i);
-  __syncthreads();
-  for (int i = warp; i < D; i += 4) {
-    float acc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-    for (int j = lane; j < p.dv; j += 32) {
-      const float pij = __ldg(Pg + (size_t)i * D + j);
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(oh[h][j], pij, acc[h]);
-    }
-    float mine = 0.f;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float sum = warp_sum(acc[h]);
-      if (lane == h) mine = sum;
-    }
-    if (lane < G) store_val(p, (bhq0 + lane) * D + i, mine);
+  // P does not depend on the attention kernel: stage it before the wait
+  const int q4 = dv / 4;                        // float4 per row (dv is a multiple of 16)
+  for (int idx = threadIdx.x; idx < D * q4; idx += kVprojThreads) {
+    const int i = idx / q4, c = idx - i * q4;
+    const float4 x = __ldg(reinterpret_cast<const float4*>(Pg + (size_t)i * D) + c);
+    float* dst = Pm + i * ld + 4 * c;
+    dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
   }
+  pdl_wait();   // the attention kernel's o^ must be complete
+  for (int idx = threadIdx.x; idx < G * D; idx += kVprojThreads) oh[idx / D][idx % D] = __ldcg(p.ohat + bhq0 * D + idx);
+  __syncthreads();
+  const int i = threadIdx.x;                    // output dim
+  float acc[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = 0.f;
+  const float* prow = Pm + i * ld;
+#pragma unroll 8
+  for (int j = 0; j < dv; ++j) {
+    const float pij = prow[j];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = fmaf(oh[h][j], pij, acc[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) store_val(p, (bhq0 + h) * D + i, acc[h]);
 }
 
 // ============================================================================
@@ -1604,7 +1612,8 @@ int launch_qproj(const DecodeParams& p, int n_units, cudaStream_t st) {
 template <int G>
 int launch_attn_bf16(const aqua_cache* c, const DecodeParams& p, int C, cudaStream_t st) {
   using S = SmemBF16<G>;
-  int rc = set_smem_limit(decode_attn_bf16_kernel<G>, S::BYTES, "decode_attn_bf16_kernel");
+  auto kernel = decode_attn_bf16_kernel<G>;
+  int rc = set_smem_limit(kernel, S::BYTES, "decode_attn_bf16_kernel");
   if (rc != AQUA_OK) return rc;
   // The tensor map depends only on the V buffer and its row count; reuse the
   // last encoding while they are unchanged (encoding costs host time every step).
@@ -1620,7 +1629,7 @@ int launch_attn_bf16(const aqua_cache* c, const DecodeParams& p, int C, cudaStre
     last_rows = rows;
     last_cols = cols;
   }
-  const cudaError_t e = launch_pdl(decode_attn_bf16_kernel<G>, dim3(C), dim3(NTHREADS_BF16), S::BYTES, st, tmap, p);
+  const cudaError_t e = launch_pdl(kernel, dim3(C), dim3(NTHREADS_BF16), S::BYTES, st, tmap, p);
   if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "decode_attn_bf16_kernel: %s", cudaGetErrorString(e));
   return check_launch("decode_attn_bf16_kernel");
 }
@@ -1644,7 +1653,9 @@ int launch_phases(const aqua_cache* c, const DecodeParams& p, int n_units, int C
   if (rc == AQUA_OK && (phases & kPhaseAttend))
     rc = bf ? launch_attn_bf16<G>(c, p, C, st) : launch_attn_f32<G>(p, C, st);
   if (rc == AQUA_OK && (phases & kPhaseAttend) && p.dv > 0) {
-    const cudaError_t e = launch_pdl(vproj_out_kernel<G>, dim3(n_units), dim3(128), 0, st, p);
+    const int smem = vproj_smem_bytes(p.dv);
+    if ((rc = set_smem_limit(vproj_out_kernel<G>, smem, "vproj_out_kernel")) != AQUA_OK) return rc;
+    const cudaError_t e = launch_pdl(vproj_out_kernel<G>, dim3(n_units), dim3(kVprojThreads), smem, st, p);
     if (e != cudaSuccess) return set_error(AQUA_ERR_CUDA, "vproj_out_kernel: %s", cudaGetErrorString(e));
     rc = check_launch("vproj_out_kernel");
   }

@@ -14,11 +14,18 @@ pytestmark = pytest.mark.gpu
 
 TOL_BF16_OUT = 2e-3   # bf16 output vs the oracle output rounded to bf16
 TOL_F32_OUT = 1e-5    # f32 output, f32 cache
-# f32 output from a bf16 cache: the stored K~ is the bf16 rounding of an f32
-# projection; where the exact value lies within the f32 rounding error of a
-# bf16 midpoint (about 2e-4 of the elements on these inputs) the two sides
-# store neighbouring bf16 values, which perturbs a few scores by ~1e-4.
-TOL_F32_OUT_BF16_CACHE = 1e-4
+# f32 output from a bf16 cache, two checks:
+#  * against the oracle evaluated on the GPU's own stored K~ and its own f32
+#    q~ (which the exact-set protocol already ties to the selection): only the
+#    kernel's arithmetic differs, held to the fp32 bound 1e-5 (measured 3.1e-6);
+#  * against the oracle end to end: the stored K~ is the bf16 rounding of an f32
+#    projection, and where the exact value lies within the f32 rounding error
+#    of a bf16 midpoint (about 2e-4 of the elements) the two sides store
+#    neighbouring values (test_key_cache_storage_rounding checks that every
+#    difference is such a midpoint).  Measured maximum 2.84e-5 over four shapes
+#    (up to 32/8 heads and 4001 tokens); the bound keeps a margin of 1.75x.
+TOL_F32_OUT_BF16_CACHE = 5e-5
+TOL_F32_OUT_OWN_CACHE = 1e-5
 
 
 def _decode_case(B, Hq, Hkv, T, k, kv="bf16", out="bf16", lens=None, d_store=None, Tcap=None, chunk=None):
@@ -38,13 +45,28 @@ def _decode_case(B, Hq, Hkv, T, k, kv="bf16", out="bf16", lens=None, d_store=Non
     Kt = oracle_cache(k_all, P64, kv, d_store)
     V = v_all.transpose(0, 2, 1, 3).astype(np.float64)
     ref = O.decode(q, P64, Kt, V, lens, k, m=d_store, out_dtype=out)
+    if kv == "bf16" and out == "f32":
+        ref["own"] = _oracle_on_gpu_state(cache, res, V, lens, k, d_store)
     return cache, res, ref, lens
+
+
+def _oracle_on_gpu_state(cache, res, V, lens, k, d_store):
+    """The oracle's decode on the GPU's own stored K~ (read back from the cache)
+    and its own f32 q~ (identity projection): the selection is then exactly the
+    GPU's and the remaining difference is the kernel's arithmetic."""
+    T = max(lens)
+    Kt_gpu = cache.k_proj.float().cpu().numpy()[..., :T].transpose(0, 1, 3, 2).astype(np.float64)
+    eye = np.broadcast_to(np.eye(128), (cache.Hkv, 128, 128))
+    return O.decode(res["qt"].astype(np.float64), eye, Kt_gpu, V[:, :, :T], lens, k, m=d_store)["out"]
 
 
 def _check_outputs(res, ref, out, lens, kv="bf16"):
     tol = TOL_BF16_OUT if out == "bf16" else (TOL_F32_OUT if kv == "f32" else TOL_F32_OUT_BF16_CACHE)
     err = rel_err_rows(res["out"], ref["out"])
     assert np.max(err) <= tol, f"max rel err {np.max(err):.3e} > {tol}"
+    if "own" in ref:
+        err = rel_err_rows(res["out"], ref["own"])
+        assert np.max(err) <= TOL_F32_OUT_OWN_CACHE, f"vs the oracle on the GPU's state: {np.max(err):.3e}"
     np.testing.assert_allclose(res["lse"], ref["lse"], rtol=1e-5, atol=1e-5)
 
 
