@@ -181,7 +181,8 @@ struct AttnSmem {
   static constexpr int TILE = 128 * 128;             // 128 rows x 128 B = 16 KB (one 64-column half)
   static constexpr int OFF_QH = 0;                   // [2 dim halves][128 rows][128 B]; prologue: P part 3
   static constexpr int OFF_QL = OFF_QH + 2 * TILE;   // prologue: the raw query rows
-  static constexpr int OFF_K0 = OFF_QL + 2 * TILE;   // K~ buffer 0: [2 token halves][d_store rows][128 B]
+  static constexpr int OFF_K0 = OFF_QL + 2 * TILE;   // K~ buffer 0: [2 token halves][d_store rows][128 B];
+                                                     // prologue: P[g] in f32 (64 KB over K0 and K1)
   static constexpr int OFF_K1 = OFF_K0 + 2 * TILE;   // K~ buffer 1
   static constexpr int OFF_V0 = OFF_K1 + 2 * TILE;   // V buffer 0: [2 dim halves][128 tokens][128 B]
   static constexpr int OFF_V1 = OFF_V0 + 2 * TILE;   // V buffer 1; prologue: P part 1
@@ -195,7 +196,8 @@ struct AttnSmem {
 };
 enum {
   BAR_Q = 0,     // raw query rows landed (TMA)
-  BAR_PS,        // P parts written (256 softmax threads)
+  BAR_PF,        // P[g] in f32 landed in the K~ buffers (bulk copies)
+  BAR_PS,        // P parts written, the K~ buffers free again (256 softmax threads)
   BAR_QT,        // q~ = q P complete in TMEM (commit)
   BAR_QM,        // masked q~ high/low parts written (both softmax warpgroups, 256 threads)
   BAR_KF0,       // K~ buffer 0 / 1 full (TMA)
@@ -313,13 +315,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive_expect_tx(&bars[BAR_Q], 2 * S::TILE);
       tma_load_3d(smem + S::OFF_QL, &tm_q, 0, g * G, b * p.L + l0, &bars[BAR_Q], pol_q);
       tma_load_3d(smem + S::OFF_QL + S::TILE, &tm_q, 64, g * G, b * p.L + l0, &bars[BAR_Q], pol_q);
+      // P[g] (f32, 64 KB) into the K~ buffers, converted there by the softmax threads
+      mbar_arrive_expect_tx(&bars[BAR_PF], D * D * 4);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        bulk_g2s_plain(smem + S::OFF_K0 + c * (D * D), p.P + (size_t)g * D * D + c * (D * D / 4), D * D, &bars[BAR_PF]);
       const uint32_t kbytes = 2u * DS * 128u;
       int jk = 0, jv = 0;                             // next K~ / V tile to load
       unsigned long long t_last = globaltimer_ns();
       while ((jk < n_tiles || jv < n_tiles) && !*abort_flag) {
         bool progress = false;
-        // K~(jk) into buffer jk&1 once the QK MMAs of tile jk-2 are done with it
-        if (jk < n_tiles && (jk < 2 || mbar_try_wait(&bars[BAR_KE0 + (jk & 1)], ((jk - 2) >> 1) & 1))) {
+        // K~(jk) into buffer jk&1 once the QK MMAs of tile jk-2 are done with it (the
+        // first two once P's conversion no longer reads the buffers)
+        if (jk < n_tiles && (jk < 2 ? mbar_try_wait(&bars[BAR_PS], 0)
+                                    : mbar_try_wait(&bars[BAR_KE0 + (jk & 1)], ((jk - 2) >> 1) & 1))) {
           unsigned char* kb = smem + ((jk & 1) ? S::OFF_K1 : S::OFF_K0);
           uint64_t* kf = &bars[BAR_KF0 + (jk & 1)];
           mbar_arrive_expect_tx(kf, kbytes);
@@ -346,7 +355,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         else if (now - t_last > kWaitLimitNs) *abort_flag = 1;
       }
       // every copy issued must have landed before the CTA exits
-      bool drained = mbar_wait_bounded(&bars[BAR_Q], 0);
+      bool drained = mbar_wait_bounded(&bars[BAR_Q], 0) && mbar_wait_bounded(&bars[BAR_PF], 0);
       for (int t = max(0, jk - 2); t < jk; ++t)
         drained = mbar_wait_bounded(&bars[BAR_KF0 + (t & 1)], (t >> 1) & 1) && drained;
       for (int t = max(0, jv - 2); t < jv; ++t)
@@ -417,36 +426,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
 
-    // ---- prologue 1: P[g] -> three bf16 parts, MN-major 128B-swizzled tiles
+    // ---- prologue 1: P[g] (f32, landed in the K~ buffers) -> three bf16 parts,
+    // MN-major 128B-swizzled tiles.  16-byte chunk `ch` holds input dim i =
+    // ch / 32, output dims 4 (ch % 32) .. +3: a warp converts one row of P per
+    // round (conflict-free loads), each part as one 8-byte store.
     {
-      const int i = tid >> 1, half = tid & 1;         // input dim i, outputs 64*half .. 64*half+63
-      const float* src = p.P + ((size_t)g * D + i) * D + half * 64;
-      const int rowoff = half * S::TILE + i * 128;
+      const bool landed = wait_or_abort(&bars[BAR_PF], 0, abort_flag);
+      if (landed) {
+        const unsigned char* pf = smem + S::OFF_K0;
 #pragma unroll 4
-      for (int c = 0; c < 8; ++c) {
-        const float4 x0 = __ldg(reinterpret_cast<const float4*>(src + 8 * c));
-        const float4 x1 = __ldg(reinterpret_cast<const float4*>(src + 8 * c + 4));
-        const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        uint32_t w1[4], w2[4], w3[4];
+        for (int it = 0; it < D * D / 4 / kSoftThreads; ++it) {
+          const int ch = it * kSoftThreads + tid;
+          const int i = ch >> 5, j0 = 4 * (ch & 31);
+          const float4 x4 = *reinterpret_cast<const float4*>(pf + (size_t)ch * 16);
+          const float x[4] = {x4.x, x4.y, x4.z, x4.w};
+          uint32_t w1[2], w2[2], w3[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float r0 = x[2 * e], r1 = x[2 * e + 1];
-          const __nv_bfloat162 a = __floats2bfloat162_rn(r0, r1);
-          r0 -= __low2float(a);
-          r1 -= __high2float(a);
-          const __nv_bfloat162 bb = __floats2bfloat162_rn(r0, r1);
-          r0 -= __low2float(bb);
-          r1 -= __high2float(bb);
-          const __nv_bfloat162 cc = __floats2bfloat162_rn(r0, r1);
-          w1[e] = *reinterpret_cast<const uint32_t*>(&a);
-          w2[e] = *reinterpret_cast<const uint32_t*>(&bb);
-          w3[e] = *reinterpret_cast<const uint32_t*>(&cc);
+          for (int e = 0; e < 2; ++e) {
+            float r0 = x[2 * e], r1 = x[2 * e + 1];
+            const __nv_bfloat162 a = __floats2bfloat162_rn(r0, r1);
+            r0 -= __low2float(a);
+            r1 -= __high2float(a);
+            const __nv_bfloat162 bb = __floats2bfloat162_rn(r0, r1);
+            r0 -= __low2float(bb);
+            r1 -= __high2float(bb);
+            const __nv_bfloat162 cc = __floats2bfloat162_rn(r0, r1);
+            w1[e] = *reinterpret_cast<const uint32_t*>(&a);
+            w2[e] = *reinterpret_cast<const uint32_t*>(&bb);
+            w3[e] = *reinterpret_cast<const uint32_t*>(&cc);
+          }
+          const int jj = j0 & 63;
+          const int off = (j0 >> 6) * S::TILE + i * 128 + ((((jj >> 3) ^ (i & 7))) << 4) + (jj & 7) * 2;
+          *reinterpret_cast<uint2*>(smem + S::OFF_V1 + off) = make_uint2(w1[0], w1[1]);
+          *reinterpret_cast<uint2*>(smem + S::OFF_PP + off) = make_uint2(w2[0], w2[1]);
+          *reinterpret_cast<uint2*>(smem + S::OFF_QH + off) = make_uint2(w3[0], w3[1]);
         }
-        const int off = rowoff + ((c ^ (i & 7)) << 4);
-        *reinterpret_cast<uint4*>(smem + S::OFF_V1 + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-        *reinterpret_cast<uint4*>(smem + S::OFF_PP + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-        *reinterpret_cast<uint4*>(smem + S::OFF_QH + off) = make_uint4(w3[0], w3[1], w3[2], w3[3]);
       }
+      if (!landed) *abort_flag = 1;
       fence_proxy_async_smem();
       mbar_arrive(&bars[BAR_PS]);
     }
