@@ -18,9 +18,10 @@
 //   warp 9     TMA producer
 // Prologue: q~ = q P on the tensor cores (P split into three bf16 parts, f32
 // accumulation, so q~ carries ~24 bits), selection per row from TMEM, masked
-// q~ * scale * log2(e) written as bf16 high and low parts (K-major tiles).
-// Per 128-token KV tile j: S = Qh K~ + Ql K~ (M=128, N=128, K=d_store) into
-// TMEM; the softmax warps copy S to registers and release it, so S(j+1) is
+// q~ * scale * log2(e) written to TMEM as bf16 high and low parts.
+// Per 128-token KV tile j: S = Qh K~ + Ql K~ (M=128, N=128, K=d_store; A from
+// TMEM, B from shared memory) into TMEM; the softmax warps copy S to registers
+// and release it, so S(j+1) is
 // computed while tile j's softmax runs (K~ and V tiles double-buffered); causal
 // mask on diagonal tiles, online softmax with a lazily raised running max, P
 // split into bf16 high/low parts written to tensor memory, O += Ph V + Pl V with
@@ -179,7 +180,7 @@ __device__ __forceinline__ uint32_t pack_hi_halves(uint32_t a, uint32_t b) { ret
 
 struct AttnSmem {
   static constexpr int TILE = 128 * 128;             // 128 rows x 128 B = 16 KB (one 64-column half)
-  static constexpr int OFF_QH = 0;                   // [2 dim halves][128 rows][128 B]; prologue: P part 3
+  static constexpr int OFF_QH = 0;                   // prologue: P part 3 ([2 halves][128 rows][128 B])
   static constexpr int OFF_QL = OFF_QH + 2 * TILE;   // prologue: the raw query rows
   static constexpr int OFF_K0 = OFF_QL + 2 * TILE;   // K~ buffer 0: [2 token halves][d_store rows][128 B];
                                                      // prologue: P[g] in f32 (64 KB over K0 and K1)
@@ -232,28 +233,45 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
-// S(j) = Qh K~(j) + Ql K~(j) into TMEM; then commits: K~ buffer j&1 free, S ready
-__device__ __forceinline__ void issue_qk(unsigned char* smem, uint32_t tm_S, int DS, int j, uint64_t* bars,
-                                         uint32_t idesc) {
+// S(j) = Qh K~(j) + Ql K~(j) into TMEM over NKS k-steps of 16 dims (NKS =
+// d_store / 16), the masked query parts (A) read from tensor memory, K~(j) (B)
+// from shared memory; then commits: K~ buffer j&1 free, S ready.  Keeping A in
+// tensor memory halves the shared-memory operand reads of these MMAs (the
+// tile loop's shared memory also takes the TMA writes of every K~ and V tile).
+// The contraction length is a template parameter so that the 2 NKS MMAs are
+// issued back to back with nothing between them: a run-time test between two
+// tcgen05.mma issues was measured to slow the tensor pipe from 64 to ~107
+// cycles per 128 x 128 x 16 MMA.
+template <int NKS>
+__device__ __forceinline__ void issue_qk_n(unsigned char* smem, uint32_t tm_S, uint32_t tm_Q, int DS, int j,
+                                           uint64_t* bars, uint32_t idesc) {
   using S = AttnSmem;
   const int kb = (j & 1) ? S::OFF_K1 : S::OFF_K0;
-  const int nks = DS / 16;
-  // Descriptors of the first k-step, built once; a later k-step adds its byte
+  // B descriptor of the first k-step, built once; a later k-step adds its byte
   // offset / 16 to the start-address field (every offset is a multiple of 16 and
-  // every address stays below 2^18, so the field never carries).  The issuing
-  // thread then spends one add per MMA.
+  // every address stays below 2^18, so the field never carries).
   const uint64_t bd0 = smem_desc_sw128(smem + kb, DS * 128, 1024);
 #pragma unroll
-  for (int part = 0; part < 2; ++part) {
-    const uint64_t ad0 = smem_desc_sw128(smem + (part == 0 ? S::OFF_QH : S::OFF_QL), 16, 1024);
+  for (int part = 0; part < 2; ++part)
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks)
-      if (ks < nks)
-        tc_mma(tm_S, ad0 + (uint64_t)(((ks >> 2) * S::TILE + (ks & 3) * 32) >> 4),
-               bd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc, part > 0 || ks > 0);
-  }
+    for (int ks = 0; ks < NKS; ++ks)
+      tc_mma_ts(tm_S, tm_Q + part * 64 + ks * 8, bd0 + (uint64_t)((ks * 16 * 128) >> 4), idesc, part > 0 || ks > 0);
   tc_commit(&bars[BAR_KE0 + (j & 1)]);
   tc_commit(&bars[BAR_S]);
+}
+
+__device__ __forceinline__ void issue_qk(unsigned char* smem, uint32_t tm_S, uint32_t tm_Q, int DS, int j,
+                                         uint64_t* bars, uint32_t idesc) {
+  switch (DS / 16) {
+    case 1: issue_qk_n<1>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 2: issue_qk_n<2>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 3: issue_qk_n<3>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 4: issue_qk_n<4>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 5: issue_qk_n<5>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 6: issue_qk_n<6>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    case 7: issue_qk_n<7>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+    default: issue_qk_n<8>(smem, tm_S, tm_Q, DS, j, bars, idesc); break;
+  }
 }
 
 template <int G>
@@ -290,7 +308,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 512);                       // S [0,128), P high/low [128,256), O (q~ first) [256,384)
+    tmem_alloc(tmem_slot, 512);                       // S [0,128), P high/low [128,256), O (q~ first) [256,384),
+                                                      // masked q~ high/low [384,512)
     tmem_relinquish();
   }
   if (tid == kTmaWarp * 32) {
@@ -304,7 +323,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_S = tmem, tm_P = tmem + 128, tm_O = tmem + 256;
+  const uint32_t tm_S = tmem, tm_P = tmem + 128, tm_O = tmem + 256, tm_Q = tmem + 384;
   constexpr uint32_t idesc = idesc_bf16(PM, 128);
 
   if (warp == kTmaWarp) {
@@ -385,7 +404,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok) ok = wait_or_abort(&bars[BAR_KF0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_qk(smem, tm_S, DS, 0, bars, idesc);
+        issue_qk(smem, tm_S, tm_Q, DS, 0, bars, idesc);
       }
       for (int j = 0; j < n_tiles && ok; ++j) {
         if (j + 1 < n_tiles) {
@@ -394,7 +413,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                wait_or_abort(&bars[BAR_KF0 + ((j + 1) & 1)], ((j + 1) >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_qk(smem, tm_S, DS, j + 1, bars, idesc);
+          issue_qk(smem, tm_S, tm_Q, DS, j + 1, bars, idesc);
         }
         ok = wait_or_abort(&bars[BAR_VF0 + (j & 1)], (j >> 1) & 1, abort_flag) &&
              wait_or_abort(&bars[BAR_P], j & 1, abort_flag);
@@ -556,10 +575,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (uint32_t word = selm[w]; word != 0u; word &= word - 1u) so[n++] = d0 + 32 * w + (__ffs(word) - 1);
       }
       if (ok) {
-        // second pass over this half of q~ (still in TMEM): masked, scaled, split, K-major swizzled rows
+        // second pass over this half of q~ (still in TMEM): masked, scaled, split into
+        // bf16 high and low parts and stored to tensor memory as the A operand of
+        // the QK MMAs (K-major, two dims per column, the lower dim in the low half):
+        // high parts in columns [tm_Q, tm_Q + 64), low parts in [tm_Q + 64, tm_Q + 128)
         float* qpo = (p.qproj_out != nullptr && live)
                          ? p.qproj_out + (((size_t)b * p.L + lr) * p.Hq + g * G + (r % G)) * D + d0
                          : nullptr;
+        uint32_t hq[32], lq[32];
 #pragma unroll
         for (int c0 = 0; c0 < 64; c0 += 32) {
           float v[32];
@@ -572,25 +595,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           const uint32_t word = selm[c0 >> 5];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {            // 8 dims = one 16-byte chunk
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int jj = 8 * cc + 2 * e;
-              const float x0 = ((word >> jj) & 1u) ? v[jj] * p.scale_log2 : 0.f;
-              const float x1 = ((word >> (jj + 1)) & 1u) ? v[jj + 1] * p.scale_log2 : 0.f;
-              // high part truncated, low part rounded: |x - hi - lo| <= 2^-16 |x|, unbiased
-              const uint32_t h0 = __float_as_uint(x0) & 0xffff0000u, h1 = __float_as_uint(x1) & 0xffff0000u;
-              hw[e] = pack_hi_halves(h0, h1);
-              lw[e] = pack_bf16(x0 - __uint_as_float(h0), x1 - __uint_as_float(h1));
-            }
-            const int chunk = ((d0 + c0) >> 3) + cc;  // 0..15
-            const int off = (chunk >> 3) * S::TILE + r * 128 + (((chunk & 7) ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(smem + S::OFF_QH + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(smem + S::OFF_QL + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          for (int e = 0; e < 16; ++e) {
+            const int jj = 2 * e;
+            const float x0 = ((word >> jj) & 1u) ? v[jj] * p.scale_log2 : 0.f;
+            const float x1 = ((word >> (jj + 1)) & 1u) ? v[jj + 1] * p.scale_log2 : 0.f;
+            // high part truncated, low part rounded: |x - hi - lo| <= 2^-16 |x|, unbiased
+            const uint32_t h0 = __float_as_uint(x0) & 0xffff0000u, h1 = __float_as_uint(x1) & 0xffff0000u;
+            hq[(c0 >> 1) + e] = pack_hi_halves(h0, h1);
+            lq[(c0 >> 1) + e] = pack_bf16(x0 - __uint_as_float(h0), x1 - __uint_as_float(h1));
           }
         }
-        fence_proxy_async_smem();
+        tmem_st32(tm_Q + lane_base + (d0 >> 1), *reinterpret_cast<const float(*)[32]>(hq));
+        tmem_st32(tm_Q + 64 + lane_base + (d0 >> 1), *reinterpret_cast<const float(*)[32]>(lq));
+        tmem_wait_st();
         tc_fence_before();
       }
       mbar_arrive(&bars[BAR_QM]);
