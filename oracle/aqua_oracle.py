@@ -371,6 +371,66 @@ def h2o_decode_step(seqs, q_b, k_new_b, v_new_b, t_abs: int, P, k: int, budget: 
 
 
 # ----------------------------------------------------------------------------
+# magnitude selection versus slicing off the first dimensions
+# ----------------------------------------------------------------------------
+#
+# The edgentiq blog ("Validation and Generalizability") reports that choosing
+# the dimensions by the query's magnitude loses about half the information that
+# keeping a fixed leading block of dimensions loses ("halving the information
+# retention loss").  It gives no formula.  Readings taken (two losses, both
+# zero when every dimension is kept):
+#   * query energy loss: the share of the projected query's squared norm on the
+#     dimensions left out, 1 - sum_{j in S} q~_j^2 / sum_j q~_j^2;
+#   * attention output loss: ||o_S - o|| / ||o||, o_S the output with scores on
+#     the dimensions S only, o the standard attention output (all dimensions).
+# The slicing baseline keeps dimensions 0 .. k-1 of the projected space (the
+# largest singular values of the calibration).
+
+def select_first_dims(k: int, d: int) -> np.ndarray:
+    """The slicing baseline: the first k projected dimensions, whatever the query."""
+    if not (1 <= k <= d):
+        raise ValueError(f"need 1 <= k <= d, got k={k} d={d}")
+    return np.arange(k)
+
+
+def query_energy_loss(qt, S) -> float:
+    """Share of the projected query's squared norm outside the kept dimensions S."""
+    qt = np.asarray(qt, dtype=np.float64)
+    total = float(np.dot(qt, qt))
+    if total == 0.0:
+        return 0.0
+    kept = float(np.sum(qt[np.asarray(S)] ** 2))
+    return 1.0 - kept / total
+
+
+def attention_output_loss(qt, S, Kt, V, scale: float) -> float:
+    """||o_S - o|| / ||o||: attention with scores on S against all dimensions (one head)."""
+    d = np.shape(qt)[-1]
+    s_full = sparse_scores(qt, np.arange(d), Kt, scale)
+    s_S = sparse_scores(qt, S, Kt, scale)
+    o = softmax(s_full)[0] @ np.asarray(V, dtype=np.float64)
+    o_S = softmax(s_S)[0] @ np.asarray(V, dtype=np.float64)
+    return float(np.linalg.norm(o_S - o) / np.linalg.norm(o))
+
+
+def retention_losses(q, P, K, V, k: int, scale: float | None = None) -> dict:
+    """Mean query-energy and attention-output losses of magnitude selection and
+    of first-k slicing, over query heads q [H, d] attending to keys K [T, d]
+    and values V [T, d] of one KV head with projection P [d, d]."""
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[-1]
+    scale = default_scale(d) if scale is None else scale
+    Kt = project(K, P)
+    out = {"magnitude": {"energy": [], "output": []}, "slicing": {"energy": [], "output": []}}
+    for h in range(q.shape[0]):
+        qt = project(q[h], P)
+        for name, S in (("magnitude", select_dims(qt, k)), ("slicing", select_first_dims(k, d))):
+            out[name]["energy"].append(query_energy_loss(qt, S))
+            out[name]["output"].append(attention_output_loss(qt, S, Kt, V, scale))
+    return {name: {m: float(np.mean(v)) for m, v in r.items()} for name, r in out.items()}
+
+
+# ----------------------------------------------------------------------------
 # counts
 # ----------------------------------------------------------------------------
 

@@ -63,6 +63,12 @@ MUTANTS = [
      "back-projection with another KV head's P"),
     ("h2o_decode_step", "unproject_values(o, P[g])", "unproject_values(o, P[0])",
      "H2O back-projection with another KV head's P"),
+    ("query_energy_loss", "np.sum(qt[np.asarray(S)] ** 2)", "np.sum(np.abs(qt[np.asarray(S)]))",
+     "retention measured on magnitudes instead of energy"),
+    ("attention_output_loss", "np.linalg.norm(o_S - o) / np.linalg.norm(o)",
+     "np.linalg.norm(o_S - o) / np.linalg.norm(o_S)", "output loss normalised by the approximate output"),
+    ("select_first_dims", "return np.arange(k)", "return np.arange(d - k, d)", "slicing the last dimensions"),
+    ("retention_losses", "select_dims(qt, k)", "select_dims(q[h], k)", "selection on the unprojected query"),
     ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * d * 1.0", "break-even without the key projection share"),
     ("breakeven_length", "d * d * (1.0 + 1.0 / G)", "d * k * (1.0 + 1.0 / G)",
      "break-even with d k instead of d^2 projection work"),
@@ -85,6 +91,8 @@ def _pins():
             continue
         if name == "test_select_dims_brute_force_tiny":
             calls += [(name, fn, {"seed": s}) for s in range(40)]
+        elif name == "test_magnitude_selection_minimises_the_energy_loss":
+            calls += [(name, fn, {"seed": s}) for s in range(6)]
         else:
             calls.append((name, fn, {}))
     return calls

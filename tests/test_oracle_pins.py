@@ -465,6 +465,70 @@ def test_h2o_victim_rule_hand_case():
     assert O.h2o_choose_victim([0.0] * 3, [5, 6, 7], 7, 3) == -1  # everything is recent
 
 
+# --------------------------------------------------------------------------- magnitude vs slicing
+
+def test_query_energy_loss_hand_values():
+    qt = np.array([3.0, 4.0, 0.0, 0.0])                 # |q|^2 = 25
+    assert O.query_energy_loss(qt, [1]) == pytest.approx(1 - 16 / 25)
+    assert O.query_energy_loss(qt, [0]) == pytest.approx(1 - 9 / 25)
+    assert O.query_energy_loss(qt, [0, 1]) == 0.0
+    assert O.query_energy_loss(qt, [2, 3]) == 1.0
+    assert O.query_energy_loss(np.zeros(4), [0]) == 0.0
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_magnitude_selection_minimises_the_energy_loss(seed):
+    """Brute force over every k-subset of a tiny projected query: the k largest
+    magnitudes lose the least squared norm."""
+    rng = np.random.default_rng(100 + seed)
+    d = 8
+    qt = rng.standard_normal(d)
+    for k in range(1, d + 1):
+        best = min(O.query_energy_loss(qt, list(S)) for S in itertools.combinations(range(d), k))
+        assert O.query_energy_loss(qt, O.select_dims(qt, k)) == pytest.approx(best, abs=1e-15)
+
+
+def test_attention_output_loss_hand_case():
+    """Two tokens with one-hot keys and values, scale 1: full scores (ln 3, ln 2)
+    give o = (3/5, 2/5); keeping dimension 0 only gives scores (ln 3, 0) and
+    o_S = (3/4, 1/4); the loss is |o_S - o| / |o| = 0.15 sqrt(2) / sqrt(0.52)."""
+    qt = np.array([np.log(3.0), np.log(2.0)])
+    Kt = np.eye(2)
+    V = np.eye(2)
+    got = O.attention_output_loss(qt, [0], Kt, V, 1.0)
+    assert got == pytest.approx(0.15 * np.sqrt(2) / np.sqrt(0.52), rel=1e-12)
+    assert O.attention_output_loss(qt, [0, 1], Kt, V, 1.0) == 0.0
+
+
+def test_slicing_is_the_leading_block_and_equals_magnitude_when_sorted():
+    assert list(O.select_first_dims(3, 8)) == [0, 1, 2]
+    d, k = 16, 6
+    rng = np.random.default_rng(7)
+    q = np.sort(np.abs(rng.standard_normal((3, d))), axis=1)[:, ::-1] * rng.choice([-1, 1], (3, d))
+    K = rng.standard_normal((20, d))
+    V = rng.standard_normal((20, d))
+    r = O.retention_losses(q, np.eye(d), K, V, k)
+    assert r["magnitude"] == r["slicing"]          # the largest magnitudes are the first dims
+
+
+def test_retention_losses_use_the_projected_query():
+    """With P a permutation that moves the query's large entries to the end of
+    the projected space, magnitude selection (on q~ = q P) keeps them and loses
+    nothing of the energy, while slicing the first k projected dims loses it all."""
+    d, k = 8, 2
+    perm = np.roll(np.eye(d), 6, axis=1)              # q~_j = q_(j - 6 mod 8): q_0, q_1 -> dims 6, 7
+    q = np.zeros((1, d))
+    q[0, :2] = [5.0, -4.0]
+    rng = np.random.default_rng(8)
+    K = rng.standard_normal((12, d))
+    V = rng.standard_normal((12, d))
+    qt = O.project(q[0], perm)
+    assert list(np.nonzero(qt)[0]) == [6, 7]
+    r = O.retention_losses(q, perm, K, V, k)
+    assert r["magnitude"]["energy"] == 0.0 and r["magnitude"]["output"] == pytest.approx(0.0, abs=1e-15)
+    assert r["slicing"]["energy"] == 1.0 and r["slicing"]["output"] > 0.0
+
+
 # --------------------------------------------------------------------------- counts
 
 def test_qk_mac_count_matches_pages_25_percent():
