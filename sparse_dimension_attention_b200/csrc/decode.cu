@@ -727,46 +727,60 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
   if (tid == 0) *s_last = (atom_add_acq_rel_gpu(p.counters + hh.u, 1) == hh.nseg - 1);
   named_bar_sync(1, NCT);
   if (!*s_last) return;
-  constexpr int MB = 8;   // partials fetched per round, loads in flight together
+  constexpr int NI = (G * D + NCT - 1) / NCT;   // outputs per thread (2 at G = 4)
+  constexpr int MB = 8 / NI;                    // partials per round: 8 loads x 3 in flight per thread
+  // one pass over the unit's partials for all of this thread's outputs at once
+  // (their loads in flight together): each round of MB partials raises the
+  // running max and rescales what was summed before (nothing in the first)
+  float M[NI], Lsum[NI], O[NI];
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    M[i] = -INFINITY;
+    Lsum[i] = 0.f;
+    O[i] = 0.f;
+  }
 #pragma unroll 1
-  for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
+  for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
+    float mv[NI][MB], lv[NI][MB], ov[NI][MB];
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int idx = tid + NCT * i;
+      const int h = idx / D, dim = idx % D;
+#pragma unroll
+      for (int j = 0; j < MB; ++j) {
+        const bool in = idx < G * D && s0 + j < hh.nseg;
+        const size_t slot = (size_t)(hh.seg0 + s0 + j) * G + h;
+        mv[i][j] = in ? __ldcg(p.part_ml + slot * 2) : -INFINITY;
+        lv[i][j] = in ? __ldcg(p.part_ml + slot * 2 + 1) : 0.f;
+        ov[i][j] = in ? __ldcg(p.part_o + slot * D + dim) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      float Mn = M[i];
+#pragma unroll
+      for (int j = 0; j < MB; ++j) Mn = fmaxf(Mn, mv[i][j]);
+      if (s0 > 0) {
+        const float c = exp2f(M[i] - Mn);
+        Lsum[i] *= c;
+        O[i] *= c;
+      }
+      M[i] = Mn;
+#pragma unroll
+      for (int j = 0; j < MB; ++j) {
+        const float f = exp2f(mv[i][j] - M[i]);
+        Lsum[i] = fmaf(f, lv[i][j], Lsum[i]);
+        O[i] = fmaf(f, ov[i][j], O[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
     const int idx = tid + NCT * i;
     if (idx >= G * D) break;
     const int h = idx / D, dim = idx % D;
-    // one pass: each round of MB partials raises the running max and rescales
-    // what was summed before (nothing when it is the first round)
-    float M = -INFINITY, Lsum = 0.f, O = 0.f;
-#pragma unroll 1
-    for (int s0 = 0; s0 < hh.nseg; s0 += MB) {
-      float mv[MB], lv[MB], ov[MB];
-#pragma unroll
-      for (int j = 0; j < MB; ++j) {
-        const bool in = s0 + j < hh.nseg;
-        const size_t slot = (size_t)(hh.seg0 + s0 + j) * G + h;
-        mv[j] = in ? __ldcg(p.part_ml + slot * 2) : -INFINITY;
-        lv[j] = in ? __ldcg(p.part_ml + slot * 2 + 1) : 0.f;
-        ov[j] = in ? __ldcg(p.part_o + slot * D + dim) : 0.f;
-      }
-      float Mn = M;
-#pragma unroll
-      for (int j = 0; j < MB; ++j) Mn = fmaxf(Mn, mv[j]);
-      if (s0 > 0) {
-        const float c = exp2f(M - Mn);
-        Lsum *= c;
-        O *= c;
-      }
-      M = Mn;
-#pragma unroll
-      for (int j = 0; j < MB; ++j) {
-        const float f = exp2f(mv[j] - M);
-        Lsum = fmaf(f, lv[j], Lsum);
-        O = fmaf(f, ov[j], O);
-      }
-    }
-    const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
-    const size_t bhq0 = (size_t)b * p.Hq + g * G;
-    store_result(p, (bhq0 + h) * D + dim, O / Lsum);
-    if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M + log2f(Lsum)) * kLn2;
+    store_result(p, (bhq0 + h) * D + dim, O[i] / Lsum[i]);
+    if (dim == 0 && p.lse_out) p.lse_out[bhq0 + h] = (M[i] + log2f(Lsum[i])) * kLn2;
   }
   if (tid == 0) p.counters[hh.u] = 0;
 }
@@ -802,6 +816,25 @@ __device__ __forceinline__ void issue_v_tile(unsigned char* st, const CUtensorMa
   mbar_arrive_expect_tx(bar, 2 * VHALF);
   tma_load_2d(st, tmap, 0, row, bar, pol);
   tma_load_2d(st + VHALF, tmap, 64, row, bar, pol);
+}
+
+// Scores of a warp's 16 tokens over NKS k-steps of 16 union rows: even k-steps
+// accumulate into (c0, c1), odd ones into (d0, d1) (two chains per n-tile).
+template <int NKS>
+__device__ __forceinline__ void score_ksteps(const unsigned char* a0, const uint32_t (&afr)[8][4], float (&c0)[4],
+                                             float (&c1)[4], float (&d0)[4], float (&d1)[4]) {
+#pragma unroll
+  for (int kk = 0; kk < NKS; ++kk) {
+    uint32_t bfr[4];
+    ldsm_x4_trans(bfr, a0 + kk * 16 * KROW_BF16);
+    if (kk & 1) {
+      mma_bf16_16816(d0, afr[kk], bfr[0], bfr[1]);
+      mma_bf16_16816(d1, afr[kk], bfr[2], bfr[3]);
+    } else {
+      mma_bf16_16816(c0, afr[kk], bfr[0], bfr[1]);
+      mma_bf16_16816(c1, afr[kk], bfr[2], bfr[3]);
+    }
+  }
 }
 
 template <int G>
@@ -1072,20 +1105,16 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       {
         const int mtx = lane >> 3, r8 = lane & 7;
         const unsigned char* a0 = ks_base + ((mtx & 1) * 8 + r8) * KROW_BF16 + (tb + (mtx >> 1) * 8) * 2;
-#pragma unroll
-        for (int kk = 0; kk < 8; kk += 2) {
-          if (kk < nks) {
-            uint32_t bfr[4];
-            ldsm_x4_trans(bfr, a0 + kk * 16 * KROW_BF16);
-            mma_bf16_16816(c0, afr[kk], bfr[0], bfr[1]);
-            mma_bf16_16816(c1, afr[kk], bfr[2], bfr[3]);
-          }
-          if (kk + 1 < nks) {
-            uint32_t bfr[4];
-            ldsm_x4_trans(bfr, a0 + (kk + 1) * 16 * KROW_BF16);
-            mma_bf16_16816(d0, afr[kk + 1], bfr[0], bfr[1]);
-            mma_bf16_16816(d1, afr[kk + 1], bfr[2], bfr[3]);
-          }
+        // the k-steps as straight-line code for the union size (no test between the MMAs)
+        switch (nks) {
+          case 8: score_ksteps<8>(a0, afr, c0, c1, d0, d1); break;
+          case 7: score_ksteps<7>(a0, afr, c0, c1, d0, d1); break;
+          case 6: score_ksteps<6>(a0, afr, c0, c1, d0, d1); break;
+          case 5: score_ksteps<5>(a0, afr, c0, c1, d0, d1); break;
+          case 4: score_ksteps<4>(a0, afr, c0, c1, d0, d1); break;
+          case 3: score_ksteps<3>(a0, afr, c0, c1, d0, d1); break;
+          case 2: score_ksteps<2>(a0, afr, c0, c1, d0, d1); break;
+          default: score_ksteps<1>(a0, afr, c0, c1, d0, d1); break;
         }
       }
       // high + low parts; tokens tb + {2q, 2q+1, 8+2q, 9+2q}
