@@ -399,6 +399,10 @@ class DecodeBench:
             time.sleep(0.05)
         barrier(world)
         torch.cuda.synchronize()
+        if g is not None:
+            # keep the GPU busy while the host submits the replay, so that the
+            # interval holds the K steps' device time, not the submission latency
+            torch.cuda._sleep(int(1e6))
         e0.record(st)
         if g is not None:
             g.replay()
@@ -476,6 +480,7 @@ class DecodeBench:
         self.rewind()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(1e6))                  # the host submits the replay while the GPU sleeps
         e0.record(st)
         g.replay()
         e1.record(st)
@@ -578,6 +583,7 @@ class PrefillBench:
             g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e6))                  # the host submits the replays while the GPU sleeps
         e0.record()
         for _ in range(K):
             g.replay()
@@ -715,6 +721,7 @@ class H2OBench:
         t_abs0 = wl["budget"] + self.n_steps                               # tokens seen so far
         reps = max(1, (wl["T_end"] - t_abs0) // self.GRAPH_STEPS)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(2e6))                  # the host submits the replays while the GPU sleeps
         e0.record()
         for _ in range(reps):
             g.replay()

@@ -179,11 +179,11 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  *              (len[b] + 1 tokens).  On the device len[b] and n_abs[b] advance
  *              when the step's last kernel finishes.  When NULL the caller
  *              appended the step's key beforehand.
- *   P          [Hkv][d][d] f32.  Read before the step waits for the
- *              preceding kernel on the stream, which is safe unless the
- *              kernel that wrote P released its dependents early through
- *              programmatic dependent launch (no kernel here that writes P
- *              does).
+ *   P          [Hkv][d][d] f32.  P (and, when B*Hkv exceeds the SM count,
+ *              q) are read before the step waits for the preceding kernel on
+ *              the stream, which is safe unless the kernel that wrote them
+ *              released its dependents early through programmatic dependent
+ *              launch (no kernel here that writes them does).
  *   k          dimensions kept per query head, 1 <= k <= d_store
  *   scale      score scale; <= 0 selects 1/sqrt(d) (d = full head dim)
  *   out        [B][Hq][d]  out_dtype (AQUA_F32 or AQUA_BF16, RNE)
@@ -192,7 +192,11 @@ AQUA_API int aqua_project_keys(aqua_cache* cache, const void* k_new, const void*
  *   scores_out nullable [B][Hq][Tcap] f32: score of every cached slot (scaled)
  *   lse_out    nullable [B][Hq] f32: log-sum-exp of the scores
  *   workspace  device, 256-byte aligned, >= aqua_decode_workspace_size bytes;
- *              caller-owned scratch, contents need no initialisation
+ *              caller-owned scratch, contents need no initialisation.  Its
+ *              selection buffers have two halves; successive calls on one
+ *              workspace alternate between them (tracked per workspace
+ *              address), so a step's selection can be written while the
+ *              previous step's attention kernel still reads the other half.
  * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4}.  A sequence with
  * len[b] = 0 gets a zero output and lse = -inf.
  * Errors: AQUA_ERR_ARG if only one of k_new, v_new is given or the cache is full.

@@ -34,6 +34,9 @@
 // f32 caches: CUDA-core FMA consumers (exact f32 products).
 #include <math.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "aqua_internal.cuh"
 
 namespace aqua {
@@ -83,6 +86,7 @@ struct DecodeParams {
   float* ohat;            // dv > 0: [B][Hq][D] outputs over the projected value dims (workspace)
   int len_add;            // 1 with a fused append: the step attends len[b] + 1 tokens
   int n_late;             // attention CTAs (the last ones) expected to start after the projection kernel
+  int early_select;       // the projection kernel selects before waiting for the previous kernel
   int out_bf16;
   float scale_log2;
 };
@@ -204,11 +208,22 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
       bulk_g2s_plain(Ps + c * CROWS * D, p.P + (size_t)g * D * D + c * CROWS * D, CROWS * D * 4, &pbars[c]);
     }
   }
-  pdl_wait();                // the other inputs and the cache may come from the previous kernel
-  // Released only after the previous kernel is complete: the attention kernel
-  // then reads lengths and history K~/V before its own wait, which this kernel
-  // does not change (it writes only slot len[b] and leaves len[b] alone).
-  pdl_launch_dependents();
+  // With early_select the projection and selection below run before the wait
+  // on the previous kernel: they read only q and P and write only this call's
+  // half of the workspace's selection buffers (calls alternate halves), so they
+  // overlap the end of the previous kernel (the H2O update, or the previous
+  // step's attention kernel, which reads the other half).  Used when the units
+  // outnumber the SMs (this kernel then runs two CTAs per SM and takes several
+  // microseconds); with fewer units its selection is shorter than the
+  // attention kernel's own prologue, which it hides when it runs after the wait.
+  // Either way every thread waits before the kernel releases its dependent (the
+  // attention kernel reads the lengths, which the previous step's attention
+  // kernel advances at its end, before its own wait), and before the append
+  // reads the lengths and writes the cache.
+  if (!p.early_select) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   if (threadIdx.x == 0) s_abort = 0;
   __syncthreads();
 
@@ -216,6 +231,10 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
     // ---- fused append of the new token of unit (b, g), in the key projection
     // order.  This warp takes no part in the selection below (which does not
     // depend on it), so the two run side by side.
+    if (p.early_select) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     if (!append) return;
     const int slot = __ldcg(p.len + b);
     const int nabs = p.pos != nullptr ? __ldcg(p.n_abs + b) : 0;
@@ -316,6 +335,10 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
   named_bar_sync(1, NPT);
   if (s_abort) {
     if (threadIdx.x == 0) record_status(p.ctrl, AQUA_ERR_TIMEOUT);
+    if (p.early_select) {
+      pdl_wait();
+      pdl_launch_dependents();
+    }
     return;
   }
 
@@ -399,6 +422,10 @@ __global__ void __launch_bounds__(QprojCfg<G>::WARPS * 32, MINB) qproj_topk_kern
   if (threadIdx.x == 0) {
     p.ucount[u] = __popc(um[0]) + __popc(um[1]) + __popc(um[2]) + __popc(um[3]);
     p.counters[u] = 0;
+  }
+  if (p.early_select) {
+    pdl_wait();
+    pdl_launch_dependents();
   }
 }
 
@@ -1697,15 +1724,30 @@ size_t decode_workspace_bytes(int n_units, int G, bool projected_values) {
   size_t off = 0;
   auto take = [&](size_t bytes) { off += (bytes + 255) & ~size_t(255); };
   const size_t nseg = (size_t)n_units + kMaxCtas;
-  take((size_t)n_units * D * G * 4);  // qm
-  take((size_t)n_units * D * G * 4);  // qmn
-  take((size_t)n_units * D * 4);      // ulist
-  take((size_t)n_units * 4);          // ucount
-  take((size_t)n_units * 4);          // counters
+  for (int half = 0; half < 2; ++half) {   // selection buffers, alternating between calls
+    take((size_t)n_units * D * G * 4);  // qm
+    take((size_t)n_units * D * G * 4);  // qmn
+    take((size_t)n_units * D * 4);      // ulist
+    take((size_t)n_units * 4);          // ucount
+    take((size_t)n_units * 4);          // counters
+  }
   take(nseg * G * 2 * 4);             // part_ml
   take(nseg * G * D * 4);             // part_o
   if (projected_values) take((size_t)n_units * G * D * 4);   // ohat
   return off;
+}
+
+// Half of a workspace's selection buffers for a call: calls that select flip
+// the workspace's half, so that a step's selection never writes the half the
+// previous step's attention kernel may still be reading; a call that only
+// attends keeps the half.  Kept per workspace address (thread-safe).
+int workspace_half(const void* ws, bool flip) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, int> halves;
+  std::lock_guard<std::mutex> lock(mu);
+  int& h = halves[ws];
+  if (flip) h ^= 1;
+  return h;
 }
 
 // One decode step, or one of its phases: kPhaseSelect launches the projection
@@ -1723,11 +1765,24 @@ int launch_decode(const aqua_cache* c, const DecodeArgs& a, int phases, cudaStre
     return ptr;
   };
   const size_t nseg = (size_t)n_units + kMaxCtas;
-  p.qm = static_cast<float*>(take((size_t)n_units * D * G * 4));
-  p.qmn = static_cast<float*>(take((size_t)n_units * D * G * 4));
-  p.ulist = static_cast<int32_t*>(take((size_t)n_units * D * 4));
-  p.ucount = static_cast<int32_t*>(take((size_t)n_units * 4));
-  p.counters = static_cast<int32_t*>(take((size_t)n_units * 4));
+  // this call's half of the selection buffers: a call with the selection phase
+  // takes the other half than the previous call on this workspace; the
+  // attention phase alone uses the half its selection phase wrote
+  const int half = workspace_half(a.ws, (phases & kPhaseSelect) != 0);
+  for (int h = 0; h < 2; ++h) {
+    float* qm = static_cast<float*>(take((size_t)n_units * D * G * 4));
+    float* qmn = static_cast<float*>(take((size_t)n_units * D * G * 4));
+    int32_t* ulist = static_cast<int32_t*>(take((size_t)n_units * D * 4));
+    int32_t* ucount = static_cast<int32_t*>(take((size_t)n_units * 4));
+    int32_t* counters = static_cast<int32_t*>(take((size_t)n_units * 4));
+    if (h == half) {
+      p.qm = qm;
+      p.qmn = qmn;
+      p.ulist = ulist;
+      p.ucount = ucount;
+      p.counters = counters;
+    }
+  }
   p.part_ml = static_cast<float*>(take(nseg * G * 2 * 4));
   p.part_o = static_cast<float*>(take(nseg * G * D * 4));
   p.dv = c->dv_store;
@@ -1750,6 +1805,7 @@ int launch_decode(const aqua_cache* c, const DecodeArgs& a, int phases, cudaStre
   // the projection kernel gives each of its CTAs an SM of its own when there
   // are no more units than SMs; that many attention CTAs then start late
   p.n_late = n_units <= device_sm_count() ? n_units : 0;
+  p.early_select = n_units > device_sm_count() ? 1 : 0;
   p.n_abs = c->n_abs;
   p.pos = c->pos;
   p.score = c->score;

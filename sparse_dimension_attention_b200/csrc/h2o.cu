@@ -46,6 +46,9 @@ __global__ void __launch_bounds__(kThreads) h2o_update_kernel(T* __restrict__ kp
   const int b = u / Hkv, g = u % Hkv;
   // launched as a dependent of the decode step: every input below is its output
   pdl_wait();
+  // the next kernel may start now: a decode step's projection kernel reads only
+  // q and P and writes its own workspace half before it waits for this kernel
+  pdl_launch_dependents();
   const int n = min(max(__ldcg(len + b), 0), Tcap);   // read before the ticket below
   const int newest = __ldcg(n_abs + b) - 1;
   const size_t ub = (size_t)u * Tcap;
