@@ -12,7 +12,19 @@ from aqua_testlib import calib_P, check_selection, fill_cache, rel_err_rows, tde
 pytestmark = pytest.mark.gpu
 
 TOL_BF16_OUT = 2e-3   # bf16 output vs the oracle output rounded to bf16
-TOL_F32_OUT = 1e-4    # f32 output (bf16 cache: stored K~ may differ by one bf16 ulp at midpoints)
+# f32 output from a bf16 cache:
+#  * against the oracle evaluated on the kernel's own exported q~ and its stored
+#    K~ (identity projection), so that only the kernel's arithmetic differs: the
+#    bf16 high/low parts of P (each truncated, |p - hi - lo| < 2^-14 p) and of
+#    the masked query, f32 accumulation.  Measured maximum 1.34e-5 over four
+#    shapes (up to 32/8 heads, two 512-row chunks); bound 3e-5;
+#  * end to end against the oracle, on rows whose every head selects the
+#    oracle's f64 set (at near ties the kernel's ~24-bit q~ may legitimately
+#    keep another dimension; those rows are covered by the check above):
+#    stored K~ differs by bf16 midpoint flips as in decode.  Bound 5e-5.
+TOL_F32_OWN = 3e-5
+TOL_F32_OUT = 5e-5
+TOL_QPROJ = 1e-5      # kernel q~ vs the oracle's f64 q~, relative to the row's largest |q~|
 
 
 def _prefill_case(Hq, Hkv, chunks, k, out="bf16", d_store=None, B=1):
@@ -52,6 +64,19 @@ def _prefill_case(Hq, Hkv, chunks, k, out="bf16", d_store=None, B=1):
             rb.append((o_ref, s_ref, qt))
             pos0 += L
         refs.append(rb)
+    # the oracle on the kernel's own state: its exported q~ (identity projection)
+    # and its stored K~ (appends never change earlier slots, so the final cache
+    # holds every chunk's keys as they were)
+    eye = np.broadcast_to(np.eye(128), (Hkv, 128, 128))
+    for b in range(B):
+        pos0 = 0
+        for c, L in enumerate(chunks):
+            n = pos0 + L
+            Kg = cache.k_proj.float().cpu().numpy()[b, :, :, :n].transpose(0, 2, 1).astype(np.float64)
+            V = inp["v"][b, :n].transpose(1, 0, 2).astype(np.float64)
+            own, _ = O.prefill(qts[c][b].astype(np.float64), pos0, eye, Kg, V, k, m=d_store)
+            refs[b][c] = refs[b][c] + (own,)
+            pos0 += L
     return outs, (sels, qts), refs
 
 
@@ -60,16 +85,24 @@ def _check(outs, sels, refs, out="bf16", k=96, m=None):
     protocol: the oracle's selection on the kernel's own f32 q~ equals the
     kernel's sets exactly, and against the f64 q~ every (row, head) whose
     k-th/(k+1)-th magnitude gap exceeds 1e-5 of the largest must match."""
-    tol = TOL_BF16_OUT if out == "bf16" else TOL_F32_OUT
     sels, qts = sels
     near = 0
     for c in range(len(outs)):
         for b in range(outs[c].shape[0]):
-            ref_out, ref_sel, ref_qt = refs[b][c]
-            err = rel_err_rows(outs[c][b], ref_out)
-            assert np.max(err) <= tol, f"chunk {c} seq {b}: max rel err {np.max(err):.3e} at {np.argmax(err)}"
+            ref_out, ref_sel, ref_qt, own = refs[b][c]
             assert np.isfinite(qts[c][b]).all(), "every live row's q~ exported"
+            qerr = np.abs(qts[c][b] - ref_qt).max(axis=-1) / np.abs(ref_qt).max(axis=-1)
+            assert qerr.max() <= TOL_QPROJ, f"chunk {c} seq {b}: q~ rel err {qerr.max():.3e}"
             near += check_selection(sels[c][b], qts[c][b], ref_sel, ref_qt, k, m)
+            err = rel_err_rows(outs[c][b], ref_out)
+            if out == "bf16":
+                assert np.max(err) <= TOL_BF16_OUT, f"chunk {c} seq {b}: max rel err {np.max(err):.3e}"
+                continue
+            err_own = rel_err_rows(outs[c][b], own)
+            assert np.max(err_own) <= TOL_F32_OWN, f"chunk {c} seq {b}: vs own state {np.max(err_own):.3e}"
+            same = np.all(sels[c][b] == ref_sel, axis=(-1, -2))          # rows whose heads all agree
+            assert same.mean() >= 0.9, f"chunk {c} seq {b}: only {same.mean():.2f} of the rows match the f64 sets"
+            assert np.max(err[same]) <= TOL_F32_OUT, f"chunk {c} seq {b}: end to end {np.max(err[same]):.3e}"
     return near
 
 
@@ -138,6 +171,8 @@ def test_prefill_row_matches_decode():
         ref_sel = np.stack([O.select_dims(qt[h], k) for h in range(Hq)])
         check_selection(sel.cpu().numpy()[0, p], qp.cpu().numpy()[0, p], ref_sel, qt, k)
         check_selection(sd.cpu().numpy()[0], qd.cpu().numpy()[0], ref_sel, qt, k)
+        # two GPU paths, each within its own-state bound of the oracle (3e-5 and
+        # 1e-5) and possibly apart at a near-tie selection: 1e-4 between them
         err = rel_err_rows(od.cpu().numpy()[0].astype(np.float64), o.cpu().numpy()[0, p].astype(np.float64))
         assert np.max(err) <= 1e-4, (p, np.max(err))
 
