@@ -697,9 +697,11 @@ class H2OBench:
         qo = B * Hq * 128 * 2 * 2
         return attn + scores + h2o + move + append + qo
 
-    def report(self, W: int, hbm_peak: float) -> dict:
+    def report(self, W: int, hbm_peak: float, max_reps: int = 0) -> dict:
         """Steady state over the whole absolute-length range, from T_abs =
-        budget + (warm-up steps) to T_end: 256-step graphs replayed back to back."""
+        budget + (warm-up steps) to T_end: 256-step graphs replayed back to back
+        (max_reps > 0 limits the replays, for profiling runs; the line reports
+        the range it ran)."""
         torch, wl = self.torch, self.wl
         G = wl["Hq"] // wl["Hkv"]
         for _ in range(W):
@@ -720,6 +722,8 @@ class H2OBench:
         torch.cuda.synchronize()
         t_abs0 = wl["budget"] + self.n_steps                               # tokens seen so far
         reps = max(1, (wl["T_end"] - t_abs0) // self.GRAPH_STEPS)
+        if max_reps > 0:
+            reps = min(reps, max_reps)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda._sleep(int(2e6))                  # the host submits the replays while the GPU sleeps
         e0.record()
@@ -872,6 +876,8 @@ def main():
                          "prefill (chunked prefill, full and truncated cache), h2o (truncated cache + H2O steady "
                          "state)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--h2o-reps", type=int, default=0,
+                    help="limit the H2O line's 256-step graph replays (profiling runs; default: the whole range)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup()
@@ -1014,7 +1020,7 @@ def main():
         torch.cuda.empty_cache()
     if "h2o" in extras:
         hb = H2OBench(H2O_WL, P)
-        line["truncated_h2o"] = hb.report(W, hbm_peak)
+        line["truncated_h2o"] = hb.report(W, hbm_peak, args.h2o_reps)
         del hb
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
