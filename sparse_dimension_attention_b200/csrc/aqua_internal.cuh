@@ -293,6 +293,14 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* addr
                : "r"(smem_u32(addr)));
 }
 
+// 8x8 b16 matrix held one row per four lanes (lane i: row i / 4, elements
+// 2 (i % 4) and 2 (i % 4) + 1) -> its transpose in the same layout
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 // D = A (16x16 bf16, row) * B (16x8 bf16, col) + D, f32 accumulators
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(

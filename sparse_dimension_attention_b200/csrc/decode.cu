@@ -845,22 +845,20 @@ __device__ __forceinline__ void issue_v_tile(unsigned char* st, const CUtensorMa
   tma_load_2d(st + VHALF, tmap, 64, row, bar, pol);
 }
 
-// Scores of a warp's 16 tokens over NKS k-steps of 16 union rows: even k-steps
-// accumulate into (c0, c1), odd ones into (d0, d1) (two chains per n-tile).
+// Scores S^T of a warp's 16 tokens (MMA rows) over NKS k-steps of 16 union
+// rows: A = the K~ tile read transposed, B = the masked queries (qb); even
+// k-steps accumulate into c, odd ones into d (two chains).
 template <int NKS>
-__device__ __forceinline__ void score_ksteps(const unsigned char* a0, const uint32_t (&afr)[8][4], float (&c0)[4],
-                                             float (&c1)[4], float (&d0)[4], float (&d1)[4]) {
+__device__ __forceinline__ void score_ksteps(const unsigned char* a0, const uint32_t (&qb)[8][2], float (&c)[4],
+                                             float (&d)[4]) {
 #pragma unroll
   for (int kk = 0; kk < NKS; ++kk) {
-    uint32_t bfr[4];
-    ldsm_x4_trans(bfr, a0 + kk * 16 * KROW_BF16);
-    if (kk & 1) {
-      mma_bf16_16816(d0, afr[kk], bfr[0], bfr[1]);
-      mma_bf16_16816(d1, afr[kk], bfr[2], bfr[3]);
-    } else {
-      mma_bf16_16816(c0, afr[kk], bfr[0], bfr[1]);
-      mma_bf16_16816(c1, afr[kk], bfr[2], bfr[3]);
-    }
+    uint32_t ka[4];
+    ldsm_x4_trans(ka, a0 + kk * 16 * KROW_BF16);
+    if (kk & 1)
+      mma_bf16_16816(d, ka, qb[kk][0], qb[kk][1]);
+    else
+      mma_bf16_16816(c, ka, qb[kk][0], qb[kk][1]);
   }
 }
 
@@ -1035,19 +1033,25 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   }
 
   // ======================= consumer warps =======================
-  // A-operand rows: row h < G carries the bf16 high part of head h, row 8 + h
-  // its low part; the thread holding row grp also holds row grp + 8.
+  // Transposed products: S^T = K~^T Q~m^T and O^T = V^T P^T, with the warp's
+  // 16 tokens as the MMA rows (M = 16) and 8 columns of (head, part) pairs:
+  // column 2h carries head h's bf16 high part, column 2h + 1 its low part.
+  // The thread of fragment column pair q4 thus holds both parts of head q4
+  // (and adds them itself); P's fragment, laid out as the scores' accumulator
+  // (tokens x columns), becomes the B operand of the P V product by one 8x8
+  // transpose per 8 tokens.
   const int grp = lane >> 2, q4 = lane & 3;    // mma fragment coordinates
   const int tb = 16 * warp;                     // this warp's tokens in every tile
-  const bool head_row = grp < G;
-  uint32_t afr[8][4];
-  float o[16][4];
-  float mu = -INFINITY, ell = 0.f;
+  const bool head_ok = q4 < G;                 // head q4 exists
+  uint32_t qb[8][2];                            // scores' B operand: column grp, union rows 16 kk + 2 q4 (+1, +8, +9)
+  float o[8][4];                                // O^T: dims 16 j + grp (+ 8) x columns 2 q4, 2 q4 + 1
+  float mu = -INFINITY;                         // running max of head q4 (the same in all its lanes)
+  float ell = 0.f;                              // this thread's share of head q4's sum (reduced at segment ends)
   int cur_u = -1, nks = 0;
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) afr[kk][0] = afr[kk][1] = afr[kk][2] = afr[kk][3] = 0u;
+  for (int kk = 0; kk < 8; ++kk) qb[kk][0] = qb[kk][1] = 0u;
 #pragma unroll
-  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   // Every consumer warp walks the schedule itself, so all warps agree on the
   // segment ends (where they synchronise) whatever happens to the data.  A
   // warp whose wait runs out records the error, stops computing and keeps
@@ -1074,9 +1078,10 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     unsigned char* st = smem + (size_t)s * S::STAGE;
     const unsigned char* ks_base = st + 2 * S::VHALF;
 
-    // A operand: the masked queries of the unit in the order of the tile's K~
+    // B operand: the masked queries of the unit in the order of the tile's K~
     // rows, dimension order on the tiles loaded before the wait, union order
-    // (from the rows' padding) from the first tile after them on
+    // (from the rows' padding) from the first tile after them on.  Column grp
+    // is head grp >> 1, part grp & 1.
     const bool nat0 = it == 0 && n_nat > 0;
     const bool comp0 = it == n_nat && n_nat > 0;
     if (!dead && ((hh.flags & kFirst) || comp0)) {
@@ -1084,23 +1089,26 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         cur_u = hh.u;
         const int nrow = nat0 ? p.d_store : hh.nU;
         nks = (nrow + 15) / 16;
-        // source of row col's query for head grp: dimension-order array or the row padding
-        const float* qsrc = nat0 ? p.qmn + (size_t)hh.u * D * G + grp
-                                 : reinterpret_cast<const float*>(ks_base + 2 * TT + grp * 4);
+        const int qh = grp >> 1;
+        const bool col_ok = qh < G, low = (grp & 1) != 0;
+        // source of row r's query for head qh: dimension-order array or the row padding
+        const float* qsrc = nat0 ? p.qmn + (size_t)hh.u * D * G + qh
+                                 : reinterpret_cast<const float*>(ks_base + 2 * TT) + qh;
         const int qstride = nat0 ? G : KROW_BF16 / 4;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            float hi2[2], lo2[2];
+            float v2[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int col = kk * 16 + half * 8 + 2 * q4 + e;
-              const float x = (head_row && col < nrow) ? qsrc[col * qstride] : 0.f;
-              split_bf16(x, hi2[e], lo2[e]);
+              const int r = kk * 16 + half * 8 + 2 * q4 + e;
+              const float x = (col_ok && r < nrow) ? qsrc[r * qstride] : 0.f;
+              float hi, lo;
+              split_bf16(x, hi, lo);
+              v2[e] = low ? lo : hi;
             }
-            afr[kk][half * 2] = pack_bf16(hi2[0], hi2[1]);       // row grp
-            afr[kk][half * 2 + 1] = pack_bf16(lo2[0], lo2[1]);   // row grp + 8
+            qb[kk][half] = pack_bf16(v2[0], v2[1]);
           }
         }
       }
@@ -1109,7 +1117,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       mu = -INFINITY;
       ell = 0.f;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     }
 
     bool wrote_smem = false;
@@ -1125,90 +1133,84 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         wrote_smem = true;
         __syncwarp();
       }
-      // ---- scores S[row][token] for this warp's 16 tokens (two accumulator
-      // chains per n-tile: even and odd k-steps)
-      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-      float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+      const int mtx = lane >> 3, r8 = lane & 7;
+      // ---- S^T for this warp's 16 tokens
+      float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
       {
-        const int mtx = lane >> 3, r8 = lane & 7;
-        const unsigned char* a0 = ks_base + ((mtx & 1) * 8 + r8) * KROW_BF16 + (tb + (mtx >> 1) * 8) * 2;
+        // matrices: (rows 0-7, tokens 0-7), (rows 0-7, tokens 8-15), (rows 8-15, tokens 0-7), (rows 8-15, tokens 8-15)
+        const unsigned char* a0 = ks_base + ((mtx >> 1) * 8 + r8) * KROW_BF16 + (tb + (mtx & 1) * 8) * 2;
         // the k-steps as straight-line code for the union size (no test between the MMAs)
         switch (nks) {
-          case 8: score_ksteps<8>(a0, afr, c0, c1, d0, d1); break;
-          case 7: score_ksteps<7>(a0, afr, c0, c1, d0, d1); break;
-          case 6: score_ksteps<6>(a0, afr, c0, c1, d0, d1); break;
-          case 5: score_ksteps<5>(a0, afr, c0, c1, d0, d1); break;
-          case 4: score_ksteps<4>(a0, afr, c0, c1, d0, d1); break;
-          case 3: score_ksteps<3>(a0, afr, c0, c1, d0, d1); break;
-          case 2: score_ksteps<2>(a0, afr, c0, c1, d0, d1); break;
-          default: score_ksteps<1>(a0, afr, c0, c1, d0, d1); break;
+          case 8: score_ksteps<8>(a0, qb, c, d); break;
+          case 7: score_ksteps<7>(a0, qb, c, d); break;
+          case 6: score_ksteps<6>(a0, qb, c, d); break;
+          case 5: score_ksteps<5>(a0, qb, c, d); break;
+          case 4: score_ksteps<4>(a0, qb, c, d); break;
+          case 3: score_ksteps<3>(a0, qb, c, d); break;
+          case 2: score_ksteps<2>(a0, qb, c, d); break;
+          default: score_ksteps<1>(a0, qb, c, d); break;
         }
       }
-      // high + low parts; tokens tb + {2q, 2q+1, 8+2q, 9+2q}
-      float sc[4] = {(c0[0] + c0[2]) + (d0[0] + d0[2]), (c0[1] + c0[3]) + (d0[1] + d0[3]),
-                     (c1[0] + c1[2]) + (d1[0] + d1[2]), (c1[1] + c1[3]) + (d1[1] + d1[3])};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int tok = tb + (e >> 1) * 8 + 2 * q4 + (e & 1);
-        if (tok >= hh.nvalid) sc[e] = -INFINITY;
-      }
-      if (p.scores_out != nullptr && head_row) {
-        const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
-        float* dst = p.scores_out + ((size_t)b * p.Hq + g * G + grp) * p.Tcap + hh.t0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int tok = tb + (e >> 1) * 8 + 2 * q4 + (e & 1);
-          if (tok < hh.nvalid) dst[tok] = sc[e] * kLn2;
-        }
-      }
-      // ---- online softmax over this warp's tokens (lazy rescale)
-      float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const bool upd = head_row && mx > mu + kLazyRescale;
-      if (__any_sync(0xffffffffu, upd)) {
-        float alpha = 1.f;
-        if (upd) {
-          alpha = exp2f(mu - mx);
-          mu = mx;
-        }
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          o[n][0] *= alpha;
-          o[n][1] *= alpha;
-          o[n][2] *= alpha;
-          o[n][3] *= alpha;
-        }
-        ell *= alpha;
-      }
-      float pv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) pv[e] = head_row ? exp2f(sc[e] - mu) : 0.f;
-      float rs = (pv[0] + pv[1]) + (pv[2] + pv[3]);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-      ell += rs;
-      // A fragments of P: high parts in row grp, low parts in row grp + 8
-      float ph[4], pl[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) split_bf16(pv[e], ph[e], pl[e]);
-      const uint32_t pa[4] = {pack_bf16(ph[0], ph[1]), pack_bf16(pl[0], pl[1]), pack_bf16(ph[2], ph[3]),
-                              pack_bf16(pl[2], pl[3])};
-      // ---- o += P V over 128 dims (16 n-tiles of 8; zeros past dv with projected values)
+      // A operand of P V: the V tile read transposed (dims x tokens), loaded
+      // ahead of the softmax; matrices (tokens 0-7, dims 0-7), (tokens 0-7,
+      // dims 8-15), (tokens 8-15, dims 0-7), (tokens 8-15, dims 8-15) of each
+      // 16-dim block
+      uint32_t va[8][4];
       {
-        const int mtx = lane >> 3, r8 = lane & 7;
-        const int tok = tb + (mtx & 1) * 8 + r8;
+        const int tok = tb + (mtx >> 1) * 8 + r8;
         const unsigned char* vrow = st + tok * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const int dim0 = 16 * j + (mtx >> 1) * 8;
+          const int dim0 = 16 * j + (mtx & 1) * 8;
           const int chunk = (dim0 & 63) >> 3;
-          uint32_t bfr[4];
-          ldsm_x4_trans(bfr, vrow + (dim0 >> 6) * S::VHALF + ((chunk ^ (tok & 7)) << 4));
-          mma_bf16_16816(o[2 * j], pa, bfr[0], bfr[1]);
-          mma_bf16_16816(o[2 * j + 1], pa, bfr[2], bfr[3]);
+          ldsm_x4_trans(va[j], vrow + (dim0 >> 6) * S::VHALF + ((chunk ^ (tok & 7)) << 4));
         }
       }
+      // head q4 at tokens tb + grp and tb + grp + 8: high + low parts
+      float sc[2] = {(c[0] + c[1]) + (d[0] + d[1]), (c[2] + c[3]) + (d[2] + d[3])};
+      if (tb + grp >= hh.nvalid) sc[0] = -INFINITY;
+      if (tb + grp + 8 >= hh.nvalid) sc[1] = -INFINITY;
+      if (p.scores_out != nullptr && head_ok) {
+        const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
+        float* dst = p.scores_out + ((size_t)b * p.Hq + g * G + q4) * p.Tcap + hh.t0 + tb + grp;
+        if (tb + grp < hh.nvalid) dst[0] = sc[0] * kLn2;
+        if (tb + grp + 8 < hh.nvalid) dst[8] = sc[1] * kLn2;
+      }
+      // ---- online softmax: the running max is raised only when a score
+      // exceeds it by 2^8 (exact; it avoids rescaling), and the warp's maximum
+      // over its tokens is formed only then
+      const bool over = head_ok && fmaxf(sc[0], sc[1]) > mu + kLazyRescale;
+      if (__any_sync(0xffffffffu, over)) {
+        float mx = fmaxf(sc[0], sc[1]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (head_ok && mx > mu + kLazyRescale) {
+          const float alpha = exp2f(mu - mx);
+          mu = mx;
+#pragma unroll
+          for (int n = 0; n < 8; ++n) {
+            o[n][0] *= alpha;
+            o[n][1] *= alpha;
+            o[n][2] *= alpha;
+            o[n][3] *= alpha;
+          }
+          ell *= alpha;
+        }
+      }
+      const float p0 = head_ok ? exp2f(sc[0] - mu) : 0.f;
+      const float p1 = head_ok ? exp2f(sc[1] - mu) : 0.f;
+      ell += p0 + p1;
+      float h0, l0, h1, l1;
+      split_bf16(p0, h0, l0);
+      split_bf16(p1, h1, l1);
+      // P as (tokens x columns) accumulator-layout fragments, transposed into
+      // the B operand (tokens x columns, column-major)
+      const uint32_t pb0 = movmatrix_trans(pack_bf16(h0, l0));
+      const uint32_t pb1 = movmatrix_trans(pack_bf16(h1, l1));
+      // ---- O^T += V^T P^T over 128 dims (zeros past dv with projected values)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mma_bf16_16816(o[j], va[j], pb0, pb1);
     }
     if (wrote_smem) fence_proxy_async_smem();
     __syncwarp();
@@ -1216,15 +1218,21 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
 
     if (!(hh.flags & kLast)) continue;
 
-    // ---- end of a segment: merge the warps' (m, l, o), then output or partial
-    if (head_row) {
+    // ---- end of a segment: the warp's sum of head q4, then merge the warps'
+    // (m, l, o) and output or partial
+    ell += __shfl_xor_sync(0xffffffffu, ell, 4);
+    ell += __shfl_xor_sync(0xffffffffu, ell, 8);
+    ell += __shfl_xor_sync(0xffffffffu, ell, 16);
+    if (head_ok) {
+      float* rw = red + ((size_t)warp * G + q4) * D + grp;
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
-        *reinterpret_cast<float2*>(red + ((size_t)warp * G + grp) * D + 8 * n + 2 * q4) =
-            make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
-      if (q4 == 0) {
-        mlb[(warp * G + grp) * 2 + 0] = mu;
-        mlb[(warp * G + grp) * 2 + 1] = ell;
+      for (int j = 0; j < 8; ++j) {
+        rw[16 * j] = o[j][0] + o[j][1];
+        rw[16 * j + 8] = o[j][2] + o[j][3];
+      }
+      if (grp == 0) {
+        mlb[(warp * G + q4) * 2 + 0] = mu;
+        mlb[(warp * G + q4) * 2 + 1] = ell;
       }
     }
     named_bar_sync(1, NCT);
