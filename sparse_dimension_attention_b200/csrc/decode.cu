@@ -1131,8 +1131,11 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
                 make_uint4(0, 0, 0, 0);
         }
         wrote_smem = true;
-        __syncwarp();
       }
+      // ldmatrix, mma.sync and movmatrix below need the whole warp converged:
+      // the query build above and the zeroing take lane-dependent paths (for
+      // G < 4 the lanes of absent heads load nothing)
+      __syncwarp();
       const int mtx = lane >> 3, r8 = lane & 7;
       // ---- S^T for this warp's 16 tokens
       float c[4] = {0.f, 0.f, 0.f, 0.f}, d[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1205,7 +1208,9 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
       split_bf16(p0, h0, l0);
       split_bf16(p1, h1, l1);
       // P as (tokens x columns) accumulator-layout fragments, transposed into
-      // the B operand (tokens x columns, column-major)
+      // the B operand (tokens x columns, column-major); the lanes of absent
+      // heads (G < 4) took other paths above
+      __syncwarp();
       const uint32_t pb0 = movmatrix_trans(pack_bf16(h0, l0));
       const uint32_t pb1 = movmatrix_trans(pack_bf16(h1, l1));
       // ---- O^T += V^T P^T over 128 dims (zeros past dv with projected values)
