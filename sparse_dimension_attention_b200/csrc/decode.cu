@@ -101,13 +101,16 @@ __device__ __forceinline__ int kv_len(const DecodeParams& p, int b) {
 }
 
 // Called once per attention CTA (thread 0) after all of its work: the last CTA
-// of the grid advances the lengths of a step with a fused append.
+// of the grid advances the lengths of a step with a fused append.  The
+// increments are atomic adds whose results nobody reads (reductions): the
+// thread issues all of them back to back instead of waiting on a load before
+// each store, which put B memory round trips at the end of every step.
 __device__ __forceinline__ void step_done(const DecodeParams& p) {
   if (p.len_add == 0) return;
   if (atom_add_acq_rel_gpu(p.ctrl + kCtrlStepTicket, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
     for (int bb = 0; bb < p.B; ++bb) {
-      p.len_w[bb] += p.len_add;
-      if (p.n_abs) p.n_abs[bb] += p.len_add;
+      atomicAdd(p.len_w + bb, p.len_add);
+      if (p.n_abs) atomicAdd(p.n_abs + bb, p.len_add);
     }
     p.ctrl[kCtrlStepTicket] = 0;
   }
