@@ -646,6 +646,47 @@ __device__ bool make_schedule(const DecodeParams& p, long long* scratch, long lo
   return S.my_end > S.my_start;
 }
 
+// L2 prefetch of the first NSTAGE tiles this CTA most likely owns, issued
+// while the schedule (which needs every length) is still being built, so the
+// first tiles' copies find their data in L2.  The guess takes every sequence
+// to have sequence 0's length, which makes it exact for equal lengths; a
+// wrong guess only spends bandwidth.  Thread tid prefetches K~ row tid % D of
+// guessed tile tid / D (the row's tokens of that tile), and row 0's thread
+// also the tile's V rows.  Every address stays inside the unit's slots:
+// u < B Hkv, r < d_store, t0 < T <= Tcap and t0 + ntok <= Tcap; the sizes
+// are multiples of 32 bytes and the offsets of 32 bytes (Tcap, t0 and dv are
+// multiples of 16 elements).
+template <int TT, int NSTG>
+__device__ __forceinline__ void prefetch_first_tiles_l2(const DecodeParams& p, int len0, int tid) {
+  const int T = min(max(len0, 0) + p.len_add, p.Tcap);
+  const int nt = (T + TT - 1) / TT;
+  const int n_units = p.B * p.Hkv;
+  const int j = tid / D, r = tid % D;                  // tile j of the first NSTG, K~ row r
+  // only with no more units than SMs (n_late > 0): measured faster there (Llama
+  // decode, long context) and slower with 256 units under H2O updates
+  if (p.n_late == 0 || nt == 0 || j >= NSTG) return;
+  const long long unitpos = (long long)nt * kTilePos + kBoundaryPos;   // positions of one unit
+  const long long NV = (long long)n_units * unitpos;
+  if (NV > 0x7fffffffLL) return;                      // 32-bit position arithmetic below
+  const Split sp = make_split(NV, gridDim.x, p.n_late);
+  if ((int)blockIdx.x >= sp.C) return;
+  const int a = (int)split_start((int)blockIdx.x, sp);   // this CTA's first position
+  const int u = a / (int)unitpos;
+  if (u >= n_units) return;
+  const int off = a - u * (int)unitpos;
+  const int t = (off > kBoundaryPos ? (off - kBoundaryPos + kTilePos - 1) / kTilePos : 0) + j;
+  if (t >= nt) return;
+  const int t0 = t * TT;
+  const int ntok = min(TT, p.Tcap - t0);
+  const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(p.kproj);
+  if (r < p.d_store) prefetch_l2_bulk(kp + ((size_t)u * p.d_store + r) * p.Tcap + t0, (uint32_t)ntok * 2u);
+  if (r == 0) {
+    const int vcols = p.dv > 0 ? p.dv : D;
+    const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(p.v);
+    prefetch_l2_bulk(vp + ((size_t)u * p.Tcap + t0) * vcols, (uint32_t)(ntok * vcols * 2));
+  }
+}
+
 // Walks the units of this CTA's tile range; one instance per producer warp.
 struct UnitWalker {
   int u = 0, b = 0, Tb = 0, nU = 0, nseg = 0, cf = 0;
@@ -882,6 +923,7 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) s_last[1] = 0;
+  const int len0 = p.len[0];   // for the L2 prefetch below; the load overlaps the zeroing
 
   // the K~ rows of every stage start zeroed: union padding rows and never-copied
   // tokens must be finite (the V halves are rewritten whole by every tile copy)
@@ -890,6 +932,8 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
     const int s = i / KQ;
     reinterpret_cast<uint4*>(smem + (size_t)s * S::STAGE + 2 * S::VHALF)[i - s * KQ] = make_uint4(0, 0, 0, 0);
   }
+  static_assert(NTHREADS_BF16 >= NSTAGE * D, "one thread per prefetched K~ row");
+  prefetch_first_tiles_l2<TT, NSTAGE>(p, len0, tid);
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       // arrivals: one cp.async arrival per producer thread + the V tensor-copy arrival
