@@ -155,3 +155,84 @@ def test_boundary_positions_balance_the_split():
         crosses = any(s < b < e for b in starts)
         (two if crosses else one).append(e - s)
     assert two and one and max(two) < max(one)
+
+
+def guess_first_tile(len0, len_add, Tcap, n_units, grid, n_late, c, TT=128):
+    """The attention kernel's guess of CTA c's first tile for its L2 prefetch
+    (prefetch_first_tiles_l2 in csrc/decode.cu): every sequence taken to have
+    sequence 0's length.  Returns (unit, tile within the unit, tiles per unit)
+    or None when the kernel prefetches nothing."""
+    T = min(max(len0, 0) + len_add, Tcap)
+    nt = (T + TT - 1) // TT
+    if nt == 0:
+        return None
+    unitpos = nt * P + W
+    NV = n_units * unitpos
+    if NV > 0x7fffffff:
+        return None
+    C, c0, E = make_split(NV, grid, P, n_late, LATE)
+    if c >= C:
+        return None
+    a = split_start(c, NV, C, c0, E)
+    u = a // unitpos
+    if u >= n_units:
+        return None
+    off = a - u * unitpos
+    t = (off - W + P - 1) // P if off > W else 0
+    return u, t, nt
+
+
+def test_prefetch_guess_is_exact_for_equal_lengths():
+    """With equal lengths the guessed first tile is the CTA's real first tile."""
+    rng = random.Random(1)
+    for _ in range(300):
+        n_units = rng.choice([1, 2, 8, 64, 100, 256])
+        T = rng.randint(1, 20000)
+        grid, n_late = rng.choice([148, 64, 16]), rng.choice([0, n_units])
+        nt = (T + 127) // 128
+        ranges, _, _, C = split([nt] * n_units, grid, n_late=n_late)
+        for c, (s, e) in enumerate(ranges):
+            if s == e:
+                continue
+            g = guess_first_tile(T - 1, 1, 1 << 20, n_units, grid, n_late, c)
+            assert g is not None
+            u, t, _ = g
+            assert u * nt + t == s, (n_units, T, grid, n_late, c)
+
+
+def test_prefetch_addresses_stay_inside_the_unit():
+    """Every byte range the guess prefetches (K~ row r of tiles t..t+2, and the
+    tiles' V rows) lies inside the unit's slots, starts on a 16-byte boundary
+    and has a positive multiple of 16 bytes, whatever the device length."""
+    rng = random.Random(2)
+    for _ in range(3000):
+        Tcap = 16 * rng.randint(1, 400)
+        len0 = rng.choice([-5, 0, 1, rng.randint(0, Tcap), Tcap, Tcap + 7, 10 ** 9])
+        len_add = rng.choice([0, 1])
+        n_units = rng.choice([1, 3, 8, 64, 256])
+        d_store = rng.randint(1, 128)
+        vcols = rng.choice([128, 16 * rng.randint(1, 8)])
+        grid = rng.randint(1, 160)
+        n_late = rng.choice([0, n_units])
+        for c in range(grid):
+            g = guess_first_tile(len0, len_add, Tcap, n_units, grid, n_late, c)
+            if g is None:
+                continue
+            u, t, nt = g
+            assert 0 <= u < n_units
+            for j in range(3):
+                if t + j >= nt:
+                    continue
+                t0 = (t + j) * 128
+                ntok = min(128, Tcap - t0)
+                assert 0 < ntok and t0 + ntok <= Tcap
+                for r in range(d_store):
+                    start = ((u * d_store + r) * Tcap + t0) * 2
+                    size = ntok * 2
+                    row0 = (u * d_store + r) * Tcap * 2
+                    assert row0 <= start and start + size <= row0 + Tcap * 2
+                    assert start % 16 == 0 and size % 16 == 0
+                vstart = (u * Tcap + t0) * vcols * 2
+                vsize = ntok * vcols * 2
+                assert u * Tcap * vcols * 2 <= vstart and vstart + vsize <= (u + 1) * Tcap * vcols * 2
+                assert vstart % 16 == 0 and vsize % 16 == 0
