@@ -619,6 +619,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // work), so a timeout never leaves a partner blocked at the barrier.
     float mu = -INFINITY, ell = 0.f;
     const int cbase = wg * 64;
+    const int pair_bar = 2 + (warp & 3);            // the row's two threads: warps w and w + 4
+    // the row maximum exchange of every tile, [tile parity][2 halves][128 rows]:
+    // in the P part-2 area (free after the prologue), past the selection's counts
+    float* xmax = reinterpret_cast<float*>(smem + S::OFF_PP + 4096);
     if (!ok) *abort_flag = 1;
     for (int j = 0; j < n_tiles; ++j) {
       const int t0 = j * PN;
@@ -636,13 +640,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < 64; ++c)
             if (tc0 + c > pos_r) s[c] = -INFINITY;
         }
+        float m8[8];                                // eight independent chains
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 8; ++c) m8[c] = s[c];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      // row maximum over both column halves
-      red[wg * 128 + r] = mx;
-      named_bar_sync(1, kSoftThreads);
-      mx = fmaxf(mx, red[(wg ^ 1) * 128 + r]);
+      // row maximum over both column halves (the buffer alternates by tile, so a
+      // value is never overwritten before the partner has read it)
+      float* xm = xmax + (j & 1) * 256;
+      xm[wg * 128 + r] = mx;
+      named_bar_sync(pair_bar, 64);
+      mx = fmaxf(mx, xm[(wg ^ 1) * 128 + r]);
       if (!ok) {
         *abort_flag = 1;
         continue;
@@ -656,7 +666,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // P = 2^(s - mu) as bf16 high + low parts, computed while the previous P V may still run;
       // the row sum takes the values exactly as the tensor cores will see them
       uint32_t hw[32], lw[32];
-      float rs0 = 0.f, rs1 = 0.f;
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // eight independent chains
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         const float p0 = ex2_ftz(s[c] - mu_new);
@@ -664,11 +674,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         uint32_t h0, l0, h1, l1;
         split_trunc(p0, h0, l0);
         split_trunc(p1, h1, l1);
-        rs0 += __uint_as_float(h0) + __uint_as_float(l0);
-        rs1 += __uint_as_float(h1) + __uint_as_float(l1);
+        rs[(c >> 1) & 7] += (__uint_as_float(h0) + __uint_as_float(l0)) + (__uint_as_float(h1) + __uint_as_float(l1));
         hw[c >> 1] = pack_hi_halves(h0, h1);
         lw[c >> 1] = pack_hi_halves(l0, l1);
       }
+      const float rs0 = (rs[0] + rs[1]) + (rs[2] + rs[3]), rs1 = (rs[4] + rs[5]) + (rs[6] + rs[7]);
       // the previous P V must be complete before O is rescaled or P is rewritten
       if (j > 0) {
         ok = wait_or_abort(&bars[BAR_O], (j - 1) & 1, abort_flag);
