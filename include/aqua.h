@@ -9,8 +9,8 @@
  * by softmax and the weighted sum of the unprojected values.  Sources: the
  * paper's abstract; edgentiq blog "How AQUA Works: A Two-Phase Approach" and
  * "AQUA-Memory: Dual Savings" (statically truncated cache); H2O eviction is
- * named in the abstract ("synergistically accelerate existing token eviction
- * methods like H2O").
+ * named in the abstract (AQUA combines with token eviction methods such as H2O
+ * and speeds them up).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers unless stated otherwise, owned by
@@ -126,8 +126,8 @@ AQUA_API int aqua_version(void);
 AQUA_API int aqua_status(const aqua_cache* cache, int* status_out, aqua_stream_t stream);
 
 /*
- * Offline calibration (abstract: "a universal, language agnostic projection
- * matrix via SVD on a calibration dataset"; edgentiq, "Offline Projection
+ * Offline calibration (abstract: one projection matrix, computed offline
+ * by an SVD of calibration data and shared across languages; edgentiq, "Offline Projection
  * Computation").  X [n][d] f32 stacks calibration queries and keys (not
  * centred).  Writes P [d][d] f32 whose COLUMNS are the right singular vectors
  * of X ordered by descending singular value, and sigma [d] f32.  Each column's
@@ -140,7 +140,7 @@ AQUA_API int aqua_calibrate(const float* X, int n, int d, float* P_out, float* s
                    void* workspace, size_t workspace_bytes, aqua_stream_t stream);
 
 /*
- * Key projection and append (abstract: "project query and key vectors";
+ * Key projection and append (abstract: queries and keys are projected by P;
  * edgentiq, "Online Inference").  For every sequence b and new token l < L:
  * k~ = k_new[b][l][g] . P[g] is computed in f32, its first d_store dimensions
  * are rounded to the cache dtype (bf16: round-to-nearest-even) and written into

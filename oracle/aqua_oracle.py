@@ -96,16 +96,16 @@ def calibrate(X) -> tuple[np.ndarray, np.ndarray]:
 # ----------------------------------------------------------------------------
 
 def project(x, P) -> np.ndarray:
-    """x~ = x P for row vectors x [..., d] (abstract: "project query and key vectors")."""
+    """x~ = x P for row vectors x [..., d] (abstract: queries and keys are projected by P)."""
     return np.asarray(x, dtype=np.float64) @ np.asarray(P, dtype=np.float64)
 
 
 def select_dims(qt, k: int, m: int | None = None) -> np.ndarray:
     """Indices S of the k largest |q~_j| among j < m, ascending.
 
-    "dynamically select a sparse subset of dimensions based on the query's
-    magnitude" (abstract); "those with the highest 'magnitude' in the
-    projected query vector" (edgentiq, Online Inference).  Magnitude reading:
+    The abstract has each query keep a sparse, query-dependent subset of
+    dimensions chosen by magnitude; the blog (edgentiq, Online Inference)
+    takes the dimensions where the projected query is largest.  Magnitude reading:
     |q~_j|.  Equal magnitudes go to the lower index.  With a truncated cache
     (AQUA-Memory) only the m stored dimensions are candidates.
     """
@@ -285,8 +285,8 @@ def prefill(q, pos0: int, P, Kt, V, k: int, scale: float | None = None, m: int |
 # H2O heavy-hitter eviction on top of AQUA
 # ----------------------------------------------------------------------------
 #
-# The pages name H2O only ("synergistically accelerate existing token eviction
-# methods like H2O", abstract).  Reading taken (the plainest H2O rule):
+# The pages only name H2O (the abstract says AQUA combines with token eviction
+# methods such as H2O and speeds them up).  Reading taken (the plainest H2O rule):
 #   * per (sequence, KV head) a set of at most `budget` cached tokens;
 #   * each token carries a cumulative score: the sum, over the G query heads
 #     of its group and over every decode step since it entered, of its AQUA
@@ -376,8 +376,7 @@ def h2o_decode_step(seqs, q_b, k_new_b, v_new_b, t_abs: int, P, k: int, budget: 
 #
 # The edgentiq blog ("Validation and Generalizability") reports that choosing
 # the dimensions by the query's magnitude loses about half the information that
-# keeping a fixed leading block of dimensions loses ("halving the information
-# retention loss").  It gives no formula.  Readings taken (two losses, both
+# keeping a fixed leading block of dimensions loses.  It gives no formula.  Readings taken (two losses, both
 # zero when every dimension is kept):
 #   * query energy loss: the share of the projected query's squared norm on the
 #     dimensions left out, 1 - sum_{j in S} q~_j^2 / sum_j q~_j^2;

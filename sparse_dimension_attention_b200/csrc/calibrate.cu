@@ -2,8 +2,8 @@
 // descending singular value), computed as the eigenvectors of the Gram matrix
 // X^T X in float64 with cyclic Jacobi rotations.
 //
-// AQUA abstract ("an efficient offline step where we compute a universal,
-// language agnostic projection matrix via SVD on a calibration dataset");
+// AQUA abstract (one projection matrix, computed offline once by an SVD of
+// calibration data and shared across languages);
 // edgentiq, "Offline Projection Computation".  The right singular vectors of X
 // are the eigenvectors of X^T X and sigma_j = sqrt(lambda_j).
 #include <math.h>

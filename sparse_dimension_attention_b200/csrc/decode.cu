@@ -6,9 +6,9 @@
 // warp that appends the step's new key and value when the call carries them
 // (k~ = k P rounded to the cache type, written at slot len[b]; the attention
 // kernel's last CTA advances the lengths):
-//   q~ = q P                                  (abstract: "project query and key vectors")
+//   q~ = q P                                  (abstract: queries and keys projected by P)
 //   S_h = k largest |q~_j|, ties to lower j  (edgentiq, Online Inference: the dimensions
-//                                             with the highest "magnitude" in the projected query)
+//                                             where the projected query is largest in magnitude)
 //   U_g = union of the group's S_h and the masked, pre-scaled query rows
 //   qm[r][h] = (U_r in S_h) ? q~_h[U_r] * scale * log2(e) : 0.
 //

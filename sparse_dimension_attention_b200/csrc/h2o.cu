@@ -1,7 +1,7 @@
 // H2O heavy-hitter update on top of AQUA decode.
 //
-// The AQUA abstract names H2O ("synergistically accelerate existing token
-// eviction methods like H2O") without giving its rule; the reading taken:
+// The AQUA abstract names H2O (AQUA combines with token eviction methods such
+// as H2O and speeds them up) without giving its rule; the reading taken:
 // every cached token of a (sequence, KV head) carries a cumulative score, the
 // sum over the group's query heads and over the decode steps it has seen of
 // its AQUA softmax probability; after a step that leaves more than `budget`
