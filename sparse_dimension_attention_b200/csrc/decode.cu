@@ -751,12 +751,13 @@ struct UnitWalker {
   }
 };
 
-// Segment result (M, L per head; O unnormalised in shared memory, [G][D]) ->
-// output, or partial + ticket + merge by the unit's last CTA.  Called by all
-// consumer threads; thread idx handles (h, dim) = (idx / D, idx % D).
+// Segment result (M, L per head; O unnormalised, thread tid holding element
+// idx = tid + NCT i of [G][D] in Ov[i]) -> output, or partial + ticket +
+// merge by the unit's last CTA.  Called by all consumer threads; element idx
+// is (h, dim) = (idx / D, idx % D).
 template <int G>
 __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int tid, const float (&Mh)[G],
-                               const float (&Lh)[G], const float* Oacc, int* s_last) {
+                               const float (&Lh)[G], const float (&Ov)[(G * D + NCT - 1) / NCT], int* s_last) {
   const int b = hh.u / p.Hkv, g = hh.u % p.Hkv;
   const size_t bhq0 = (size_t)b * p.Hq + g * G;
 #pragma unroll
@@ -768,7 +769,7 @@ __device__ void finish_segment(const DecodeParams& p, const StageHdr& hh, int ti
 #pragma unroll
       for (int x = 0; x < G; ++x)
         if (x == h) lh = Lh[x];
-      const float o = Oacc[h * D + dim];
+      const float o = Ov[i];
       if (hh.seg < 0)
         store_result(p, (bhq0 + h) * D + dim, o / lh);
       else
@@ -1324,14 +1325,10 @@ __global__ void __launch_bounds__(NTHREADS_BF16, 1)
         for (int w2 = 0; w2 < NCW; ++w2) acc = fmaf(fac[w2 * G + h], red[((size_t)w2 * G + h) * D + dim], acc);
         merged[i] = acc;
       }
-    }    named_bar_sync(1, NCT);
-#pragma unroll
-    for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
-      const int idx = tid + NCT * i;
-      if (idx < G * D) red[idx] = merged[i];
     }
-    named_bar_sync(1, NCT);
-    finish_segment<G>(p, hh, tid, Mh, Lh, red, s_last);
+    // each thread passes its own merged elements on; red is next written at the
+    // following segment end, after the barrier below
+    finish_segment<G>(p, hh, tid, Mh, Lh, merged, s_last);
     named_bar_sync(1, NCT);
   }
   named_bar_sync(1, NCT);               // every consumer warp is done with this CTA's work
@@ -1636,14 +1633,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_attn_f32_kernel(DecodePara
         merged[i] = acc;
       }
     }
-    named_bar_sync(1, NCT);
-#pragma unroll
-    for (int i = 0; i < (G * D + NCT - 1) / NCT; ++i) {
-      const int idx = tid + NCT * i;
-      if (idx < G * D) red[idx] = merged[i];
-    }
-    named_bar_sync(1, NCT);
-    finish_segment<G>(p, hh, tid, m_run, l_run, red, s_last);
+    finish_segment<G>(p, hh, tid, m_run, l_run, merged, s_last);
     named_bar_sync(1, NCT);
   }
   named_bar_sync(1, NCT);               // every consumer warp is done with this CTA's work
