@@ -14,10 +14,10 @@
 //
 // decode_attn_*_kernel -- persistent, one CTA per SM.  The cached tokens of all
 // (b, g) units are cut into tiles of TT tokens and the flat tile sequence is
-// split over the CTAs by a position model (see kTilePos).  Per tile the producer warps gather the |U_g|
-// selected rows of the dimension-major K~ cache (one union read per GQA group)
-// and the V tile into shared memory with asynchronous bulk / tensor copies,
-// three stages deep.  Consumer warps compute the scores on the selected
+// split over the CTAs by a position model (see kTilePos).  Per tile the
+// producer warps gather the |U_g| selected rows of the dimension-major K~
+// cache (one union read per GQA group) and the V tile into shared memory with
+// asynchronous copies, three stages deep.  Consumer warps compute the scores on the selected
 // dimensions only, s_{h,t} = sum_r qm[r][h] K~[U_r][t], an online softmax, and
 // o_h += p_{h,t} V_t over the unprojected values (AQUA abstract; edgentiq,
 // "How AQUA Works").  A CTA that ends inside a unit writes (m, l, o) and takes
@@ -25,9 +25,10 @@
 // ever waits for another.
 //
 // bf16 caches: the consumers use the tensor cores (mma.sync m16n8k16, bf16 in,
-// f32 accumulate).  q~ and p are split into bf16 high and low parts (rows
-// 0..G-1 and 8..8+G-1 of the 16-row A operand), so the products keep ~16
-// significant bits; each warp owns 16 tokens of every tile and keeps its own
+// f32 accumulate) on the transposed products S^T = K~^T qm^T and
+// O^T += V^T P^T: each warp's 16 tokens of a tile are the 16 MMA rows, and
+// the 8 columns are (head, part) pairs, q~ and p split into bf16 high and low
+// parts, so the products keep ~16 significant bits.  Each warp keeps its own
 // running max, merged at the end of a segment.  The K~ rows are gathered with
 // 16-byte cp.async by four producer warps (many small bulk copies from one warp
 // cannot keep HBM busy); the V tile arrives by a 128B-swizzled tensor copy.
