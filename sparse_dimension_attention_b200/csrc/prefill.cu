@@ -25,8 +25,8 @@
 // computed while tile j's softmax runs (K~ and V tiles double-buffered); causal
 // mask on diagonal tiles, online softmax with a lazily raised running max, P
 // split into bf16 high/low parts written to tensor memory, O += Ph V + Pl V with
-// the A operand read from tensor memory (shared-memory bandwidth is the limit of
-// this loop: P never goes through it).
+// the A operand read from tensor memory (P never goes through shared memory).
+// The softmax warpgroups' per-tile work, not the MMAs, sets the tile time.
 #include <math.h>
 
 #include "aqua_internal.cuh"
