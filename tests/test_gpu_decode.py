@@ -281,6 +281,23 @@ def test_fused_append_equals_separate_append(kv):
     assert np.max(err) <= (TOL_F32_OUT if kv == "f32" else TOL_F32_OUT_BF16_CACHE)
 
 
+@pytest.mark.parametrize("kv,out,d_store,k,G", [
+    ("bf16", "bf16", 100, 64, 4),
+    ("bf16", "bf16", 40, 33, 2),
+    ("bf16", "bf16", 1, 1, 1),       # one stored dimension
+    ("f32", "f32", 100, 80, 4),
+])
+def test_decode_d_store_not_a_multiple_of_16(kv, out, d_store, k, G):
+    """Decode takes any d_store up to d: the union and the dimension-order tiles
+    then end inside a 16-row MMA block whose rows past d_store are never
+    copied, so they must hold zeros (or finite values multiplied by zero
+    queries)."""
+    Hkv = 2
+    cache, res, ref, lens = _decode_case(2, G * Hkv, Hkv, 700, k, kv=kv, out=out, d_store=d_store)
+    _check_outputs(res, ref, out, lens, kv=kv)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], k, d_store)
+
+
 @pytest.mark.parametrize("G,d_store,seed", [(4, None, 0), (2, 96, 1), (1, None, 2), (4, 64, 3)])
 def test_decode_bf16_mixed_lengths(G, d_store, seed):
     """Per-sequence lengths from one token to several tiles (one exactly one

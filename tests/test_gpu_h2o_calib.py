@@ -74,11 +74,13 @@ def test_h2o_decision_is_bit_exact():
         assert int(cache.len[0].item()) == min(n, budget)
 
 
-@pytest.mark.parametrize("fused", [False, True])
-def test_h2o_steps_match_oracle(fused):
+@pytest.mark.parametrize("fused,G", [(False, 4), (True, 4), (True, 2), (True, 1)])
+def test_h2o_steps_match_oracle(fused, G):
     """Truncated cache (m = 96), k = 64 within it, budget 64 = 16 recent + 48 heavy, 40 steps;
-    the step's key/value appended by aqua_project_keys or by the decode call itself."""
-    B, Hq, Hkv, T0, m, k, budget, recent, steps = 2, 8, 2, 64, 96, 64, 64, 16, 40
+    the step's key/value appended by aqua_project_keys or by the decode call
+    itself; G query heads per KV head (the update sums the group's heads)."""
+    B, Hkv, T0, m, k, budget, recent, steps = 2, 2, 64, 96, 64, 64, 16, 40
+    Hq = G * Hkv
     P64, P32, cache = _h2o_setup(B, Hq, Hkv, T0, m, budget)
     inp = synth.decode_inputs(B, Hq, Hkv, T0, bf16=True, steps=steps)
     Pt = fill_cache(cache, inp["k_hist"], inp["v_hist"], P32)
