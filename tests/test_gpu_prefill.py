@@ -132,6 +132,15 @@ def test_prefill_truncated_cache():
     _check(outs, sels, refs, k=64, m=96)
 
 
+@pytest.mark.parametrize("d_store,k", [(16, 1), (32, 32)])
+def test_prefill_narrow_truncated_cache(d_store, k):
+    """The narrowest stored widths: one 16-dim k-step of score MMAs with a
+    single selected dimension, and k = d_store (every stored dimension kept,
+    the selection's early exit on its first round)."""
+    outs, sels, refs = _prefill_case(8, 2, [150, 30], k, d_store=d_store)
+    _check(outs, sels, refs, k=k, m=d_store)
+
+
 def test_prefill_batch_of_two():
     outs, sels, refs = _prefill_case(8, 2, [70], 32, B=2)
     _check(outs, sels, refs, k=32)
