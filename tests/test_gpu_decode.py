@@ -336,6 +336,21 @@ def test_decode_bf16_more_units_than_sms():
     check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 48)
 
 
+@pytest.mark.parametrize("kv", ["bf16", "f32"])
+def test_decode_units_beyond_the_scan_threads(kv):
+    """800 (sequence, KV head) units of 1..150 tokens: more units than the
+    schedule's scan has threads (384, or 288 in the f32 kernel), so each
+    thread sums several units' tiles and positions; the projection kernel runs
+    800 CTAs."""
+    rng = np.random.default_rng(11)
+    B, Hkv = 200, 4
+    lens = [int(x) for x in rng.integers(1, 150, size=B)]
+    out = "bf16" if kv == "bf16" else "f32"
+    cache, res, ref, _ = _decode_case(B, 2 * Hkv, Hkv, max(lens) - 1, 48, kv=kv, out=out, lens=lens)
+    _check_outputs(res, ref, out, lens, kv=kv)
+    check_selection(res["sel"], res["qt"], ref["sel"], ref["qt"], 48)
+
+
 @pytest.mark.parametrize("fused", [False, True])
 def test_select_then_attend_equals_one_call(fused):
     """aqua_decode_select + aqua_decode_attend (back to back, and with a
