@@ -33,10 +33,10 @@ def test_calibration_matches_svd(n):
     assert np.all(Pg[idx, np.arange(128)] > 0)
 
 
-def _h2o_setup(B, Hq, Hkv, T0, m, budget):
+def _h2o_setup(B, Hq, Hkv, T0, m, budget, dtype=torch.bfloat16):
     P64, P32 = calib_P(Hkv)
     Tcap = (budget + 1 + 15) // 16 * 16
-    cache = aq.AquaCache(B, Hkv, Tcap, d_store=m, h2o=True)
+    cache = aq.AquaCache(B, Hkv, Tcap, d_store=m, h2o=True, dtype=dtype)
     return P64, P32, cache
 
 
@@ -74,19 +74,22 @@ def test_h2o_decision_is_bit_exact():
         assert int(cache.len[0].item()) == min(n, budget)
 
 
-@pytest.mark.parametrize("fused,G", [(False, 4), (True, 4), (True, 2), (True, 1)])
-def test_h2o_steps_match_oracle(fused, G):
+@pytest.mark.parametrize("fused,G,kv", [(False, 4, "bf16"), (True, 4, "bf16"), (True, 2, "bf16"), (True, 1, "bf16"),
+                                         (True, 4, "f32")])
+def test_h2o_steps_match_oracle(fused, G, kv):
     """Truncated cache (m = 96), k = 64 within it, budget 64 = 16 recent + 48 heavy, 40 steps;
     the step's key/value appended by aqua_project_keys or by the decode call
-    itself; G query heads per KV head (the update sums the group's heads)."""
+    itself; G query heads per KV head (the update sums the group's heads);
+    bf16 or f32 cache."""
     B, Hkv, T0, m, k, budget, recent, steps = 2, 2, 64, 96, 64, 64, 16, 40
     Hq = G * Hkv
-    P64, P32, cache = _h2o_setup(B, Hq, Hkv, T0, m, budget)
-    inp = synth.decode_inputs(B, Hq, Hkv, T0, bf16=True, steps=steps)
+    dt = torch.bfloat16 if kv == "bf16" else torch.float32
+    P64, P32, cache = _h2o_setup(B, Hq, Hkv, T0, m, budget, dtype=dt)
+    inp = synth.decode_inputs(B, Hq, Hkv, T0, bf16=(kv == "bf16"), steps=steps)
     Pt = fill_cache(cache, inp["k_hist"], inp["v_hist"], P32)
     # oracle state after the same warm-up
     seqs = [[O.H2OSeq(pos=list(range(T0)), score=[0.0] * T0,
-                      kt=list(O.build_key_cache(inp["k_hist"][b, :, g][:, None], P64[g][None], "bf16", m)[:, 0]),
+                      kt=list(O.build_key_cache(inp["k_hist"][b, :, g][:, None], P64[g][None], kv, m)[:, 0]),
                       v=list(inp["v_hist"][b, :, g].astype(np.float64)))
              for g in range(Hkv)] for b in range(B)]
     sc = torch.zeros((B, Hq, cache.Tcap), dtype=torch.float32, device="cuda")
@@ -95,13 +98,13 @@ def test_h2o_steps_match_oracle(fused, G):
     ws = torch.zeros(aq.aqua_decode_workspace_size(cache.desc, Hq), dtype=torch.uint8, device="cuda")
     ev = torch.empty((B, Hkv), dtype=torch.int32, device="cuda")
     for s in range(steps):
-        kn, vn = tdev(inp["k_new"][s], torch.bfloat16), tdev(inp["v_new"][s], torch.bfloat16)
+        kn, vn = tdev(inp["k_new"][s], dt), tdev(inp["v_new"][s], dt)
         if fused:
-            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], torch.bfloat16), Pt, Hq, k, out, ws, scores_out=sc,
+            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], dt), Pt, Hq, k, out, ws, scores_out=sc,
                                 lse_out=lse, k_new=kn, v_new=vn)
         else:
             aq.aqua_project_keys(cache.desc, kn[:, None], vn[:, None], Pt, 1)
-            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], torch.bfloat16), Pt, Hq, k, out, ws, scores_out=sc,
+            aq.aqua_decode_attn(cache.desc, tdev(inp["q"][s], dt), Pt, Hq, k, out, ws, scores_out=sc,
                                 lse_out=lse)
         aq.aqua_h2o_update(cache.desc, sc, lse, Hq, budget, recent, ev)
         torch.cuda.synchronize()
@@ -109,7 +112,7 @@ def test_h2o_steps_match_oracle(fused, G):
         got_ev = ev.cpu().numpy()
         for b in range(B):
             o_ref, ev_ref = O.h2o_decode_step(seqs[b], inp["q"][s, b], inp["k_new"][s, b], inp["v_new"][s, b],
-                                              T0 + s, P64, k, budget, recent, "bf16", m)
+                                              T0 + s, P64, k, budget, recent, kv, m)
             assert list(got_ev[b]) == ev_ref, f"step {s} seq {b}: {list(got_ev[b])} vs {ev_ref}"
             err = rel_err_rows(got_out[b], O.round_bf16(o_ref))
             assert np.max(err) <= 2e-3, (s, b, np.max(err))
