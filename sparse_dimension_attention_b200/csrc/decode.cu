@@ -36,6 +36,7 @@
 #include <math.h>
 
 #include <mutex>
+#include <iterator>
 #include <unordered_map>
 
 #include "aqua_internal.cuh"
@@ -1791,13 +1792,30 @@ size_t decode_workspace_bytes(int n_units, int G, bool projected_values) {
 // Half of a workspace's selection buffers for a call: calls that select flip
 // the workspace's half, so that a step's selection never writes the half the
 // previous step's attention kernel may still be reading; a call that only
-// attends keeps the half.  Kept per workspace address (thread-safe).
+// attends keeps the half.  Kept per workspace address (thread-safe).  The
+// record stays bounded however many workspaces a process uses: once it holds
+// more than kMaxTracked addresses, those not used in the last kMaxTracked / 2
+// calls are dropped (their kernels completed long ago, so they may start again
+// from half 0).
 int workspace_half(const void* ws, bool flip) {
+  constexpr size_t kMaxTracked = 4096;
+  struct Entry {
+    int half;
+    unsigned long long last;   // call count at the latest use
+  };
   static std::mutex mu;
-  static std::unordered_map<const void*, int> halves;
+  static std::unordered_map<const void*, Entry> halves;
+  static unsigned long long calls = 0;
   std::lock_guard<std::mutex> lock(mu);
-  int& h = halves[ws];
-  if (flip) h ^= 1;
+  ++calls;
+  Entry& e = halves[ws];   // a new address starts at half 0
+  e.last = calls;
+  if (flip) e.half ^= 1;
+  const int h = e.half;
+  if (halves.size() > kMaxTracked) {
+    for (auto it = halves.begin(); it != halves.end();)
+      it = (calls - it->second.last >= kMaxTracked / 2) ? halves.erase(it) : std::next(it);
+  }
   return h;
 }
 
