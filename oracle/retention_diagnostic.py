@@ -19,7 +19,6 @@ import json
 import os
 import sys
 
-import numpy as np
 
 _ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if _ROOT not in sys.path:
